@@ -1,0 +1,126 @@
+"""Seeded synthetic inputs for the attention workloads.
+
+This module holds no attention arithmetic: it only draws random tensors and
+names the workload shapes.  It is the one module that both the CUDA-path
+tests/bench and the CPU oracle's callers use.
+
+Recipe (fixed so that every caller sees the same tensors for a seed):
+  * ``torch.Generator(device).manual_seed(seed)``;
+  * ``randn`` in fp32, drawn in the order Q, K, V (shape order below);
+  * Q multiplied by ``q_mult`` (a power of two, so the product is exact);
+  * rounded to bf16 (round-to-nearest-even, torch's ``.to(bfloat16)``).
+  * decode: per-sequence KV lengths ``randint(lmin, lmax + 1)`` drawn after
+    K and V from the same generator; cache positions at or beyond a
+    sequence's length are filled with ``pad_value`` (NaN by default) so that
+    any read of them shows up in the output.
+The CPU and CUDA generators give different streams for the same seed; a test
+draws once and hands the same tensors to both sides.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Dict, Optional
+
+import torch
+
+
+@dataclass(frozen=True)
+class PrefillShape:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Sq: int
+    Skv: int
+    d: int
+    causal: bool
+    q_mult: float
+    seed: int
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / (self.d ** 0.5)
+
+    def flops(self) -> float:
+        """4*B*Hq*Sq*Skv*d, halved for a causal mask (the metric's convention)."""
+        f = 4.0 * self.B * self.Hq * self.Sq * self.Skv * self.d
+        return f / 2.0 if self.causal else f
+
+
+@dataclass(frozen=True)
+class DecodeShape:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Lmin: int
+    Lmax: int
+    d: int
+    seed: int
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / (self.d ** 0.5)
+
+
+# The five workloads of the exact-attention forward path.
+CONFIGS: Dict[str, object] = {
+    "mha_s512_d64": PrefillShape("mha_s512_d64", 1, 4, 4, 512, 512, 64, False, 1.0, 1),
+    "causal_mha_s2048_d128_qx8": PrefillShape(
+        "causal_mha_s2048_d128_qx8", 4, 16, 16, 2048, 2048, 128, True, 8.0, 2),
+    "causal_gqa_s8192_d128": PrefillShape(
+        "causal_gqa_s8192_d128", 2, 32, 8, 8192, 8192, 128, True, 1.0, 3),
+    "causal_gqa_s32768_d128": PrefillShape(
+        "causal_gqa_s32768_d128", 1, 32, 8, 32768, 32768, 128, True, 1.0, 4),
+    "decode_b64_splitkv_d128": DecodeShape(
+        "decode_b64_splitkv_d128", 64, 32, 8, 4096, 16384, 128, 5),
+}
+
+
+def prefill_inputs(B: int, Hq: int, Hkv: int, Sq: int, Skv: int, d: int, seed: int,
+                   q_mult: float = 1.0, device="cpu"):
+    """q [B,Hq,Sq,d], k/v [B,Hkv,Skv,d], bf16, contiguous."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    q = torch.randn((B, Hq, Sq, d), generator=g, device=device, dtype=torch.float32)
+    k = torch.randn((B, Hkv, Skv, d), generator=g, device=device, dtype=torch.float32)
+    v = torch.randn((B, Hkv, Skv, d), generator=g, device=device, dtype=torch.float32)
+    if q_mult != 1.0:
+        q.mul_(q_mult)
+    return (q.to(torch.bfloat16).contiguous(), k.to(torch.bfloat16).contiguous(),
+            v.to(torch.bfloat16).contiguous())
+
+
+def prefill_inputs_for(shape: PrefillShape, device="cpu"):
+    return prefill_inputs(shape.B, shape.Hq, shape.Hkv, shape.Sq, shape.Skv, shape.d,
+                          shape.seed, shape.q_mult, device)
+
+
+def decode_inputs(B: int, Hq: int, Hkv: int, Lmin: int, Lmax: int, d: int, seed: int,
+                  device="cpu", pad_value: Optional[float] = float("nan")):
+    """q [B,Hq,d], k/v caches [B,Hkv,Lmax,d] (bf16), seqlens [B] (int32).
+
+    The cache is drawn in fp32 one sequence at a time, so the peak host memory
+    stays one sequence's worth above the bf16 caches."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    q = torch.randn((B, Hq, d), generator=g, device=device,
+                    dtype=torch.float32).to(torch.bfloat16)
+    kc = torch.empty((B, Hkv, Lmax, d), device=device, dtype=torch.bfloat16)
+    vc = torch.empty((B, Hkv, Lmax, d), device=device, dtype=torch.bfloat16)
+    for cache in (kc, vc):
+        for b in range(B):
+            cache[b].copy_(torch.randn((Hkv, Lmax, d), generator=g, device=device,
+                                       dtype=torch.float32))
+    seqlens = torch.randint(Lmin, Lmax + 1, (B,), generator=g, device=device,
+                            dtype=torch.int64).to(torch.int32)
+    if pad_value is not None:
+        for b, L in enumerate(seqlens.tolist()):
+            kc[b, :, L:, :] = pad_value
+            vc[b, :, L:, :] = pad_value
+    return q.contiguous(), kc.contiguous(), vc.contiguous(), seqlens.contiguous()
+
+
+def decode_inputs_for(shape: DecodeShape, device="cpu", pad_value=float("nan")):
+    return decode_inputs(shape.B, shape.Hq, shape.Hkv, shape.Lmin, shape.Lmax, shape.d,
+                         shape.seed, device, pad_value)

@@ -1,0 +1,176 @@
+"""fp64 CPU attention oracle -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never calls it, and it
+shares no code with the CUDA library: the arithmetic lives in
+``attn_oracle.c`` (plain C, fp64, OpenMP over rows), this module only builds
+that file with gcc and marshals numpy arrays through ctypes.
+
+What it computes (see ``attn_oracle.c`` for the per-function citations):
+the one-shot, materialising softmax attention of "I/O-Aware Kernels", section
+"The Memory Bottleneck", with scores scaled as in "FlashAttention & IO-aware
+attention", section "Code", and LSE = max + ln(sum of exp).
+
+Parity pins (tests/test_oracle_pins.py): closed-form golden cases, an
+independent online-softmax recurrence, invariants, torch fp64 SDPA on small
+shapes, GQA/decode/split reductions.  Every function here is pinned.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "_attn_oracle.so")
+_lib: Optional[ctypes.CDLL] = None
+
+_D = ctypes.POINTER(ctypes.c_double)
+_I32 = ctypes.POINTER(ctypes.c_int32)
+_I64 = ctypes.POINTER(ctypes.c_int64)
+
+
+def build(src: str = _SRC, out: str = _LIB_PATH, force: bool = False) -> str:
+    """Compile the C oracle into a shared object (gcc, -O2, no fast-math)."""
+    if (not force and os.path.exists(out)
+            and os.path.getmtime(out) >= os.path.getmtime(src)):
+        return out
+    tmp = out + ".tmp%d" % os.getpid()
+    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+           "-fno-fast-math", "-ffp-contract=off", src, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
+    return out
+
+
+def load(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load (building first if needed) the oracle library."""
+    global _lib
+    if path is not None:
+        return _bind(ctypes.CDLL(path))
+    if _lib is None:
+        _lib = _bind(ctypes.CDLL(build()))
+    return _lib
+
+
+def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
+    ci = ctypes.c_int
+    lib.oracle_attn_fwd.argtypes = [_D, _D, _D, _D, _D] + [ci] * 7 + [ctypes.c_double]
+    lib.oracle_attn_fwd.restype = ci
+    lib.oracle_attn_rows.argtypes = ([_D, _D, _D, _I64, ctypes.c_int64, _D, _D]
+                                     + [ci] * 7 + [ctypes.c_double])
+    lib.oracle_attn_rows.restype = ci
+    lib.oracle_decode.argtypes = [_D, _D, _D, _I32, _D, _D] + [ci] * 5 + [ctypes.c_double]
+    lib.oracle_decode.restype = ci
+    lib.oracle_split_partials.argtypes = ([_D, _D, _D, _I32, _D, _D] + [ci] * 6
+                                          + [ctypes.c_double])
+    lib.oracle_split_partials.restype = ci
+    lib.oracle_combine.argtypes = [_D, _D, _D, _D] + [ci] * 4
+    lib.oracle_combine.restype = ci
+    lib.oracle_num_threads.argtypes = []
+    lib.oracle_num_threads.restype = ci
+    return lib
+
+
+def _f64(a) -> np.ndarray:
+    """Exact conversion to a contiguous float64 array (bf16 and fp32 values are
+    exactly representable in fp64)."""
+    if hasattr(a, "detach"):  # torch tensor
+        a = a.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _p(a: np.ndarray, t=_D):
+    return a.ctypes.data_as(t)
+
+
+def attn_fwd(q, k, v, causal: bool, scale: float, lib: Optional[ctypes.CDLL] = None):
+    """O [B,Hq,Sq,d] and LSE [B,Hq,Sq] (float64) of softmax(scale*QK^T [+mask]) V.
+
+    q: [B,Hq,Sq,d]; k, v: [B,Hkv,Skv,d]."""
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Sq, d = q.shape
+    _, Hkv, Skv, _ = k.shape
+    o = np.zeros((B, Hq, Sq, d))
+    lse = np.zeros((B, Hq, Sq))
+    rc = lib.oracle_attn_fwd(_p(q), _p(k), _p(v), _p(o), _p(lse), B, Hq, Hkv, Sq,
+                             Skv, d, int(bool(causal)), float(scale))
+    if rc != 0:
+        raise ValueError("oracle_attn_fwd rejected its arguments")
+    return o, lse
+
+
+def attn_rows(q_rows, k, v, rows: Sequence[Sequence[int]], Hq: int, Sq: int,
+              causal: bool, scale: float, lib: Optional[ctypes.CDLL] = None):
+    """Selected output rows.  q_rows[n, d] are the query rows named by
+    rows[n] = (b, h, i); k, v are the full [B,Hkv,Skv,d] key/value tensors."""
+    lib = lib or load()
+    q_rows, k, v = _f64(q_rows), _f64(k), _f64(v)
+    B, Hkv, Skv, d = k.shape
+    idx = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+    n = idx.shape[0]
+    o = np.zeros((n, d))
+    lse = np.zeros((n,))
+    rc = lib.oracle_attn_rows(_p(q_rows), _p(k), _p(v), _p(idx, _I64), n, _p(o),
+                              _p(lse), B, Hq, Hkv, Sq, Skv, d, int(bool(causal)),
+                              float(scale))
+    if rc != 0:
+        raise ValueError("oracle_attn_rows rejected its arguments")
+    return o, lse
+
+
+def decode(q, k_cache, v_cache, seqlens, scale: float, lib: Optional[ctypes.CDLL] = None):
+    """Single-query decode: q [B,Hq,d], caches [B,Hkv,Lmax,d], seqlens [B]."""
+    lib = lib or load()
+    q, kc, vc = _f64(q), _f64(k_cache), _f64(v_cache)
+    sl = np.ascontiguousarray(np.asarray(
+        seqlens.cpu().numpy() if hasattr(seqlens, "cpu") else seqlens, dtype=np.int32))
+    B, Hq, d = q.shape
+    _, Hkv, Lmax, _ = kc.shape
+    o = np.zeros((B, Hq, d))
+    lse = np.zeros((B, Hq))
+    rc = lib.oracle_decode(_p(q), _p(kc), _p(vc), _p(sl, _I32), _p(o), _p(lse), B, Hq,
+                           Hkv, Lmax, d, float(scale))
+    if rc != 0:
+        raise ValueError("oracle_decode rejected its arguments")
+    return o, lse
+
+
+def split_partials(q, k_cache, v_cache, seqlens, num_splits: int, scale: float,
+                   lib: Optional[ctypes.CDLL] = None):
+    """Per-chunk normalised outputs [B,Hq,n,d] and chunk LSEs [B,Hq,n]."""
+    lib = lib or load()
+    q, kc, vc = _f64(q), _f64(k_cache), _f64(v_cache)
+    sl = np.ascontiguousarray(np.asarray(
+        seqlens.cpu().numpy() if hasattr(seqlens, "cpu") else seqlens, dtype=np.int32))
+    B, Hq, d = q.shape
+    _, Hkv, Lmax, _ = kc.shape
+    o = np.zeros((B, Hq, num_splits, d))
+    lse = np.zeros((B, Hq, num_splits))
+    rc = lib.oracle_split_partials(_p(q), _p(kc), _p(vc), _p(sl, _I32), _p(o), _p(lse),
+                                   B, Hq, Hkv, Lmax, d, int(num_splits), float(scale))
+    if rc != 0:
+        raise ValueError("oracle_split_partials rejected its arguments")
+    return o, lse
+
+
+def combine(o_part, lse_part, lib: Optional[ctypes.CDLL] = None):
+    """Merge split partials o_part [B,Hq,n,d], lse_part [B,Hq,n]."""
+    lib = lib or load()
+    op, lp = _f64(o_part), _f64(lse_part)
+    B, Hq, n, d = op.shape
+    o = np.zeros((B, Hq, d))
+    lse = np.zeros((B, Hq))
+    rc = lib.oracle_combine(_p(op), _p(lp), _p(o), _p(lse), B, Hq, n, d)
+    if rc != 0:
+        raise ValueError("oracle_combine rejected its arguments")
+    return o, lse
+
+
+def num_threads(lib: Optional[ctypes.CDLL] = None) -> int:
+    return int((lib or load()).oracle_num_threads())

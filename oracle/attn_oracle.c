@@ -1,0 +1,278 @@
+/*
+ * attn_oracle.c -- plain, slow, fp64 CPU attention.  TEST INFRASTRUCTURE ONLY.
+ *
+ * This file is the correctness oracle for the CUDA library in
+ * io_aware_exact_flashattention_b200/.  Only the test suite, the package's
+ * smoke check and the benchmark's CPU-baseline leg may load it.  It shares no
+ * code, header, table or helper with the CUDA path, and the CUDA path never
+ * calls it.
+ *
+ * What it computes is the textbook ("naive", materialising) attention that the
+ * pages set against FlashAttention:
+ *   - "I/O-Aware Kernels", section "The Memory Bottleneck": scores Q K^T, a
+ *     softmax over each row of the k x k score matrix, then the product with V.
+ *   - "FlashAttention & IO-aware attention", section "Code": the score of a
+ *     query/key pair is their dot product divided by sqrt(d) (here: times the
+ *     caller's `scale`, which the configurations set to 1/sqrt(d)).
+ *   - Same page, section "Direct answer": the streamed (online) softmax is the
+ *     exact one-shot softmax, so the one-shot form below is the definition the
+ *     fused kernel must reproduce up to rounding.
+ *
+ * For every query row the whole score row is materialised in fp64, its maximum
+ * M taken, Z = sum_j exp(s_j - M) formed, and
+ *     LSE = M + ln Z,        O = sum_j exp(s_j - LSE) * v_j.
+ * There is no blocking, no online recurrence and no reordering beyond that.
+ *
+ * Readings of points the pages leave open (the pages never mention a causal
+ * mask or grouped-query head sharing beyond naming GQA):
+ *   - causal: key j is visible to query i when j <= i + (Skv - Sq)
+ *     (bottom-right alignment; equals j <= i when Sq == Skv).  Masked keys are
+ *     excluded exactly.  A row with no visible key has O = 0 and LSE = -inf.
+ *   - GQA: query head h reads key/value head h / (Hq / Hkv).
+ *   - LSE is in natural-log units of the scaled scores.
+ *
+ * Layouts (row-major, contiguous): q/o [B,Hq,Sq,d], k/v [B,Hkv,Skv,d],
+ * lse [B,Hq,Sq].  Decode: q/o [B,Hq,d], caches [B,Hkv,Lmax,d], seqlens [B].
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Keys [0, n_vis) of one head against one query row.  s is scratch of >= n_vis
+ * doubles.  Materialises the full score row (one-shot softmax). */
+static void attn_one_row(const double *q, const double *k, const double *v,
+                         int64_t n_vis, int d, double scale, double *s,
+                         double *o, double *lse)
+{
+    if (n_vis <= 0) {
+        for (int t = 0; t < d; ++t) o[t] = 0.0;
+        *lse = -INFINITY;
+        return;
+    }
+    double m = -INFINITY;
+    for (int64_t j = 0; j < n_vis; ++j) {
+        const double *kj = k + j * (int64_t)d;
+        double acc = 0.0;
+        for (int t = 0; t < d; ++t) acc += q[t] * kj[t];
+        s[j] = scale * acc;
+        if (s[j] > m) m = s[j];
+    }
+    double z = 0.0;
+    for (int64_t j = 0; j < n_vis; ++j) z += exp(s[j] - m);
+    const double l = m + log(z);
+    for (int t = 0; t < d; ++t) o[t] = 0.0;
+    for (int64_t j = 0; j < n_vis; ++j) {
+        const double w = exp(s[j] - l);
+        const double *vj = v + j * (int64_t)d;
+        for (int t = 0; t < d; ++t) o[t] += w * vj[t];
+    }
+    *lse = l;
+}
+
+static int64_t visible_keys(int64_t i, int64_t Sq, int64_t Skv, int causal)
+{
+    if (!causal) return Skv;
+    int64_t n = i + (Skv - Sq) + 1;
+    if (n < 0) n = 0;
+    if (n > Skv) n = Skv;
+    return n;
+}
+
+/* Full forward pass.  Returns 0, or -1 on a bad argument. */
+int oracle_attn_fwd(const double *q, const double *k, const double *v,
+                    double *o, double *lse, int B, int Hq, int Hkv, int Sq,
+                    int Skv, int d, int causal, double scale)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Sq < 0 || Skv < 0 || d <= 0) return -1;
+    if (Hq % Hkv != 0) return -1;
+    const int group = Hq / Hkv;
+    const int64_t rows = (int64_t)B * Hq * Sq;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Skv > 0 ? Skv : 1));
+        if (!s) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t r = 0; r < rows; ++r) {
+                const int64_t i = r % Sq;
+                const int64_t bh = r / Sq;
+                const int64_t h = bh % Hq;
+                const int64_t b = bh / Hq;
+                const int64_t g = h / group;
+                const double *kh = k + ((b * Hkv + g) * (int64_t)Skv) * d;
+                const double *vh = v + ((b * Hkv + g) * (int64_t)Skv) * d;
+                attn_one_row(q + r * d, kh, vh, visible_keys(i, Sq, Skv, causal),
+                             d, scale, s, o + r * d, lse + r);
+            }
+            free(s);
+        }
+    }
+    return err ? -1 : 0;
+}
+
+/* Selected rows of the forward pass.  rows[3*n] holds (b, h, i) triples; the
+ * outputs are o_rows[n, d] and lse_rows[n].  Used to check full-size launches
+ * at sampled outputs. */
+int oracle_attn_rows(const double *q_rows, const double *k, const double *v,
+                     const int64_t *rows, int64_t n, double *o_rows,
+                     double *lse_rows, int B, int Hq, int Hkv, int Sq, int Skv,
+                     int d, int causal, double scale)
+{
+    if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || d <= 0) return -1;
+    const int group = Hq / Hkv;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Skv > 0 ? Skv : 1));
+        if (!s) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < n; ++r) {
+                const int64_t b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+                if (b < 0 || b >= B || h < 0 || h >= Hq || i < 0 || i >= Sq) {
+#pragma omp atomic write
+                    err = 1;
+                    continue;
+                }
+                const int64_t g = h / group;
+                const double *kh = k + ((b * Hkv + g) * (int64_t)Skv) * d;
+                const double *vh = v + ((b * Hkv + g) * (int64_t)Skv) * d;
+                attn_one_row(q_rows + r * d, kh, vh, visible_keys(i, Sq, Skv, causal),
+                             d, scale, s, o_rows + r * d, lse_rows + r);
+            }
+            free(s);
+        }
+    }
+    return err ? -1 : 0;
+}
+
+/* Single-query decode: the forward pass with Sq = 1, no mask, and key count
+ * seqlens[b] (positions >= seqlens[b] of the cache are never read).  This is
+ * the 1 x S score vector of "FlashAttention & IO-aware attention", section
+ * "Direct answer". */
+int oracle_decode(const double *q, const double *kc, const double *vc,
+                  const int32_t *seqlens, double *o, double *lse, int B, int Hq,
+                  int Hkv, int Lmax, int d, double scale)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || Lmax < 0) return -1;
+    for (int b = 0; b < B; ++b)
+        if (seqlens[b] < 0 || seqlens[b] > Lmax) return -1;
+    const int group = Hq / Hkv;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Lmax > 0 ? Lmax : 1));
+        if (!s) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < (int64_t)B * Hq; ++r) {
+                const int64_t b = r / Hq, h = r % Hq, g = h / group;
+                const double *kh = kc + ((b * Hkv + g) * (int64_t)Lmax) * d;
+                const double *vh = vc + ((b * Hkv + g) * (int64_t)Lmax) * d;
+                attn_one_row(q + r * d, kh, vh, seqlens[b], d, scale, s, o + r * d, lse + r);
+            }
+            free(s);
+        }
+    }
+    return err ? -1 : 0;
+}
+
+/* Split-KV partials of the decode step: the KV length of sequence b is cut
+ * into num_splits chunks of ceil(L_b / num_splits) keys; chunk c covers
+ * [c*cs, min(L_b, (c+1)*cs)).  For each chunk the one-shot softmax over that
+ * chunk alone gives a normalised partial output and the chunk's LSE.  An
+ * empty chunk has o = 0 and lse = -inf.  (Splitting the KV length across SMs
+ * is the FlashDecoding idea named in "FlashAttention & IO-aware attention",
+ * sections "Deep dive" and "Interviewer follow-ups".)
+ * Outputs: o_part [B,Hq,num_splits,d], lse_part [B,Hq,num_splits]. */
+int oracle_split_partials(const double *q, const double *kc, const double *vc,
+                          const int32_t *seqlens, double *o_part, double *lse_part,
+                          int B, int Hq, int Hkv, int Lmax, int d, int num_splits,
+                          double scale)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || num_splits < 1) return -1;
+    for (int b = 0; b < B; ++b)
+        if (seqlens[b] < 0 || seqlens[b] > Lmax) return -1;
+    const int group = Hq / Hkv;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Lmax > 0 ? Lmax : 1));
+        if (!s) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < (int64_t)B * Hq * num_splits; ++r) {
+                const int64_t c = r % num_splits;
+                const int64_t bh = r / num_splits;
+                const int64_t b = bh / Hq, h = bh % Hq, g = h / group;
+                const int64_t L = seqlens[b];
+                const int64_t cs = (L + num_splits - 1) / num_splits;
+                int64_t lo = c * cs, hi = lo + cs;
+                if (lo > L) lo = L;
+                if (hi > L) hi = L;
+                const double *kh = kc + ((b * Hkv + g) * (int64_t)Lmax + lo) * d;
+                const double *vh = vc + ((b * Hkv + g) * (int64_t)Lmax + lo) * d;
+                attn_one_row(q + bh * d, kh, vh, hi - lo, d, scale, s,
+                             o_part + r * d, lse_part + r);
+            }
+            free(s);
+        }
+    }
+    return err ? -1 : 0;
+}
+
+/* Merge of split partials.  With M = max_c lse_c the merged statistics are
+ * LSE = M + ln sum_c exp(lse_c - M) and O = sum_c exp(lse_c - LSE) * o_c: the
+ * e^(m - m_new) rescale rule of the online softmax ("FlashAttention &
+ * IO-aware attention", section "Direct answer") applied between chunks.  All
+ * chunks empty gives O = 0, LSE = -inf. */
+int oracle_combine(const double *o_part, const double *lse_part, double *o,
+                   double *lse, int B, int Hq, int num_splits, int d)
+{
+    if (B < 0 || Hq <= 0 || num_splits < 1 || d <= 0) return -1;
+    for (int64_t r = 0; r < (int64_t)B * Hq; ++r) {
+        const double *ls = lse_part + r * num_splits;
+        double m = -INFINITY;
+        for (int c = 0; c < num_splits; ++c)
+            if (ls[c] > m) m = ls[c];
+        double *orow = o + r * d;
+        for (int t = 0; t < d; ++t) orow[t] = 0.0;
+        if (m == -INFINITY) {
+            lse[r] = -INFINITY;
+            continue;
+        }
+        double z = 0.0;
+        for (int c = 0; c < num_splits; ++c) z += exp(ls[c] - m);
+        const double l = m + log(z);
+        for (int c = 0; c < num_splits; ++c) {
+            const double w = exp(ls[c] - l);
+            const double *oc = o_part + (r * num_splits + c) * d;
+            for (int t = 0; t < d; ++t) orow[t] += w * oc[t];
+        }
+        lse[r] = l;
+    }
+    return 0;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

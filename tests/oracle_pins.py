@@ -1,0 +1,354 @@
+"""Checks that pin the fp64 oracle to facts other than itself.
+
+Each ``pin_*`` function takes a loaded oracle library (the real one, or a
+mutant built by tests/test_oracle_mutants.py) and raises AssertionError when the
+oracle disagrees with:
+  * hand-derived closed forms (tests/golden/closed_forms.json);
+  * an independent block-wise online-softmax recurrence written here from the
+    description in "FlashAttention & IO-aware attention", section "Direct
+    answer" (running max m, normaliser l and accumulator O, rescaled by
+    e^(m - m_new) whenever the max grows) -- that page states the streamed
+    result equals the one-shot softmax;
+  * invariants of softmax attention;
+  * torch's fp64 scaled_dot_product_attention (an independent implementation);
+  * reductions: GQA == MHA with repeated K/V, decode == prefill with one query,
+    split + combine == unsplit.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "closed_forms.json")
+
+_MATH_NAMES = {"log": math.log, "exp": math.exp, "inf": math.inf}
+
+
+def _ev(x):
+    """Evaluate a golden expression string ("log(4)", "-inf", "7") with math."""
+    if isinstance(x, (int, float)):
+        return float(x)
+    return float(eval(x, {"__builtins__": {}}, _MATH_NAMES))
+
+
+def _evarr(a):
+    return np.vectorize(_ev, otypes=[np.float64])(np.asarray(a, dtype=object))
+
+
+def _close(got, want, tol, what):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    assert got.shape == want.shape, f"{what}: shape {got.shape} != {want.shape}"
+    both_inf = np.isinf(got) & np.isinf(want) & (np.sign(got) == np.sign(want))
+    with np.errstate(invalid="ignore"):
+        diff = np.where(both_inf, 0.0, np.abs(got - want))
+    diff = np.where(np.isnan(diff), np.inf, diff)
+    err = float(diff.max()) if diff.size else 0.0
+    assert err <= tol, f"{what}: max abs error {err:.3e} > {tol:.1e}"
+
+
+def _rand(shape, rng, scale=1.0):
+    return rng.standard_normal(shape) * scale
+
+
+# --------------------------------------------------------------------------
+# Independent reference algorithms written for the pins
+# --------------------------------------------------------------------------
+
+def online_softmax_attention(q, k, v, causal, scale, block):
+    """Block-wise streaming softmax attention in fp64 (per query row, keys in
+    blocks of `block`, left to right).  Independent of the C oracle."""
+    B, Hq, Sq, d = q.shape
+    _, Hkv, Skv, _ = k.shape
+    grp = Hq // Hkv
+    o = np.zeros_like(q)
+    lse = np.zeros((B, Hq, Sq))
+    for b in range(B):
+        for h in range(Hq):
+            kh, vh = k[b, h // grp], v[b, h // grp]
+            for i in range(Sq):
+                n_vis = Skv if not causal else max(0, min(Skv, i + Skv - Sq + 1))
+                m, l = -math.inf, 0.0
+                acc = np.zeros(d)
+                for j0 in range(0, n_vis, block):
+                    j1 = min(n_vis, j0 + block)
+                    s = scale * (kh[j0:j1] @ q[b, h, i])
+                    m_new = max(m, float(s.max()))
+                    shrink = 0.0 if m == -math.inf else math.exp(m - m_new)
+                    p = np.exp(s - m_new)
+                    l = l * shrink + float(p.sum())
+                    acc = acc * shrink + p @ vh[j0:j1]
+                    m = m_new
+                if n_vis == 0:
+                    o[b, h, i] = 0.0
+                    lse[b, h, i] = -math.inf
+                else:
+                    o[b, h, i] = acc / l
+                    lse[b, h, i] = m + math.log(l)
+    return o, lse
+
+
+def torch_sdpa_fp64(q, k, v, causal, scale):
+    """torch's fp64 CPU scaled_dot_product_attention with K/V repeated per
+    query group, a bottom-right causal boolean mask, and LSE from logsumexp."""
+    tq, tk, tv = (torch.from_numpy(np.ascontiguousarray(x)) for x in (q, k, v))
+    grp = tq.shape[1] // tk.shape[1]
+    tk = tk.repeat_interleave(grp, dim=1)
+    tv = tv.repeat_interleave(grp, dim=1)
+    Sq, Skv = tq.shape[2], tk.shape[2]
+    mask = None
+    if causal:
+        i = torch.arange(Sq).unsqueeze(1)
+        j = torch.arange(Skv).unsqueeze(0)
+        mask = j <= i + (Skv - Sq)
+    o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask,
+                                                         scale=scale)
+    s = (tq @ tk.transpose(-1, -2)) * scale
+    if mask is not None:
+        s = s.masked_fill(~mask, -math.inf)
+    lse = torch.logsumexp(s, dim=-1)
+    return o.numpy(), lse.numpy()
+
+
+# --------------------------------------------------------------------------
+# Pins
+# --------------------------------------------------------------------------
+
+def pin_golden_prefill(lib):
+    cases = json.load(open(GOLDEN))["prefill"]
+    for c in cases:
+        q, k, v = (np.asarray(c[x], dtype=np.float64) for x in ("q", "k", "v"))
+        scale = _ev(c["scale_expr"]) if "scale_expr" in c else float(c["scale"])
+        o, lse = oracle.attn_fwd(q, k, v, c["causal"], scale, lib=lib)
+        _close(o, _evarr(c["o"]), 1e-12, c["name"] + " O")
+        _close(lse, _evarr(c["lse"]), 1e-12, c["name"] + " LSE")
+
+
+def pin_golden_combine(lib):
+    for c in json.load(open(GOLDEN))["combine"]:
+        o, lse = oracle.combine(_evarr(c["o_part"]), _evarr(c["lse_part"]), lib=lib)
+        _close(o, _evarr(c["o"]), 1e-12, c["name"] + " O")
+        _close(lse, _evarr(c["lse"]), 1e-12, c["name"] + " LSE")
+
+
+def pin_online_equals_one_shot(lib):
+    rng = np.random.default_rng(11)
+    shapes = [  # B, Hq, Hkv, Sq, Skv, d, causal
+        (1, 2, 2, 5, 9, 4, False),
+        (2, 4, 2, 7, 7, 3, True),
+        (1, 3, 1, 9, 4, 5, True),   # Sq > Skv: leading rows see no key
+        (1, 2, 1, 3, 11, 2, True),  # Sq < Skv
+    ]
+    for (B, Hq, Hkv, Sq, Skv, d, causal) in shapes:
+        q = _rand((B, Hq, Sq, d), rng, 2.0)
+        k = _rand((B, Hkv, Skv, d), rng)
+        v = _rand((B, Hkv, Skv, d), rng)
+        scale = 1.0 / math.sqrt(d)
+        o, lse = oracle.attn_fwd(q, k, v, causal, scale, lib=lib)
+        for blk in (1, 2, 3, 7, 128):
+            o2, lse2 = online_softmax_attention(q, k, v, causal, scale, blk)
+            _close(o, o2, 1e-12, f"online block={blk} O {B,Hq,Hkv,Sq,Skv,d,causal}")
+            _close(lse, lse2, 1e-12, f"online block={blk} LSE")
+
+
+def pin_invariants(lib):
+    rng = np.random.default_rng(12)
+    B, Hq, Hkv, S, d = 1, 2, 2, 6, 6
+    scale = 0.37
+    q = _rand((B, Hq, S, d), rng)
+    k = _rand((B, Hkv, S, d), rng)
+    # constant V rows -> that row
+    row = _rand((d,), rng)
+    v = np.broadcast_to(row, (B, Hkv, S, d)).copy()
+    for causal in (False, True):
+        o, _ = oracle.attn_fwd(q, k, v, causal, scale, lib=lib)
+        _close(o, np.broadcast_to(row, o.shape), 1e-12, "constant V rows")
+    # identical keys -> mean of V, LSE = s + ln n
+    k1 = np.broadcast_to(_rand((d,), rng), (B, Hkv, S, d)).copy()
+    v = _rand((B, Hkv, S, d), rng)
+    o, lse = oracle.attn_fwd(q, k1, v, False, scale, lib=lib)
+    _close(o, np.broadcast_to(v.mean(axis=2, keepdims=True), o.shape), 1e-12, "identical keys O")
+    s = scale * np.einsum("bhsd,d->bhs", q, k1[0, 0, 0])
+    _close(lse, s + math.log(S), 1e-12, "identical keys LSE")
+    # V = identity (Skv = d): O rows are the probability rows: >= 0, sum to 1
+    eye = np.broadcast_to(np.eye(S), (B, Hkv, S, S)).copy()
+    for causal in (False, True):
+        o, lse = oracle.attn_fwd(q, k, eye, causal, scale, lib=lib)
+        assert (o >= 0).all(), "softmax weights must be non-negative"
+        _close(o.sum(-1), np.ones((B, Hq, S)), 1e-12, "softmax rows sum to 1")
+        # the weights are exp(s - LSE): check against the scores directly
+        sc = scale * np.einsum("bhid,bhjd->bhij", q, k)
+        if causal:
+            sc = np.where(np.tril(np.ones((S, S), bool)), sc, -np.inf)
+        _close(o, np.exp(sc - lse[..., None]), 1e-12, "weights = exp(s - LSE)")
+        if causal:
+            # masked weights are exactly zero
+            assert (o[..., np.triu(np.ones((S, S), bool), 1)] == 0).all()
+    # shifting every key by u: LSE shifts by scale*q.u, O unchanged
+    u = _rand((d,), rng)
+    v = _rand((B, Hkv, S, d), rng)
+    o, lse = oracle.attn_fwd(q, k, v, True, scale, lib=lib)
+    o2, lse2 = oracle.attn_fwd(q, k + u, v, True, scale, lib=lib)
+    _close(o2, o, 1e-12, "key shift O")
+    _close(lse2, lse + scale * (q @ u), 1e-12, "key shift LSE")
+    # jointly permuting keys and values (no mask) leaves the result unchanged
+    perm = rng.permutation(S)
+    o, lse = oracle.attn_fwd(q, k, v, False, scale, lib=lib)
+    o2, lse2 = oracle.attn_fwd(q, k[:, :, perm], v[:, :, perm], False, scale, lib=lib)
+    _close(o2, o, 1e-12, "permutation O")
+    _close(lse2, lse, 1e-12, "permutation LSE")
+    # causal first row sees key 0 only: O = v_0, LSE = its score
+    o, lse = oracle.attn_fwd(q, k, v, True, scale, lib=lib)
+    _close(o[:, :, 0], v[:, :, 0], 1e-12, "causal row 0 O")
+    _close(lse[:, :, 0], scale * np.einsum("bhd,bhd->bh", q[:, :, 0], k[:, :, 0]), 1e-12,
+           "causal row 0 LSE")
+
+
+def pin_large_logits(lib):
+    """Scores of order 1e3..1e4 (Q x 1024): no overflow, and the softmax is
+    one-hot on the arg-max key (the gaps between scores are >> 40)."""
+    rng = np.random.default_rng(13)
+    B, H, S, d = 1, 2, 16, 8
+    q = np.round(_rand((B, H, S, d), rng) * 4) * 1024.0
+    k = np.round(_rand((B, H, S, d), rng) * 4)
+    v = _rand((B, H, S, d), rng)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = oracle.attn_fwd(q, k, v, False, scale, lib=lib)
+    assert np.isfinite(o).all() and np.isfinite(lse).all(), "overflow at large logits"
+    s = scale * np.einsum("bhid,bhjd->bhij", q, k)
+    srt = np.sort(s, axis=-1)
+    gap = srt[..., -1] - srt[..., -2]
+    top = s.argmax(-1)
+    one_hot = np.take_along_axis(v, top[..., None], axis=2)
+    ok = gap > 50.0  # exp(-50) ~ 2e-22: below fp64 resolution of O
+    assert ok.any(), "test case lost its large gaps"
+    _close(np.where(ok[..., None], o, 0), np.where(ok[..., None], one_hot, 0), 1e-12,
+           "one-hot limit O")
+    _close(np.where(ok, lse, 0), np.where(ok, srt[..., -1], 0), 1e-9, "one-hot limit LSE")
+
+
+def pin_torch_sdpa(lib):
+    rng = np.random.default_rng(14)
+    shapes = [  # B, Hq, Hkv, Sq, Skv, d, causal
+        (2, 4, 4, 33, 33, 16, False),
+        (2, 4, 4, 33, 33, 16, True),
+        (1, 8, 2, 20, 20, 8, True),
+        (1, 4, 1, 7, 19, 8, True),
+        (1, 4, 2, 19, 7, 8, True),
+        (1, 2, 2, 12, 40, 32, False),
+    ]
+    for (B, Hq, Hkv, Sq, Skv, d, causal) in shapes:
+        q = _rand((B, Hq, Sq, d), rng, 3.0)
+        k = _rand((B, Hkv, Skv, d), rng)
+        v = _rand((B, Hkv, Skv, d), rng)
+        scale = 1.0 / math.sqrt(d)
+        o, lse = oracle.attn_fwd(q, k, v, causal, scale, lib=lib)
+        o2, lse2 = torch_sdpa_fp64(q, k, v, causal, scale)
+        # torch returns NaN for rows with no visible key; the oracle's reading
+        # is O = 0, LSE = -inf for them.
+        empty = np.isneginf(lse2)
+        o2 = np.where(empty[..., None], 0.0, o2)
+        _close(o, o2, 1e-12, f"sdpa O {B,Hq,Hkv,Sq,Skv,d,causal}")
+        _close(lse, lse2, 1e-12, f"sdpa LSE {B,Hq,Hkv,Sq,Skv,d,causal}")
+
+
+def pin_rows_match_full(lib):
+    rng = np.random.default_rng(15)
+    B, Hq, Hkv, Sq, Skv, d = 2, 4, 2, 13, 17, 8
+    q = _rand((B, Hq, Sq, d), rng)
+    k = _rand((B, Hkv, Skv, d), rng)
+    v = _rand((B, Hkv, Skv, d), rng)
+    for causal in (False, True):
+        o, lse = oracle.attn_fwd(q, k, v, causal, 0.3, lib=lib)
+        rows = [(b, h, i) for b in range(B) for h in range(Hq) for i in (0, 5, Sq - 1)]
+        qr = np.stack([q[b, h, i] for (b, h, i) in rows])
+        o2, lse2 = oracle.attn_rows(qr, k, v, rows, Hq, Sq, causal, 0.3, lib=lib)
+        _close(o2, np.stack([o[r] for r in rows]), 0.0, "rows O")
+        _close(lse2, np.array([lse[r] for r in rows]), 0.0, "rows LSE")
+
+
+def pin_gqa_equals_repeated_mha(lib):
+    rng = np.random.default_rng(16)
+    B, Hq, Hkv, S, d = 2, 8, 2, 9, 4
+    q = _rand((B, Hq, S, d), rng)
+    k = _rand((B, Hkv, S, d), rng)
+    v = _rand((B, Hkv, S, d), rng)
+    rep_k = np.repeat(k, Hq // Hkv, axis=1)
+    rep_v = np.repeat(v, Hq // Hkv, axis=1)
+    for causal in (False, True):
+        o, lse = oracle.attn_fwd(q, k, v, causal, 0.5, lib=lib)
+        o2, lse2 = oracle.attn_fwd(q, rep_k, rep_v, causal, 0.5, lib=lib)
+        _close(o, o2, 0.0, "GQA O")
+        _close(lse, lse2, 0.0, "GQA LSE")
+        # and each query head against its own explicit kv head
+        for h in range(Hq):
+            o3, _ = oracle.attn_fwd(q[:, h:h + 1], k[:, h // (Hq // Hkv)][:, None],
+                                    v[:, h // (Hq // Hkv)][:, None], causal, 0.5, lib=lib)
+            _close(o[:, h:h + 1], o3, 0.0, f"GQA head {h}")
+
+
+def _decode_case(rng, B=3, Hq=4, Hkv=2, Lmax=23, d=8, lens=(23, 1, 10)):
+    q = _rand((B, Hq, d), rng)
+    kc = _rand((B, Hkv, Lmax, d), rng)
+    vc = _rand((B, Hkv, Lmax, d), rng)
+    sl = np.asarray(lens, dtype=np.int32)
+    return q, kc, vc, sl
+
+
+def pin_decode_equals_prefill(lib):
+    rng = np.random.default_rng(17)
+    q, kc, vc, sl = _decode_case(rng)
+    # cache positions beyond a sequence's length must never be read
+    for b, L in enumerate(sl):
+        kc[b, :, L:] = np.nan
+        vc[b, :, L:] = np.nan
+    o, lse = oracle.decode(q, kc, vc, sl, 0.25, lib=lib)
+    for b, L in enumerate(sl):
+        o2, lse2 = oracle.attn_fwd(q[b:b + 1, :, None], kc[b:b + 1, :, :L], vc[b:b + 1, :, :L],
+                                   False, 0.25, lib=lib)
+        _close(o[b], o2[0, :, 0], 0.0, f"decode O b={b}")
+        _close(lse[b], lse2[0, :, 0], 0.0, f"decode LSE b={b}")
+
+
+def pin_split_combine_equals_unsplit(lib):
+    rng = np.random.default_rng(18)
+    q, kc, vc, sl = _decode_case(rng, lens=(23, 1, 10))
+    o, lse = oracle.decode(q, kc, vc, sl, 0.25, lib=lib)
+    for n in (1, 2, 3, 5, 7, 30):  # 30 > every length: empty chunks occur
+        op, lp = oracle.split_partials(q, kc, vc, sl, n, 0.25, lib=lib)
+        o2, lse2 = oracle.combine(op, lp, lib=lib)
+        _close(o2, o, 1e-12, f"split {n} O")
+        _close(lse2, lse, 1e-12, f"split {n} LSE")
+        # chunk c of sequence b covers [c*cs, min(L,(c+1)*cs)), cs = ceil(L/n)
+        for b, L in enumerate(sl):
+            cs = -(-int(L) // n)
+            for c in range(n):
+                lo, hi = min(L, c * cs), min(L, (c + 1) * cs)
+                if hi <= lo:
+                    assert np.isneginf(lp[b, :, c]).all() and (op[b, :, c] == 0).all(), \
+                        "empty chunk must give lse=-inf, o=0"
+                else:
+                    o3, l3 = oracle.attn_fwd(q[b:b + 1, :, None], kc[b:b + 1, :, lo:hi],
+                                             vc[b:b + 1, :, lo:hi], False, 0.25, lib=lib)
+                    _close(op[b, :, c], o3[0, :, 0], 1e-12, f"chunk {b},{c} O")
+                    _close(lp[b, :, c], l3[0, :, 0], 1e-12, f"chunk {b},{c} LSE")
+
+
+ALL_PINS = [
+    pin_golden_prefill,
+    pin_golden_combine,
+    pin_online_equals_one_shot,
+    pin_invariants,
+    pin_large_logits,
+    pin_torch_sdpa,
+    pin_rows_match_full,
+    pin_gqa_equals_repeated_mha,
+    pin_decode_equals_prefill,
+    pin_split_combine_equals_unsplit,
+]

@@ -1,0 +1,51 @@
+"""Plant plausible mistakes in a copy of the oracle's C source and check that
+the pins catch every one (CPU only).  The real oracle is never modified."""
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+import oracle
+from oracle_pins import ALL_PINS
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "attn_oracle.c")
+
+# (name, exact text in attn_oracle.c, replacement)
+MUTANTS = [
+    ("dropped_scale", "s[j] = scale * acc;", "s[j] = acc;"),
+    ("exp_sign_flipped", "z += exp(s[j] - m);", "z += exp(m - s[j]);"),
+    ("lse_missing_max", "const double l = m + log(z);\n    for (int t = 0; t < d; ++t) o[t] = 0.0;",
+     "const double l = log(z);\n    for (int t = 0; t < d; ++t) o[t] = 0.0;"),
+    ("weights_not_normalised", "const double w = exp(s[j] - l);", "const double w = exp(s[j] - m);"),
+    ("key_index_frozen", "const double *kj = k + j * (int64_t)d;", "const double *kj = k;"),
+    ("value_from_key", "const double *vj = v + j * (int64_t)d;", "const double *vj = k + j * (int64_t)d;"),
+    ("causal_off_by_one", "int64_t n = i + (Skv - Sq) + 1;", "int64_t n = i + (Skv - Sq);"),
+    ("causal_top_left", "int64_t n = i + (Skv - Sq) + 1;", "int64_t n = i + 1;"),
+    ("gqa_modulo_map", "const int64_t g = h / group;\n                const double *kh = k + ((b * Hkv + g) * (int64_t)Skv) * d;\n                const double *vh = v + ((b * Hkv + g) * (int64_t)Skv) * d;\n                attn_one_row(q + r * d",
+     "const int64_t g = h % Hkv;\n                const double *kh = k + ((b * Hkv + g) * (int64_t)Skv) * d;\n                const double *vh = v + ((b * Hkv + g) * (int64_t)Skv) * d;\n                attn_one_row(q + r * d"),
+    ("split_chunk_floor", "const int64_t cs = (L + num_splits - 1) / num_splits;",
+     "const int64_t cs = L / num_splits + 1;"),
+    ("combine_weight_uses_max", "const double w = exp(ls[c] - l);", "const double w = exp(ls[c] - m);"),
+    ("combine_lse_missing_max", "const double l = m + log(z);\n        for (int c = 0;",
+     "const double l = log(z);\n        for (int c = 0;"),
+    ("decode_reads_lmax", "attn_one_row(q + r * d, kh, vh, seqlens[b],", "attn_one_row(q + r * d, kh, vh, Lmax,"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_planted_mistake(name, old, new, tmp_path):
+    text = open(SRC).read()
+    assert text.count(old) == 1, f"mutation site for {name} not unique/absent"
+    src = tmp_path / "mutant.c"
+    src.write_text(text.replace(old, new))
+    so = str(tmp_path / "mutant.so")
+    oracle.build(str(src), so, force=True)
+    lib = oracle.load(so)
+    caught = []
+    for pin in ALL_PINS:
+        try:
+            pin(lib)
+        except (AssertionError, ValueError) as e:
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught the planted mistake {name}"
