@@ -1,0 +1,156 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention library libfa.so.
+ *
+ * The library computes exact softmax attention without writing the score
+ * matrix to HBM: query blocks stay on chip while key/value blocks stream past
+ * them, and an online softmax keeps a running max and sum per row, rescaling
+ * the partial output whenever the max grows ("I/O-Aware Kernels", section
+ * "FlashAttention"; "FlashAttention & IO-aware attention", section "Direct
+ * answer").  Single-query decode splits the key/value length across SMs and
+ * merges the pieces by their log-sum-exp ("FlashAttention & IO-aware
+ * attention", sections "Deep dive" and "Interviewer follow-ups").
+ *
+ * Conventions shared by every entry point
+ *  - Pointers are DEVICE pointers of the current CUDA device, unless stated.
+ *    The caller owns every buffer; the library allocates no device memory and
+ *    keeps no per-call state.  All tensors are contiguous, row-major.
+ *  - bf16 is IEEE-754 binary16-bfloat (the bit pattern of __nv_bfloat16).
+ *  - Calls only enqueue work on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and return without synchronising.  A fault during
+ *    execution surfaces at the caller's next synchronisation.
+ *  - Errors are returned, never printed and never trapped.  Argument checks
+ *    run before any CUDA call; a call that fails them launches nothing.
+ *  - Unsupported head sizes are rejected with FA_ERR_UNSUPPORTED: there is no
+ *    slower fallback path ("FlashAttention & IO-aware attention", section
+ *    "Interviewer follow-ups", warns that a silent fallback to a materialising
+ *    kernel is why a "flash" path can fail to be fast).
+ *  - Thread safety: calls hold no shared mutable state apart from the
+ *    one-time lookup of the driver's tensor-map encoder, which is guarded.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque stream handle; pass a cudaStream_t. */
+typedef struct CUstream_st *fa_stream_t;
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,     /* null pointer, negative or inconsistent size */
+    FA_ERR_UNSUPPORTED = 2,     /* valid but not implemented (e.g. head size) */
+    FA_ERR_ALIGNMENT = 3,       /* a pointer is not 16-byte aligned */
+    FA_ERR_CUDA = 4,            /* a CUDA runtime/driver call or launch failed */
+    FA_ERR_DEVICE_TIMEOUT = 5   /* a kernel gave up a bounded wait (see below) */
+} fa_status;
+
+/*
+ * fa_fwd -- fused exact attention forward (prefill).
+ *
+ *   O[b,h,i,:] = sum_j softmax_j(scale * q[b,h,i,:] . k[b,g,j,:]) * v[b,g,j,:]
+ *   LSE[b,h,i] = ln sum_j exp(scale * q[b,h,i,:] . k[b,g,j,:])
+ *
+ * over the visible keys j, with g = h / (Hq / Hkv) (grouped-query heads share
+ * a key/value head; MHA when Hq == Hkv).  The naive form of this computation
+ * is the one "I/O-Aware Kernels", section "The Memory Bottleneck", describes;
+ * this call never materialises the score matrix.
+ *
+ *   q    [B, Hq,  Sq,  d] bf16      o   [B, Hq, Sq, d] bf16 (written)
+ *   k, v [B, Hkv, Skv, d] bf16      lse [B, Hq, Sq]    fp32 (written, natural log)
+ *   causal != 0: key j is visible to query i iff j <= i + (Skv - Sq)
+ *       (bottom-right alignment).  A query row that sees no key gets
+ *       O = 0 and LSE = -inf.
+ *   scale: multiplies q.k before the softmax (normally 1/sqrt(d)).
+ *
+ * Supported: d in {64, 128}; Hq % Hkv == 0; B, Hq, Hkv >= 1; Sq, Skv >= 0
+ * (Sq == 0 or B == 0 is a no-op).  All five pointers 16-byte aligned.
+ * Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT before any
+ * CUDA call; FA_ERR_CUDA if the tensor-map encoder or the launch fails.
+ */
+fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                 int B, int Hq, int Hkv, int Sq, int Skv, int d, int causal,
+                 float scale, fa_stream_t stream);
+
+/*
+ * fa_decode_splitkv -- first half of single-query decode (Sq = 1, no mask).
+ *
+ * The key/value length L_b = seqlens_k[b] of sequence b is cut into
+ * num_splits chunks of cs = ceil(L_b / num_splits) keys; chunk c covers keys
+ * [c*cs, min(L_b, (c+1)*cs)).  For every (b, query head h, chunk c) the call
+ * writes the chunk's normalised partial output and its log-sum-exp:
+ *
+ *   o_partial[b,h,c,:] = softmax over the chunk's keys, times their values
+ *   lse_partial[b,h,c] = ln sum over the chunk's keys of exp(scale * q.k)
+ *
+ * An empty chunk writes o_partial = 0 and lse_partial = -inf.  Cache
+ * positions >= L_b are never read.
+ *
+ *   q            [B, Hq, d]           bf16
+ *   k_cache,
+ *   v_cache      [B, Hkv, Lmax, d]    bf16
+ *   seqlens_k    [B]                  int32, device (4-byte aligned), 0 <= L_b <= Lmax
+ *                                     (values outside that range are clamped)
+ *   o_partial    [B, Hq, num_splits, d] fp32 (written; caller-owned scratch)
+ *   lse_partial  [B, Hq, num_splits]    fp32 (written; caller-owned scratch)
+ *
+ * Supported: d in {64, 128}; Hq / Hkv in {1, 2, 4, 8}; 1 <= num_splits <= 256.
+ */
+fa_status fa_decode_splitkv(const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *seqlens_k, float *o_partial,
+                            float *lse_partial, int B, int Hq, int Hkv, int Lmax,
+                            int d, int num_splits, float scale, fa_stream_t stream);
+
+/*
+ * fa_combine -- second half of decode: merge split partials by their LSE.
+ *
+ * With M = max_c lse_partial[b,h,c]:
+ *   lse[b,h] = M + ln sum_c exp(lse_partial[b,h,c] - M)
+ *   o[b,h,:] = sum_c exp(lse_partial[b,h,c] - lse[b,h]) * o_partial[b,h,c,:]
+ * which is the online softmax's e^(m - m_new) rescale applied between chunks
+ * ("FlashAttention & IO-aware attention", section "Direct answer").  All
+ * chunks empty gives o = 0, lse = -inf.
+ *
+ *   o_partial [B, Hq, num_splits, d] fp32,  lse_partial [B, Hq, num_splits] fp32
+ *   o         [B, Hq, d] bf16 (written),    lse [B, Hq] fp32 (written)
+ *
+ * Supported: d in {64, 128}; 1 <= num_splits <= 256.
+ */
+fa_status fa_combine(const float *o_partial, const float *lse_partial, void *o,
+                     float *lse, int B, int Hq, int num_splits, int d,
+                     fa_stream_t stream);
+
+/*
+ * Host-only helper: a split count for fa_decode_splitkv that gives the GPU's
+ * num_sms SMs enough independent chunks.  Never fails; returns >= 1.
+ */
+int fa_decode_default_splits(int B, int Hkv, int Lmax, int num_sms);
+
+/* Host-only: a static, human-readable name for a status code. */
+const char *fa_status_string(fa_status s);
+
+/*
+ * Reads and clears the device status word of the current device.  Every
+ * wait inside the kernels (on an mbarrier) is bounded in time; a kernel whose
+ * wait runs out records FA_ERR_DEVICE_TIMEOUT there, drains its own copies,
+ * frees its tensor memory and returns instead of hanging.  Synchronises the
+ * device.  Returns FA_OK when nothing was recorded.
+ */
+fa_status fa_get_device_status(void);
+
+/*
+ * Test hook for the bounded waits: launches one CTA that waits on an
+ * mbarrier nothing will complete, with a time limit of limit_us
+ * microseconds, then returns.  The wait must run out, so a following
+ * fa_get_device_status() reports FA_ERR_DEVICE_TIMEOUT.  Enqueued on stream.
+ */
+fa_status fa_debug_timeout_probe(unsigned int limit_us, fa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

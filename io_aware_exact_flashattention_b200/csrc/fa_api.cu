@@ -1,0 +1,277 @@
+// fa_api.cu -- the C ABI of libfa.so (declared in include/fa.h): argument
+// checks, TMA tensor-map encoding and kernel launches.  Every kernel of the
+// library lives in this one translation unit.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include "fa.h"
+#include "sm100.cuh"
+#include "prefill_sm100.cuh"
+#include "decode_sm100.cuh"
+
+namespace {
+
+constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s per mbarrier wait
+constexpr int kMaxDevices = 64;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// --- driver entry point for the tensor-map encoder (no link to libcuda) ----
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+// [planes, rows, d] bf16 tensor as a 3-D map with 64 x 128 x 1 boxes, 128B
+// swizzle; rows beyond `rows` read as zeros.
+bool encode_bhsd(CUtensorMap* map, const void* base, int d, int rows, long long planes) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t r = static_cast<cuuint64_t>(rows > 0 ? rows : 1);
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), r, static_cast<cuuint64_t>(planes)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, r * static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// One-time per-device opt-in to the prefill kernels' dynamic shared memory.
+std::once_flag g_attr_once[kMaxDevices];
+cudaError_t g_attr_err[kMaxDevices];
+
+cudaError_t prepare_prefill(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::call_once(g_attr_once[dev], [dev] {
+    cudaError_t e = cudaFuncSetAttribute(fa::fa_prefill_kernel<64>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         fa::PrefillLayout<64>::kBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fa::fa_prefill_kernel<128>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::PrefillLayout<128>::kBytes);
+    g_attr_err[dev] = e;
+  });
+  return g_attr_err[dev];
+}
+
+template <int D>
+fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int Hq, int Hkv, int Sq, int Skv, int causal, float scale,
+                         cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  if (!encode_bhsd(&tq, q, D, Sq, static_cast<long long>(B) * Hq) ||
+      !encode_bhsd(&tk, k, D, Skv, static_cast<long long>(B) * Hkv) ||
+      !encode_bhsd(&tv, v, D, Skv, static_cast<long long>(B) * Hkv))
+    return FA_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (prepare_prefill(dev) != cudaSuccess) return FA_ERR_CUDA;
+
+  fa::PrefillParams p;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Sq = Sq;
+  p.Skv = Skv;
+  p.group = Hq / Hkv;
+  p.causal = causal ? 1 : 0;
+  const int q_tiles = (Sq + fa::kBM - 1) / fa::kBM;
+  p.n_qpairs = (q_tiles + 1) / 2;
+  p.n_kv_tiles = (Skv + fa::kBN - 1) / fa::kBN;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_limit_ns = kWaitLimitNs;
+  const long long grid = static_cast<long long>(p.n_qpairs) * B * Hq;
+  fa::fa_prefill_kernel<D><<<static_cast<unsigned>(grid), fa::kPrefillThreads,
+                             fa::PrefillLayout<D>::kBytes, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D, int G>
+void launch_decode(const void* q, const void* kc, const void* vc, const int32_t* seqlens,
+                   float* o_part, float* lse_part, int B, int Hq, int Hkv, int Lmax,
+                   int num_splits, float scale, cudaStream_t stream) {
+  dim3 grid(num_splits, Hkv, B);
+  fa::fa_decode_split_kernel<D, G><<<grid, fa::kDecodeThreads, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(kc),
+      static_cast<const __nv_bfloat16*>(vc), seqlens, o_part, lse_part, Hq, Hkv, Lmax,
+      num_splits, scale * 1.4426950408889634f);
+}
+
+template <int D>
+bool dispatch_decode_group(int G, const void* q, const void* kc, const void* vc,
+                           const int32_t* seqlens, float* o_part, float* lse_part, int B, int Hq,
+                           int Hkv, int Lmax, int num_splits, float scale, cudaStream_t stream) {
+  switch (G) {
+    case 1: launch_decode<D, 1>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, stream); return true;
+    case 2: launch_decode<D, 2>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, stream); return true;
+    case 4: launch_decode<D, 4>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, stream); return true;
+    case 8: launch_decode<D, 8>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, stream); return true;
+    default: return false;
+  }
+}
+
+__global__ void timeout_probe_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t b = fa::smem_addr(&bar);
+  if (threadIdx.x == 0) {
+    fa::mbar_init(b, 1);
+    abort_flag = 0;
+    fa::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // Nothing ever arrives on this barrier: the bounded wait must give up.
+    fa::mbar_wait(b, 0u, &abort_flag, limit_ns);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                 int Hkv, int Sq, int Skv, int d, int causal, float scale, fa_stream_t stream) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || Sq < 0 || Skv < 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || Sq == 0) return FA_OK;  // nothing to compute
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_ALIGNMENT;
+  const long long q_tiles = (static_cast<long long>(Sq) + fa::kBM - 1) / fa::kBM;
+  const long long grid = (q_tiles + 1) / 2 * B * static_cast<long long>(Hq);
+  if (grid > 0x7fffffffLL || static_cast<long long>(B) * Hq > 0x7fffffffLL ||
+      static_cast<long long>(B) * Hkv > 0x7fffffffLL)
+    return FA_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_prefill<64>(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, causal, scale, s)
+                 : launch_prefill<128>(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, causal, scale, s);
+}
+
+fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* seqlens_k, float* o_partial, float* lse_partial, int B,
+                            int Hq, int Hkv, int Lmax, int d, int num_splits, float scale,
+                            fa_stream_t stream) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || Lmax < 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (num_splits < 1 || num_splits > 256) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
+  if (B == 0) return FA_OK;
+  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || seqlens_k == nullptr ||
+      o_partial == nullptr || lse_partial == nullptr)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (reinterpret_cast<uintptr_t>(seqlens_k) & 3u) != 0 ||
+      !aligned16(o_partial) || !aligned16(lse_partial))
+    return FA_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool ok = d == 64 ? dispatch_decode_group<64>(G, q, k_cache, v_cache, seqlens_k, o_partial,
+                                                      lse_partial, B, Hq, Hkv, Lmax, num_splits,
+                                                      scale, s)
+                          : dispatch_decode_group<128>(G, q, k_cache, v_cache, seqlens_k,
+                                                       o_partial, lse_partial, B, Hq, Hkv, Lmax,
+                                                       num_splits, scale, s);
+  if (!ok) return FA_ERR_UNSUPPORTED;
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_combine(const float* o_partial, const float* lse_partial, void* o, float* lse, int B,
+                     int Hq, int num_splits, int d, fa_stream_t stream) {
+  if (B < 0 || Hq < 1) return FA_ERR_INVALID_ARG;
+  if (num_splits < 1 || num_splits > 256) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (B == 0) return FA_OK;
+  if (o_partial == nullptr || lse_partial == nullptr || o == nullptr || lse == nullptr)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned16(o_partial) || !aligned16(lse_partial) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_ALIGNMENT;
+  const long long rows = static_cast<long long>(B) * Hq;
+  if (rows > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  const unsigned blocks = static_cast<unsigned>((rows + 3) / 4);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64)
+    fa::fa_combine_kernel<64><<<blocks, 128, 0, s>>>(o_partial, lse_partial,
+                                                     static_cast<__nv_bfloat16*>(o), lse,
+                                                     static_cast<int>(rows), num_splits);
+  else
+    fa::fa_combine_kernel<128><<<blocks, 128, 0, s>>>(o_partial, lse_partial,
+                                                      static_cast<__nv_bfloat16*>(o), lse,
+                                                      static_cast<int>(rows), num_splits);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_decode_default_splits(int B, int Hkv, int Lmax, int num_sms) {
+  if (B < 1 || Hkv < 1 || Lmax < 1) return 1;
+  if (num_sms < 1) num_sms = 1;
+  // About 1024 keys per chunk, and at least 8 CTAs per SM overall.
+  long long n = (Lmax + 1023) / 1024;
+  const long long units = static_cast<long long>(B) * Hkv;
+  const long long want = (8LL * num_sms + units - 1) / units;
+  if (n < want) n = want;
+  const long long max_useful = (Lmax + 63) / 64;  // keep chunks >= 64 keys
+  if (n > max_useful) n = max_useful;
+  if (n < 1) n = 1;
+  if (n > 256) n = 256;
+  return static_cast<int>(n);
+}
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: null pointer or bad size";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: shape or head size not implemented";
+    case FA_ERR_ALIGNMENT: return "FA_ERR_ALIGNMENT: pointer not 16-byte aligned";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA call or kernel launch failed";
+    case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT: a kernel gave up a bounded wait";
+  }
+  return "unknown fa_status";
+}
+
+fa_status fa_get_device_status(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, fa::g_device_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(fa::g_device_status, &zero, sizeof(int)) != cudaSuccess)
+      return FA_ERR_CUDA;
+  }
+  return static_cast<fa_status>(v);
+}
+
+fa_status fa_debug_timeout_probe(unsigned int limit_us, fa_stream_t stream) {
+  if (limit_us == 0 || limit_us > 10000000u) return FA_ERR_INVALID_ARG;
+  timeout_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<unsigned long long>(limit_us) * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,432 @@
+// prefill_sm100.cuh -- fused exact-attention forward for sm_100a.
+//
+// One CTA owns two 128-row query tiles of one (batch, query head) and streams
+// the key/value tiles of that head's key/value head past them, so the score
+// matrix never leaves the SM ("I/O-Aware Kernels", section "FlashAttention":
+// query blocks stay resident while K and V blocks stream through; "Tracing
+// Tiled QKV Data Movement in FlashAttention's Memory Hierarchy", section 2,
+// tiling plus online softmax).  The loop order is query-stationary: the
+// output tile is accumulated on chip and written to HBM once.
+//
+// Roles (320 threads):
+//   warps 0-3  softmax warpgroup for query tile 0 (thread = row = TMEM lane)
+//   warps 4-7  softmax warpgroup for query tile 1
+//   warp  8    TMA producer: Q tiles once, then K_j, V_j into a smem ring
+//   warp  9    MMA issuer: S_w = Q_w K_j^T and O_w += P_w V_j on tcgen05
+// Tensor memory (512 columns x 128 lanes x 32 bit):
+//   [0,128)   S_0 (fp32 scores); P_0 (bf16) overwrites its first 64 columns
+//   [128,256) S_1 / P_1
+//   [256, 256+D) O_0 accumulator, then O_1
+// Online softmax ("FlashAttention & IO-aware attention", section "Direct
+// answer"): each row keeps a running max m and sum l; when the max grows the
+// accumulated l and O are multiplied by e^(m - m_new).  Here the reference max
+// only moves when it grows by more than 2^8 in the exponent, so the rescale
+// of O is rare; the result is unchanged because the final O / l and LSE use
+// the same reference max.  Exponentials are 2^x on scores pre-multiplied by
+// scale*log2(e).
+#pragma once
+
+#include <climits>
+#include <cuda.h>
+#include "sm100.cuh"
+
+namespace fa {
+
+constexpr int kBM = 128;       // query rows per tile (= TMEM lanes)
+constexpr int kBN = 128;       // keys per key/value tile
+constexpr int kPrefillThreads = 320;
+constexpr int kSwzBytes = 128 * 128;  // one 128-row x 64-element bf16 box, 128B swizzled
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+struct PrefillParams {
+  __nv_bfloat16* o;
+  float* lse;
+  int B, Hq, Hkv, Sq, Skv, group;
+  int causal;
+  int n_qpairs;    // ceil(ceil(Sq / 128) / 2)
+  int n_kv_tiles;  // ceil(Skv / 128)
+  float scale;     // natural units
+  float scale_log2;
+  unsigned long long wait_limit_ns;
+};
+
+template <int D>
+struct PrefillLayout {
+  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kTileBytes = kBM * D * 2;
+  static constexpr int kQOff = 0;
+  static constexpr int kRingOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
+  // q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], mma_done
+  static constexpr int kBarQ = 0;
+  static constexpr int kBarKvFull = 1;
+  static constexpr int kBarKvEmpty = 1 + kStages;
+  static constexpr int kBarSFull = 1 + 2 * kStages;
+  static constexpr int kBarPFull = kBarSFull + 2;
+  static constexpr int kBarOFull = kBarPFull + 2;
+  static constexpr int kBarDone = kBarOFull + 2;
+  static constexpr int kNumBars = kBarDone + 1;
+  static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
+  static constexpr int kAbortOff = kTmemSlotOff + 4;
+  static constexpr int kBytes = kAbortOff + 4 + 1024;  // + slack for 1024-byte alignment
+};
+
+// Number of key/value tiles query tile starting at row r0 must visit.
+__device__ __forceinline__ int prefill_tiles_for(const PrefillParams& p, int r0) {
+  if (r0 >= p.Sq || p.Skv <= 0) return 0;
+  if (!p.causal) return p.n_kv_tiles;
+  const int last_row = min(r0 + kBM - 1, p.Sq - 1);
+  const long long last_key = static_cast<long long>(last_row) + (p.Skv - p.Sq);
+  if (last_key < 0) return 0;
+  return min(p.n_kv_tiles, static_cast<int>(last_key / kBN) + 1);
+}
+
+// ---------------------------------------------------------------------------
+// Softmax warpgroup: one thread per query row.
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t tmem,
+                                                uint32_t bar_s, uint32_t bar_p, uint32_t bar_o,
+                                                int w, int n_tiles, int q_row0, int b, int h,
+                                                volatile int* abort_flag) {
+  const int warp_in_wg = (threadIdx.x >> 5) & 3;
+  const int row_in_tile = warp_in_wg * 32 + (threadIdx.x & 31);
+  const int row = q_row0 + row_in_tile;
+  const uint32_t lane_off = static_cast<uint32_t>(warp_in_wg * 32) << 16;
+  const uint32_t tS = tmem + lane_off + static_cast<uint32_t>(w * 128);
+  const uint32_t tO = tmem + lane_off + static_cast<uint32_t>(256 + w * D);
+  const float c = p.scale_log2;
+  const int off = p.Skv - p.Sq;
+  // keys with index > last_key are masked for this row
+  const long long last_key_ll = p.causal ? static_cast<long long>(row) + off
+                                         : static_cast<long long>(p.Skv) - 1;
+  const int last_key = static_cast<int>(min(last_key_ll, static_cast<long long>(p.Skv) - 1));
+
+  float m = -INFINITY;
+  float l = 0.f;
+  const size_t row_index = (static_cast<size_t>(b) * p.Hq + h) * p.Sq + row;
+
+  if (n_tiles == 0) {
+    if (row < p.Sq) {
+      uint4* dst = reinterpret_cast<uint4*>(p.o + row_index * D);
+#pragma unroll
+      for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+      p.lse[row_index] = -INFINITY;
+    }
+    return;
+  }
+
+  for (int j = 0; j < n_tiles; ++j) {
+    bool ok = mbar_wait(bar_s, static_cast<uint32_t>(j & 1), abort_flag, p.wait_limit_ns);
+    if (!__all_sync(0xffffffffu, ok)) return;
+    tc_fence_after();
+
+    float s[kBN];
+#pragma unroll
+    for (int q4 = 0; q4 < kBN / 32; ++q4) {
+      uint32_t r[32];
+      tmem_ld32(tS + q4 * 32, r);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) s[q4 * 32 + e] = __uint_as_float(r[e]);
+    }
+
+    const int key0 = j * kBN;
+    const bool tile_masked = (key0 + kBN > p.Skv) ||
+                             (p.causal && static_cast<long long>(key0) + kBN - 1 >
+                                              static_cast<long long>(q_row0) + off);
+    if (tile_masked) {
+      const int lim = last_key - key0;  // columns > lim are invisible
+#pragma unroll
+      for (int e = 0; e < kBN; ++e)
+        if (e > lim) s[e] = -INFINITY;
+    }
+
+    // row max (exact in any order)
+    float mx[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mx[e] = s[e];
+#pragma unroll
+    for (int e = 8; e < kBN; ++e) mx[e & 7] = fmaxf(mx[e & 7], s[e]);
+    const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+    const float m_new = fmaxf(m, mt);
+    float alpha = 1.f;
+    if ((m_new - m) * c > kRescaleThreshold) {  // false while both are -inf (NaN)
+      alpha = ex2((m - m_new) * c);              // 0 when m was -inf
+      l *= alpha;
+      m = m_new;
+    }
+    const bool rescale_o = (j > 0) && __any_sync(0xffffffffu, alpha != 1.f);
+    const float mc = (m == -INFINITY) ? 0.f : m * c;
+
+    uint32_t pk0[32], pk1[32];
+    float rs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float p0 = ex2(fmaf(s[2 * i], c, -mc));
+      const float p1 = ex2(fmaf(s[2 * i + 1], c, -mc));
+      rs[i & 3] += p0 + p1;
+      pk0[i] = pack_bf16x2(p0, p1);
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float p0 = ex2(fmaf(s[64 + 2 * i], c, -mc));
+      const float p1 = ex2(fmaf(s[64 + 2 * i + 1], c, -mc));
+      rs[i & 3] += p0 + p1;
+      pk1[i] = pack_bf16x2(p0, p1);
+    }
+    l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+
+    if (rescale_o) {
+      // PV for tile j-1 has completed (its commit precedes this tile's S
+      // commit) and PV for tile j waits for our arrive below.
+#pragma unroll
+      for (int q4 = 0; q4 < D / 32; ++q4) {
+        uint32_t r[32];
+        tmem_ld32(tO + q4 * 32, r);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+        tmem_st32(tO + q4 * 32, r);
+      }
+    }
+    tmem_st32(tS, pk0);
+    tmem_st32(tS + 32, pk1);
+    tmem_st_wait();
+    tc_fence_before();
+    mbar_arrive(bar_p);
+  }
+
+  // epilogue: O / l -> bf16, LSE = m*scale + ln l
+  bool ok = mbar_wait(bar_o, 0u, abort_flag, p.wait_limit_ns);
+  if (!__all_sync(0xffffffffu, ok)) return;
+  tc_fence_after();
+  const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+  uint4* dst = reinterpret_cast<uint4*>(p.o + row_index * D);
+#pragma unroll
+  for (int q4 = 0; q4 < D / 32; ++q4) {
+    uint32_t r[32];
+    tmem_ld32(tO + q4 * 32, r);
+    if (row < p.Sq) {
+#pragma unroll
+      for (int v4 = 0; v4 < 4; ++v4) {
+        uint4 pkt;
+        pkt.x = pack_bf16x2(__uint_as_float(r[v4 * 8 + 0]) * inv_l, __uint_as_float(r[v4 * 8 + 1]) * inv_l);
+        pkt.y = pack_bf16x2(__uint_as_float(r[v4 * 8 + 2]) * inv_l, __uint_as_float(r[v4 * 8 + 3]) * inv_l);
+        pkt.z = pack_bf16x2(__uint_as_float(r[v4 * 8 + 4]) * inv_l, __uint_as_float(r[v4 * 8 + 5]) * inv_l);
+        pkt.w = pack_bf16x2(__uint_as_float(r[v4 * 8 + 6]) * inv_l, __uint_as_float(r[v4 * 8 + 7]) * inv_l);
+        dst[q4 * 4 + v4] = pkt;
+      }
+    }
+  }
+  if (row < p.Sq) p.lse[row_index] = (l > 0.f) ? m * p.scale + logf(l) : -INFINITY;
+}
+
+// ---------------------------------------------------------------------------
+// TMA producer (one thread).
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ void prefill_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                                                 const CUtensorMap* tm_v, const PrefillParams& p,
+                                                 uint32_t sbase, int pair, int b, int h, int g,
+                                                 int n_max, volatile int* abort_flag) {
+  using L = PrefillLayout<D>;
+  const uint32_t bars = sbase + L::kBarOff;
+  tma_prefetch_desc(tm_q);
+  tma_prefetch_desc(tm_k);
+  tma_prefetch_desc(tm_v);
+
+  const uint32_t bar_q = bars + 8 * L::kBarQ;
+  mbar_arrive_expect_tx(bar_q, 2 * L::kTileBytes);
+#pragma unroll
+  for (int w = 0; w < 2; ++w)
+#pragma unroll
+    for (int kb = 0; kb < D / 64; ++kb)
+      tma_load_3d(sbase + L::kQOff + w * L::kTileBytes + kb * kSwzBytes, tm_q, bar_q, kb * 64,
+                  (2 * pair + w) * kBM, b * p.Hq + h);
+
+  int issued = 0;
+  for (int idx = 0; idx < 2 * n_max; ++idx) {
+    const int stage = idx % L::kStages;
+    const uint32_t round = static_cast<uint32_t>(idx / L::kStages);
+    if (!mbar_wait(bars + 8 * (L::kBarKvEmpty + stage), (round & 1u) ^ 1u, abort_flag,
+                   p.wait_limit_ns))
+      break;
+    const uint32_t bar_full = bars + 8 * (L::kBarKvFull + stage);
+    mbar_arrive_expect_tx(bar_full, L::kTileBytes);
+    const CUtensorMap* tm = (idx & 1) ? tm_v : tm_k;
+#pragma unroll
+    for (int kb = 0; kb < D / 64; ++kb)
+      tma_load_3d(sbase + L::kRingOff + stage * L::kTileBytes + kb * kSwzBytes, tm, bar_full,
+                  kb * 64, (idx >> 1) * kBN, b * p.Hkv + g);
+    issued = idx + 1;
+  }
+
+  // Drain: no copy may still be in flight when the CTA exits.
+  mbar_wait(bar_q, 0u, nullptr, p.wait_limit_ns);
+  for (int idx = (issued > L::kStages ? issued - L::kStages : 0); idx < issued; ++idx)
+    mbar_wait(bars + 8 * (L::kBarKvFull + idx % L::kStages),
+              static_cast<uint32_t>(idx / L::kStages) & 1u, nullptr, p.wait_limit_ns);
+}
+
+// ---------------------------------------------------------------------------
+// MMA issuer (one thread).
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ void prefill_mma(const PrefillParams& p, uint32_t sbase, uint32_t tmem,
+                                            const int (&n_t)[2], int n_max,
+                                            volatile int* abort_flag) {
+  using L = PrefillLayout<D>;
+  const uint32_t bars = sbase + L::kBarOff;
+  constexpr uint32_t kIdS = idesc_bf16_f32(kBM, kBN, false);
+  constexpr uint32_t kIdPV = idesc_bf16_f32(kBM, D, true);
+
+  auto kv_stage = [](int idx) { return idx % L::kStages; };
+  auto kv_wait = [&](int idx) -> bool {
+    return mbar_wait(bars + 8 * (L::kBarKvFull + kv_stage(idx)),
+                     static_cast<uint32_t>(idx / L::kStages) & 1u, abort_flag, p.wait_limit_ns);
+  };
+  // S_w = Q_w K^T: M=128 rows, N=128 keys, K=D in steps of 16 (32 bytes).
+  auto issue_s = [&](int w, int stage) {
+    const uint32_t qa = sbase + L::kQOff + w * L::kTileBytes;
+    const uint32_t ka = sbase + L::kRingOff + stage * L::kTileBytes;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t o = (kk >> 2) * kSwzBytes + (kk & 3) * 32;
+      mma_ss(tmem + w * 128, sw128_desc(qa + o, 16, 1024), sw128_desc(ka + o, 16, 1024), kIdS,
+             kk > 0 ? 1u : 0u);
+    }
+  };
+  // O_w += P_w V: A = P_w in TMEM (bf16, 8 columns per 16 keys), B = V tile
+  // (keys x D, D contiguous: MN-major; 64-element column blocks 16 KB apart).
+  auto issue_pv = [&](int w, int stage, bool accumulate) {
+    const uint32_t va = sbase + L::kRingOff + stage * L::kTileBytes;
+#pragma unroll
+    for (int kk = 0; kk < kBN / 16; ++kk) {
+      mma_ts(tmem + 256 + w * D, tmem + w * 128 + kk * 8,
+             sw128_desc(va + kk * 16 * 128, kSwzBytes, 1024), kIdPV,
+             (accumulate || kk > 0) ? 1u : 0u);
+    }
+  };
+
+  if (!mbar_wait(bars + 8 * L::kBarQ, 0u, abort_flag, p.wait_limit_ns)) goto done;
+  if (n_max == 0) goto done;
+
+  if (!kv_wait(0)) goto done;
+  tc_fence_after();
+  if (n_t[0] > 0) { issue_s(0, kv_stage(0)); mma_commit(bars + 8 * (L::kBarSFull + 0)); }
+  if (n_t[1] > 0) { issue_s(1, kv_stage(0)); mma_commit(bars + 8 * (L::kBarSFull + 1)); }
+  mma_commit(bars + 8 * (L::kBarKvEmpty + kv_stage(0)));
+
+  for (int j = 0; j < n_max; ++j) {
+    const int iv = 2 * j + 1, ik = 2 * j + 2;
+    if (!kv_wait(iv)) goto done;
+    tc_fence_after();
+    if (j < n_t[0]) {
+      if (!mbar_wait(bars + 8 * (L::kBarPFull + 0), static_cast<uint32_t>(j & 1), abort_flag,
+                     p.wait_limit_ns))
+        goto done;
+      tc_fence_after();
+      issue_pv(0, kv_stage(iv), j > 0);
+      if (j == n_t[0] - 1) mma_commit(bars + 8 * (L::kBarOFull + 0));
+    }
+    const bool next = (j + 1 < n_max);
+    if (next) {
+      if (!kv_wait(ik)) goto done;
+      tc_fence_after();
+      if (j + 1 < n_t[0]) { issue_s(0, kv_stage(ik)); mma_commit(bars + 8 * (L::kBarSFull + 0)); }
+    }
+    if (j < n_t[1]) {
+      if (!mbar_wait(bars + 8 * (L::kBarPFull + 1), static_cast<uint32_t>(j & 1), abort_flag,
+                     p.wait_limit_ns))
+        goto done;
+      tc_fence_after();
+      issue_pv(1, kv_stage(iv), j > 0);
+      if (j == n_t[1] - 1) mma_commit(bars + 8 * (L::kBarOFull + 1));
+    }
+    mma_commit(bars + 8 * (L::kBarKvEmpty + kv_stage(iv)));
+    if (next) {
+      if (j + 1 < n_t[1]) { issue_s(1, kv_stage(ik)); mma_commit(bars + 8 * (L::kBarSFull + 1)); }
+      mma_commit(bars + 8 * (L::kBarKvEmpty + kv_stage(ik)));
+    }
+  }
+done:
+  // Every MMA this thread issued completes before tensor memory is freed.
+  mma_commit(bars + 8 * L::kBarDone);
+  mbar_wait(bars + 8 * L::kBarDone, 0u, nullptr, p.wait_limit_ns);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPrefillThreads, 1)
+fa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+  using L = PrefillLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sbase = raw + pad;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // Work item: the query-tile pair index is reversed under a causal mask so
+  // the longest items start first.
+  const int bh_count = p.B * p.Hq;
+  int pair = static_cast<int>(blockIdx.x) / bh_count;
+  const int bh = static_cast<int>(blockIdx.x) % bh_count;
+  if (p.causal) pair = p.n_qpairs - 1 - pair;
+  const int b = bh / p.Hq;
+  const int h = bh % p.Hq;
+  const int g = h / p.group;
+  int n_t[2];
+  n_t[0] = prefill_tiles_for(p, (2 * pair) * kBM);
+  n_t[1] = prefill_tiles_for(p, (2 * pair + 1) * kBM);
+  const int n_max = max(n_t[0], n_t[1]);
+
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbortOff);
+  const uint32_t bars = sbase + L::kBarOff;
+  if (threadIdx.x == 0) {
+    mbar_init(bars + 8 * L::kBarQ, 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(bars + 8 * (L::kBarKvFull + s), 1);
+      mbar_init(bars + 8 * (L::kBarKvEmpty + s), 1);
+    }
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(bars + 8 * (L::kBarSFull + w), 1);
+      mbar_init(bars + 8 * (L::kBarPFull + w), 128);
+      mbar_init(bars + 8 * (L::kBarOFull + w), 1);
+    }
+    mbar_init(bars + 8 * L::kBarDone, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(sbase + L::kTmemSlotOff, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlotOff);
+
+  if (warp < 8) {
+    const int w = warp >> 2;
+    prefill_softmax<D>(p, tmem, bars + 8 * (L::kBarSFull + w), bars + 8 * (L::kBarPFull + w),
+                       bars + 8 * (L::kBarOFull + w), w, n_t[w], (2 * pair + w) * kBM, b, h,
+                       abort_flag);
+  } else if (warp == 8) {
+    if (lane == 0)
+      prefill_producer<D>(&tm_q, &tm_k, &tm_v, p, sbase, pair, b, h, g, n_max, abort_flag);
+  } else if (warp == 9) {
+    if (lane == 0) prefill_mma<D>(p, sbase, tmem, n_t, n_max, abort_flag);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fa

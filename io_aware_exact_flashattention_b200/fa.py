@@ -1,0 +1,217 @@
+"""Python binding of libfa.so (include/fa.h): argument marshalling only.
+
+Every step of the attention path runs in the library's CUDA kernels; torch is
+used here to hold device memory and to name the current CUDA stream.  There is
+no CPU or library fallback: if libfa.so is missing or a call fails, these
+functions raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfa.so")
+
+FA_OK = 0
+STATUS_NAMES = {
+    0: "FA_OK",
+    1: "FA_ERR_INVALID_ARG",
+    2: "FA_ERR_UNSUPPORTED",
+    3: "FA_ERR_ALIGNMENT",
+    4: "FA_ERR_CUDA",
+    5: "FA_ERR_DEVICE_TIMEOUT",
+}
+
+# Every symbol include/fa.h declares, with (restype, argtypes).
+_VP, _FP, _I32P = ctypes.c_void_p, ctypes.POINTER(ctypes.c_float), ctypes.c_void_p
+_I, _F = ctypes.c_int, ctypes.c_float
+SIGNATURES = {
+    "fa_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _VP]),
+    "fa_decode_splitkv": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP]),
+    "fa_combine": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP]),
+    "fa_decode_default_splits": (_I, [_I, _I, _I, _I]),
+    "fa_status_string": (ctypes.c_char_p, [_I]),
+    "fa_get_device_status": (_I, []),
+    "fa_debug_timeout_probe": (_I, [ctypes.c_uint, _VP]),
+}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+class FAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__("%s failed: %s" % (fn, status_string(status)))
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfa.so (built by io_aware_exact_flashattention_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libfa.so is not built; run "
+                               "`python -m io_aware_exact_flashattention_b200.build`")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(l, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = l
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().fa_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != FA_OK:
+        raise FAError(fn, status)
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> Optional[int]:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream or None
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else (t.data_ptr() or None)
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, name: str) -> None:
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+# ---------------------------------------------------------------------------
+# Raw C-ABI calls on device tensors (outputs preallocated by the caller)
+# ---------------------------------------------------------------------------
+
+def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+           lse: torch.Tensor, causal: bool, scale: float,
+           stream: Optional[torch.cuda.Stream] = None) -> None:
+    """fa_fwd on q [B,Hq,Sq,d], k/v [B,Hkv,Skv,d] (bf16), o [B,Hq,Sq,d] bf16,
+    lse [B,Hq,Sq] fp32, all on the same CUDA device."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _need(t, torch.bfloat16, n)
+    _need(lse, torch.float32, "lse")
+    B, Hq, Sq, d = q.shape
+    _, Hkv, Skv, _ = k.shape
+    if tuple(v.shape) != tuple(k.shape) or k.shape[0] != B or k.shape[3] != d:
+        raise ValueError("k/v shapes %s/%s do not match q %s" % (tuple(k.shape), tuple(v.shape),
+                                                                 tuple(q.shape)))
+    if tuple(o.shape) != tuple(q.shape) or tuple(lse.shape) != (B, Hq, Sq):
+        raise ValueError("output shapes do not match q")
+    _check("fa_fwd", lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Sq,
+                                  Skv, d, int(bool(causal)), float(scale), _stream_ptr(stream)))
+
+
+def fa_decode_splitkv(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                      seqlens_k: torch.Tensor, o_partial: torch.Tensor,
+                      lse_partial: torch.Tensor, scale: float,
+                      stream: Optional[torch.cuda.Stream] = None) -> None:
+    """fa_decode_splitkv on q [B,Hq,d], caches [B,Hkv,Lmax,d] (bf16), seqlens
+    [B] int32; o_partial [B,Hq,n,d] and lse_partial [B,Hq,n] fp32."""
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, torch.bfloat16, n)
+    _need(seqlens_k, torch.int32, "seqlens_k")
+    _need(o_partial, torch.float32, "o_partial")
+    _need(lse_partial, torch.float32, "lse_partial")
+    B, Hq, d = q.shape
+    _, Hkv, Lmax, _ = k_cache.shape
+    n = o_partial.shape[2]
+    if tuple(o_partial.shape) != (B, Hq, n, d) or tuple(lse_partial.shape) != (B, Hq, n):
+        raise ValueError("partial buffers must be [B,Hq,n,d] and [B,Hq,n]")
+    _check("fa_decode_splitkv", lib().fa_decode_splitkv(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens_k), _ptr(o_partial),
+        _ptr(lse_partial), B, Hq, Hkv, Lmax, d, n, float(scale), _stream_ptr(stream)))
+
+
+def fa_combine(o_partial: torch.Tensor, lse_partial: torch.Tensor, o: torch.Tensor,
+               lse: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """fa_combine: o_partial [B,Hq,n,d], lse_partial [B,Hq,n] fp32 -> o [B,Hq,d]
+    bf16, lse [B,Hq] fp32."""
+    _need(o_partial, torch.float32, "o_partial")
+    _need(lse_partial, torch.float32, "lse_partial")
+    _need(o, torch.bfloat16, "o")
+    _need(lse, torch.float32, "lse")
+    B, Hq, n, d = o_partial.shape
+    if tuple(o.shape) != (B, Hq, d) or tuple(lse.shape) != (B, Hq):
+        raise ValueError("outputs must be [B,Hq,d] and [B,Hq]")
+    _check("fa_combine", lib().fa_combine(_ptr(o_partial), _ptr(lse_partial), _ptr(o), _ptr(lse),
+                                          B, Hq, n, d, _stream_ptr(stream)))
+
+
+def decode_default_splits(B: int, Hkv: int, Lmax: int, num_sms: int) -> int:
+    return int(lib().fa_decode_default_splits(B, Hkv, Lmax, num_sms))
+
+
+def get_device_status() -> int:
+    """Read and clear the device status word (synchronises the device)."""
+    return int(lib().fa_get_device_status())
+
+
+def debug_timeout_probe(limit_us: int, stream: Optional[torch.cuda.Stream] = None) -> None:
+    _check("fa_debug_timeout_probe", lib().fa_debug_timeout_probe(int(limit_us),
+                                                                  _stream_ptr(stream)))
+
+
+# ---------------------------------------------------------------------------
+# User-level calls: allocate outputs; host tensors are copied in and out
+# ---------------------------------------------------------------------------
+
+def flash_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+                    scale: Optional[float] = None, device: Optional[torch.device] = None
+                    ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Exact attention O = softmax(scale*QK^T [+causal mask]) V and its LSE.
+
+    CUDA inputs stay where they are; CPU inputs (ideally pinned) are copied to
+    `device` (default: the current CUDA device) and the results copied back."""
+    host = not q.is_cuda
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    if host:
+        dev = device or torch.device("cuda", torch.cuda.current_device())
+        q, k, v = (t.to(dev, non_blocking=True) for t in (q, k, v))
+    B, Hq, Sq, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Sq), device=q.device, dtype=torch.float32)
+    fa_fwd(q, k, v, o, lse, causal, scale)
+    if host:
+        o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        o_h.copy_(o, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+        return o_h, lse_h
+    return o, lse
+
+
+def decode_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                     seqlens_k: torch.Tensor, scale: Optional[float] = None,
+                     num_splits: Optional[int] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Single-query decode over a contiguous cache: split-KV partials, then the
+    LSE-weighted merge.  All tensors on one CUDA device."""
+    B, Hq, d = q.shape
+    _, Hkv, Lmax, _ = k_cache.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if num_splits is None:
+        sms = torch.cuda.get_device_properties(q.device).multi_processor_count
+        num_splits = decode_default_splits(B, Hkv, Lmax, sms)
+    o_part = torch.empty((B, Hq, num_splits, d), device=q.device, dtype=torch.float32)
+    lse_part = torch.empty((B, Hq, num_splits), device=q.device, dtype=torch.float32)
+    fa_decode_splitkv(q, k_cache, v_cache, seqlens_k, o_part, lse_part, scale)
+    o = torch.empty((B, Hq, d), device=q.device, dtype=torch.bfloat16)
+    lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32)
+    fa_combine(o_part, lse_part, o, lse)
+    return o, lse
