@@ -170,12 +170,15 @@ def debug_timeout_probe(limit_us: int, stream: Optional[torch.cuda.Stream] = Non
 # ---------------------------------------------------------------------------
 
 def flash_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
-                    scale: Optional[float] = None, device: Optional[torch.device] = None
+                    scale: Optional[float] = None, device: Optional[torch.device] = None,
+                    out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None
                     ) -> Tuple[torch.Tensor, torch.Tensor]:
     """Exact attention O = softmax(scale*QK^T [+causal mask]) V and its LSE.
 
     CUDA inputs stay where they are; CPU inputs (ideally pinned) are copied to
-    `device` (default: the current CUDA device) and the results copied back."""
+    `device` (default: the current CUDA device), and the results are copied
+    back into `out` = (o, lse) host tensors when given, else into new pinned
+    tensors.  With host inputs the call returns after the results landed."""
     host = not q.is_cuda
     if scale is None:
         scale = 1.0 / math.sqrt(q.shape[-1])
@@ -183,12 +186,18 @@ def flash_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: b
         dev = device or torch.device("cuda", torch.cuda.current_device())
         q, k, v = (t.to(dev, non_blocking=True) for t in (q, k, v))
     B, Hq, Sq, d = q.shape
-    o = torch.empty_like(q)
-    lse = torch.empty((B, Hq, Sq), device=q.device, dtype=torch.float32)
+    if out is not None and not host:
+        o, lse = out
+    else:
+        o = torch.empty_like(q)
+        lse = torch.empty((B, Hq, Sq), device=q.device, dtype=torch.float32)
     fa_fwd(q, k, v, o, lse, causal, scale)
     if host:
-        o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-        lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        if out is not None:
+            o_h, lse_h = out
+        else:
+            o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+            lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
         o_h.copy_(o, non_blocking=True)
         lse_h.copy_(lse, non_blocking=True)
         torch.cuda.current_stream().synchronize()
