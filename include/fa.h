@@ -149,6 +149,41 @@ fa_status fa_get_device_status(void);
  */
 fa_status fa_debug_timeout_probe(unsigned int limit_us, fa_stream_t stream);
 
+/*
+ * fa_decode_noalloc -- single-query decode that allocates nothing.
+ *
+ * The pages have no counterpart to this call.  It computes exactly what
+ * fa_decode_splitkv followed by fa_combine computes, with the same arguments
+ * and the same meaning of q, k_cache, v_cache, seqlens_k, o and lse, but the
+ * split partials live in a fixed array inside the library instead of a
+ * buffer from the caller.  It is meant for callers that can neither call
+ * cudaMalloc nor hand the library a workspace: a plugin whose host framework
+ * owns every device allocation and passes an op nothing but its own tensors,
+ * or a serving loop that must not allocate once it runs, because cudaMalloc
+ * can synchronise the device and stall all of its streams.
+ *
+ * Limits and behaviour:
+ *  - The array is 32 MiB on every device that loads libfa.so, held until the
+ *    process exits.  The partials need B*Hq*num_splits*d*4 bytes, rounded up
+ *    to 256, plus B*Hq*num_splits*4; a call that needs more returns
+ *    FA_ERR_UNSUPPORTED before any CUDA call (use fewer splits, or
+ *    fa_decode_splitkv with a caller buffer).
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and keeps it; make that
+ *    first call before any stream capture.  No call allocates device or host
+ *    memory: no cudaMalloc, no cudaFree, no allocating library routine.
+ *  - All calls on a device share the one array, which keeps the previous
+ *    call's partials.  Calls whose kernels overlap on the GPU (other streams,
+ *    other host threads) race on it; order them on one stream.  Nothing in it
+ *    needs to start at zero: every partial the merge reads is written first.
+ *  - Supported shapes and the other errors are those of fa_decode_splitkv and
+ *    fa_combine.
+ */
+fa_status fa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *seqlens_k, void *o, float *lse, int B, int Hq,
+                            int Hkv, int Lmax, int d, int num_splits, float scale,
+                            fa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -147,6 +147,32 @@ __global__ void timeout_probe_kernel(unsigned long long limit_ns) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Fixed, library-owned scratch for fa_decode_noalloc.
+// ---------------------------------------------------------------------------
+// 32 MiB on every device that loads this library, held until the process
+// exits.  The name is only a host-side stand-in: host code obtains the
+// device address with cudaGetSymbolAddress (once per device, that device
+// current) and passes that address to the kernels.
+constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(32) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices];  // device address per device; null until set up
+
+cudaError_t noalloc_scratch_address(int dev, void** addr) {
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_addr[dev] = p;
+  }
+  *addr = g_noalloc_addr[dev];
+  return cudaSuccess;
+}
+
 }  // namespace
 
 extern "C" {
@@ -272,6 +298,36 @@ fa_status fa_debug_timeout_probe(unsigned int limit_us, fa_stream_t stream) {
   timeout_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<unsigned long long>(limit_us) * 1000ull);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* seqlens_k, void* o, float* lse, int B, int Hq,
+                            int Hkv, int Lmax, int d, int num_splits, float scale,
+                            fa_stream_t stream) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || Lmax < 0) return FA_ERR_INVALID_ARG;
+  if (num_splits < 1 || num_splits > 256) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  // Split partials: o_part [B,Hq,n,d] fp32 at offset 0, lse_part [B,Hq,n] fp32
+  // at the next 256-byte boundary.  Larger than the fixed array: refuse.
+  const unsigned long long rows = static_cast<unsigned long long>(B) * Hq * num_splits;
+  const unsigned long long o_bytes = rows * static_cast<unsigned long long>(d) * 4ull;
+  const unsigned long long lse_off = (o_bytes + 255ull) & ~255ull;
+  if (lse_off + rows * 4ull > kNoAllocScratchBytes) return FA_ERR_UNSUPPORTED;
+  if (B == 0) return FA_OK;
+  if (o == nullptr || lse == nullptr) return FA_ERR_INVALID_ARG;
+  if (!aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGNMENT;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  void* base = nullptr;
+  if (noalloc_scratch_address(dev, &base) != cudaSuccess) return FA_ERR_CUDA;
+  float* o_part = static_cast<float*>(base);
+  float* lse_part = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + lse_off);
+  // Every partial the merge reads is written by the split pass first, so the
+  // array's previous contents never matter and nothing is cleared.
+  const fa_status st = fa_decode_splitkv(q, k_cache, v_cache, seqlens_k, o_part, lse_part, B,
+                                         Hq, Hkv, Lmax, d, num_splits, scale, stream);
+  if (st != FA_OK) return st;
+  return fa_combine(o_part, lse_part, o, lse, B, Hq, num_splits, d, stream);
 }
 
 }  // extern "C"

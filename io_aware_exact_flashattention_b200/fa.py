@@ -38,6 +38,7 @@ SIGNATURES = {
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_get_device_status": (_I, []),
     "fa_debug_timeout_probe": (_I, [ctypes.c_uint, _VP]),
+    "fa_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
