@@ -59,6 +59,10 @@ def parse_args():
                     help="prefill workload name (io_aware_exact_flashattention_b200.inputs)")
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                     help="restrict the step (for profiling captures)")
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="override the decode workload's batch (smaller profiling captures)")
+    ap.add_argument("--decode-splits", type=int, default=None,
+                    help="override the decode split count (default: fa_decode_default_splits)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -287,10 +291,14 @@ def run_ours(args, world, rank, local):
     o = torch.empty_like(q)
     lse = torch.empty((c.B, c.Hq, c.Sq), device=dev, dtype=torch.float32)
     if do_dec:
+        if args.decode_batch is not None:
+            import dataclasses
+            cd = dataclasses.replace(cd, B=args.decode_batch,
+                                     name="%s_b%d" % (cd.name, args.decode_batch))
         qd, kc, vc, sl = decode_inputs(cd.B, cd.Hq, cd.Hkv, cd.Lmin, cd.Lmax, cd.d,
                                        cd.seed + seed_off, device=dev)
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
-        n_split = fa.decode_default_splits(cd.B, cd.Hkv, cd.Lmax, sms)
+        n_split = args.decode_splits or fa.decode_default_splits(cd.B, cd.Hkv, cd.Lmax, sms)
         op = torch.empty((cd.B, cd.Hq, n_split, cd.d), device=dev, dtype=torch.float32)
         lp = torch.empty((cd.B, cd.Hq, n_split), device=dev, dtype=torch.float32)
         od = torch.empty((cd.B, cd.Hq, cd.d), device=dev, dtype=torch.bfloat16)
@@ -413,13 +421,17 @@ def run_ours(args, world, rank, local):
             "frac_of_measured_copy": dec_achieved / hbm, "num_splits": n_split,
             "bytes_per_call": dec_bytes}
         line["roofline_decode"] = {
-            "bound": "hbm", "kernel": "fa_decode_split_kernel<128,4> + fa_combine_kernel<128>",
+            "bound": "hbm", "kernel": "fa_decode_split_kernel<128,4> + fa_combine_kernel<128> (timed together)",
             "achieved": dec_achieved, "peak": hbm, "unit": "GB/s", "frac": dec_achieved / hbm,
             "peak_source": "%s copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" % peaks_kind,
             "traffic": profiled_traffic("decode_b64_splitkv_d128.md", DECODE_SOURCES),
             "algorithmic": "%d bytes per call (K,V visible rows + q + O + LSE)" % dec_bytes}
-        if not do_pre:
-            line["roofline"] = line["roofline_decode"]
+    # `roofline` describes the kernel that takes most of the step's time.
+    if do_pre and do_dec and dec_ms > pre_ms:
+        line["roofline_prefill"] = line.pop("roofline")
+        line["roofline"] = line.pop("roofline_decode")
+    elif do_dec and not do_pre:
+        line["roofline"] = line.pop("roofline_decode")
     if cpu is not None:
         line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)

@@ -107,27 +107,107 @@ fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, f
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// Per device: SM count, and the decode kernels' shared-memory opt-in.
+std::once_flag g_dec_once[kMaxDevices];
+cudaError_t g_dec_err[kMaxDevices];
+int g_num_sms[kMaxDevices];
+
+template <int D>
+cudaError_t decode_attr() {
+  cudaError_t e = cudaSuccess;
+  auto set = [&e](const void* fn) {
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::DecodeLayout<D>::kBytes);
+  };
+  set(reinterpret_cast<const void*>(fa::fa_decode_split_kernel<D, 1>));
+  set(reinterpret_cast<const void*>(fa::fa_decode_split_kernel<D, 2>));
+  set(reinterpret_cast<const void*>(fa::fa_decode_split_kernel<D, 4>));
+  set(reinterpret_cast<const void*>(fa::fa_decode_split_kernel<D, 8>));
+  return e;
+}
+
+cudaError_t prepare_decode(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::call_once(g_dec_once[dev], [dev] {
+    cudaError_t e = cudaDeviceGetAttribute(&g_num_sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = decode_attr<64>();
+    if (e == cudaSuccess) e = decode_attr<128>();
+    g_dec_err[dev] = e;
+  });
+  return g_dec_err[dev];
+}
+
+// [planes, rows, d] bf16 cache as a 3-D map with 64 x box_rows x 1 boxes.
+bool encode_cache(CUtensorMap* map, const void* base, int d, int rows, long long planes,
+                  int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t r = static_cast<cuuint64_t>(rows > 0 ? rows : 1);
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), r, static_cast<cuuint64_t>(planes)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, r * static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [rows, d] bf16 query matrix as a 2-D map with 64 x 16 boxes.
+bool encode_query(CUtensorMap* map, const void* base, int d, long long rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(fa::kDecNPad)};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D, int G>
-void launch_decode(const void* q, const void* kc, const void* vc, const int32_t* seqlens,
-                   float* o_part, float* lse_part, int B, int Hq, int Hkv, int Lmax,
-                   int num_splits, float scale, cudaStream_t stream) {
-  dim3 grid(num_splits, Hkv, B);
-  fa::fa_decode_split_kernel<D, G><<<grid, fa::kDecodeThreads, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(kc),
-      static_cast<const __nv_bfloat16*>(vc), seqlens, o_part, lse_part, Hq, Hkv, Lmax,
-      num_splits, scale * 1.4426950408889634f);
+fa_status launch_decode(const void* q, const void* kc, const void* vc, const int32_t* seqlens,
+                        float* o_part, float* lse_part, int B, int Hq, int Hkv, int Lmax,
+                        int num_splits, float scale, int num_sms, cudaStream_t stream) {
+  CUtensorMap tk, tv, tk32, tv32, tq;
+  const long long planes = static_cast<long long>(B) * Hkv;
+  if (!encode_cache(&tk, kc, D, Lmax, planes, fa::kDecBN) ||
+      !encode_cache(&tv, vc, D, Lmax, planes, fa::kDecBN) ||
+      !encode_cache(&tk32, kc, D, Lmax, planes, fa::kDecSubRows) ||
+      !encode_cache(&tv32, vc, D, Lmax, planes, fa::kDecSubRows) ||
+      !encode_query(&tq, q, D, static_cast<long long>(B) * Hq))
+    return FA_ERR_CUDA;
+  fa::DecodeParams p;
+  p.o_part = o_part;
+  p.lse_part = lse_part;
+  p.seqlens = seqlens;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Lmax = Lmax;
+  p.n_splits = num_splits;
+  p.n_items = B * Hkv * num_splits;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_limit_ns = kWaitLimitNs;
+  const int grid = p.n_items < num_sms ? p.n_items : num_sms;
+  fa::fa_decode_split_kernel<D, G><<<grid, fa::kDecThreads, fa::DecodeLayout<D>::kBytes,
+                                     stream>>>(tk, tv, tk32, tv32, tq, p);
+  return FA_OK;
 }
 
 template <int D>
-bool dispatch_decode_group(int G, const void* q, const void* kc, const void* vc,
-                           const int32_t* seqlens, float* o_part, float* lse_part, int B, int Hq,
-                           int Hkv, int Lmax, int num_splits, float scale, cudaStream_t stream) {
+fa_status dispatch_decode_group(int G, const void* q, const void* kc, const void* vc,
+                                const int32_t* seqlens, float* o_part, float* lse_part, int B,
+                                int Hq, int Hkv, int Lmax, int num_splits, float scale,
+                                int num_sms, cudaStream_t stream) {
   switch (G) {
-    case 1: launch_decode<D, 1>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, stream); return true;
-    case 2: launch_decode<D, 2>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, stream); return true;
-    case 4: launch_decode<D, 4>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, stream); return true;
-    case 8: launch_decode<D, 8>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, stream); return true;
-    default: return false;
+    case 1: return launch_decode<D, 1>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, num_sms, stream);
+    case 2: return launch_decode<D, 2>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, num_sms, stream);
+    case 4: return launch_decode<D, 4>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, num_sms, stream);
+    case 8: return launch_decode<D, 8>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, num_sms, stream);
+    default: return FA_ERR_UNSUPPORTED;
   }
 }
 
@@ -209,7 +289,6 @@ fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_ca
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   const int G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8) return FA_ERR_UNSUPPORTED;
-  if (B > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
   if (B == 0) return FA_OK;
   if (q == nullptr || k_cache == nullptr || v_cache == nullptr || seqlens_k == nullptr ||
       o_partial == nullptr || lse_partial == nullptr)
@@ -218,14 +297,19 @@ fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_ca
       (reinterpret_cast<uintptr_t>(seqlens_k) & 3u) != 0 ||
       !aligned16(o_partial) || !aligned16(lse_partial))
     return FA_ERR_ALIGNMENT;
+  if (static_cast<long long>(B) * Hkv * num_splits > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (prepare_decode(dev) != cudaSuccess) return FA_ERR_CUDA;
+  const int sms = g_num_sms[dev];
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const bool ok = d == 64 ? dispatch_decode_group<64>(G, q, k_cache, v_cache, seqlens_k, o_partial,
-                                                      lse_partial, B, Hq, Hkv, Lmax, num_splits,
-                                                      scale, s)
-                          : dispatch_decode_group<128>(G, q, k_cache, v_cache, seqlens_k,
-                                                       o_partial, lse_partial, B, Hq, Hkv, Lmax,
-                                                       num_splits, scale, s);
-  if (!ok) return FA_ERR_UNSUPPORTED;
+  const fa_status st =
+      d == 64 ? dispatch_decode_group<64>(G, q, k_cache, v_cache, seqlens_k, o_partial,
+                                          lse_partial, B, Hq, Hkv, Lmax, num_splits, scale, sms, s)
+              : dispatch_decode_group<128>(G, q, k_cache, v_cache, seqlens_k, o_partial,
+                                           lse_partial, B, Hq, Hkv, Lmax, num_splits, scale, sms,
+                                           s);
+  if (st != FA_OK) return st;
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

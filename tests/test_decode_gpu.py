@@ -15,7 +15,11 @@ pytestmark = pytest.mark.gpu
 
 O_TOL = 2e-2
 LSE_TOL = 1e-3
-PART_TOL = 5e-5  # fp32 partials: no bf16 step on the output side
+# Partials are fp32, but their P.V product takes the probabilities in bf16:
+# each weight carries a relative rounding error <= 2^-9, so a partial (a convex
+# combination of value rows) is off by at most 2^-9 * max|v| (~0.01 for
+# N(0,1) values); the same bound covers the fp32 normaliser's mismatch.
+PART_TOL = 1e-2
 
 
 @pytest.fixture(scope="module", autouse=True)
