@@ -57,12 +57,27 @@ bool encode_bhsd(CUtensorMap* map, const void* base, int d, int rows, long long 
 std::once_flag g_attr_once[kMaxDevices];
 cudaError_t g_attr_err[kMaxDevices];
 
+// The prefill kernel moves registers between its warpgroups (setmaxnreg);
+// that is only safe when every thread was launched with the register count
+// the split was computed for, so a build that compiled to another count is
+// refused instead of launched.
+template <int D>
+cudaError_t check_prefill_regs() {
+  cudaFuncAttributes a;
+  cudaError_t e = cudaFuncGetAttributes(&a, fa::fa_prefill_kernel<D>);
+  if (e != cudaSuccess) return e;
+  return a.numRegs == fa::kPrefillLaunchRegs ? cudaSuccess : cudaErrorInvalidKernelImage;
+}
+
 cudaError_t prepare_prefill(int dev) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::call_once(g_attr_once[dev], [dev] {
-    cudaError_t e = cudaFuncSetAttribute(fa::fa_prefill_kernel<64>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         fa::PrefillLayout<64>::kBytes);
+    cudaError_t e = check_prefill_regs<64>();
+    if (e == cudaSuccess) e = check_prefill_regs<128>();
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fa::fa_prefill_kernel<64>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::PrefillLayout<64>::kBytes);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(fa::fa_prefill_kernel<128>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,

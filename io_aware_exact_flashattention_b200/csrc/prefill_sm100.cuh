@@ -8,11 +8,14 @@
 // tiling plus online softmax).  The loop order is query-stationary: the
 // output tile is accumulated on chip and written to HBM once.
 //
-// Roles (320 threads):
+// Roles (384 threads, three warpgroups):
 //   warps 0-3  softmax warpgroup for query tile 0 (thread = row = TMEM lane)
 //   warps 4-7  softmax warpgroup for query tile 1
 //   warp  8    TMA producer: Q tiles once, then K_j, V_j into a smem ring
 //   warp  9    MMA issuer: S_w = Q_w K_j^T and O_w += P_w V_j on tcgen05
+//   warps 10-11 idle
+// Registers are moved from the third warpgroup to the softmax warpgroups
+// (setmaxnreg): 224 + 224 + 56 per SM sub-partition = 3 x 168 at launch.
 // Tensor memory (512 columns x 128 lanes x 32 bit):
 //   [0,128)   S_0 (fp32 scores); P_0 (bf16) overwrites its first 64 columns
 //   [128,256) S_1 / P_1
@@ -27,6 +30,7 @@
 #pragma once
 
 #include <climits>
+#include <type_traits>
 #include <cuda.h>
 #include "sm100.cuh"
 
@@ -34,9 +38,41 @@ namespace fa {
 
 constexpr int kBM = 128;       // query rows per tile (= TMEM lanes)
 constexpr int kBN = 128;       // keys per key/value tile
-constexpr int kPrefillThreads = 320;
+constexpr int kPrefillThreads = 384;
+constexpr int kPrefillLaunchRegs = 168;   // 65536 / 384, rounded down to a multiple of 8
+constexpr int kSoftmaxRegs = 224;
+constexpr int kControlRegs = 56;
+static_assert(2 * kSoftmaxRegs + kControlRegs <= 3 * kPrefillLaunchRegs,
+              "register split exceeds the launch budget");
 constexpr int kSwzBytes = 128 * 128;  // one 128-row x 64-element bf16 box, 128B swizzled
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+// 2^x for part of the softmax on the FMA pipe instead of the MUFU: with
+// n = round(x) and f = x - n in [-1/2, 1/2], 2^x = 2^n * p(f) where p is the
+// degree-3 minimax fit of 2^f below (max relative error 7.5e-5; derived by
+// exp2_poly_fit.py next to this file).  2^n is applied by adding n to the
+// exponent field.  Arguments are clamped to >= -126; larger ones stay <= 8
+// because the reference max is never more than 2^8 below the row max.
+constexpr float kExp2C0 = 9.999280572e-01f;
+constexpr float kExp2C1 = 6.932609677e-01f;
+constexpr float kExp2C2 = 2.426111251e-01f;
+constexpr float kExp2C3 = 5.517166853e-02f;
+constexpr int kPolyPairsPer8 = 3;  // of every 8 pairs of scores, this many use the polynomial
+
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = fadd2(x, make_float2(kRound, kRound));
+  const float2 n = fadd2(t, make_float2(-kRound, -kRound));
+  const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
+  float2 q = ffma2(f, make_float2(kExp2C3, kExp2C3), make_float2(kExp2C2, kExp2C2));
+  q = ffma2(q, f, make_float2(kExp2C1, kExp2C1));
+  q = ffma2(q, f, make_float2(kExp2C0, kExp2C0));
+  // the low bits of t hold n, so (bits(t) << 23) == (n << 23) modulo 2^32
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
 
 struct PrefillParams {
   __nv_bfloat16* o;
@@ -57,13 +93,13 @@ struct PrefillLayout {
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = 2 * kTileBytes;
   static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
-  // q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], mma_done
+  // q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2][2 halves], o_full[2], mma_done
   static constexpr int kBarQ = 0;
   static constexpr int kBarKvFull = 1;
   static constexpr int kBarKvEmpty = 1 + kStages;
   static constexpr int kBarSFull = 1 + 2 * kStages;
   static constexpr int kBarPFull = kBarSFull + 2;
-  static constexpr int kBarOFull = kBarPFull + 2;
+  static constexpr int kBarOFull = kBarPFull + 4;
   static constexpr int kBarDone = kBarOFull + 2;
   static constexpr int kNumBars = kBarDone + 1;
   static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
@@ -121,13 +157,18 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
     if (!__all_sync(0xffffffffu, ok)) return;
     tc_fence_after();
 
+    // scores: the second half streams in while the first half's max runs
     float s[kBN];
+    {
+      uint32_t ra[64], rb[64];
+      tmem_ld64_nowait(tS, ra);
+      tmem_ld_wait_hold(ra);
+      tmem_ld64_nowait(tS + 64, rb);
 #pragma unroll
-    for (int q4 = 0; q4 < kBN / 32; ++q4) {
-      uint32_t r[32];
-      tmem_ld32(tS + q4 * 32, r);
+      for (int e = 0; e < 64; ++e) s[e] = __uint_as_float(ra[e]);
+      tmem_ld_wait_hold(rb);
 #pragma unroll
-      for (int e = 0; e < 32; ++e) s[q4 * 32 + e] = __uint_as_float(r[e]);
+      for (int e = 0; e < 64; ++e) s[64 + e] = __uint_as_float(rb[e]);
     }
 
     const int key0 = j * kBN;
@@ -141,14 +182,16 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
         if (e > lim) s[e] = -INFINITY;
     }
 
-    // row max (exact in any order)
+    // row max (exact in any order): three-input max over eight partial maxima
     float mx[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) mx[e] = s[e];
+    for (int k = 0; k < 8; ++k) mx[k] = fmaxf(s[2 * k], s[2 * k + 1]);
 #pragma unroll
-    for (int e = 8; e < kBN; ++e) mx[e & 7] = fmaxf(mx[e & 7], s[e]);
-    const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+    for (int i = 16; i < kBN; i += 16)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], s[i + 2 * k], s[i + 2 * k + 1]);
+    const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                           fmaxf(mx[6], mx[7]));
     const float m_new = fmaxf(m, mt);
     float alpha = 1.f;
     if ((m_new - m) * c > kRescaleThreshold) {  // false while both are -inf (NaN)
@@ -159,27 +202,9 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
     const bool rescale_o = (j > 0) && __any_sync(0xffffffffu, alpha != 1.f);
     const float mc = (m == -INFINITY) ? 0.f : m * c;
 
-    uint32_t pk0[32], pk1[32];
-    float rs[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float p0 = ex2(fmaf(s[2 * i], c, -mc));
-      const float p1 = ex2(fmaf(s[2 * i + 1], c, -mc));
-      rs[i & 3] += p0 + p1;
-      pk0[i] = pack_bf16x2(p0, p1);
-    }
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float p0 = ex2(fmaf(s[64 + 2 * i], c, -mc));
-      const float p1 = ex2(fmaf(s[64 + 2 * i + 1], c, -mc));
-      rs[i & 3] += p0 + p1;
-      pk1[i] = pack_bf16x2(p0, p1);
-    }
-    l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-
     if (rescale_o) {
       // PV for tile j-1 has completed (its commit precedes this tile's S
-      // commit) and PV for tile j waits for our arrive below.
+      // commit) and PV for tile j waits for the arrives below.
 #pragma unroll
       for (int q4 = 0; q4 < D / 32; ++q4) {
         uint32_t r[32];
@@ -189,11 +214,46 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
         tmem_st32(tO + q4 * 32, r);
       }
     }
-    tmem_st32(tS, pk0);
-    tmem_st32(tS + 32, pk1);
-    tmem_st_wait();
-    tc_fence_before();
-    mbar_arrive(bar_p);
+
+    // p = 2^(s*c - m*c) on pairs; l sums the fp32 p, P keeps them as bf16.
+    // Each half of the row (64 keys) is stored to tensor memory and
+    // announced on its own barrier, so P.V on the first 64 keys runs while
+    // the second half is computed.
+    const float2 c2 = make_float2(c, c);
+    const float2 nmc2 = make_float2(-mc, -mc);
+    float2 rs[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                    make_float2(0.f, 0.f)};
+    // Masked tiles take every exponential on the MUFU (2^-inf is exactly 0);
+    // the others move kPolyPairsPer8 of every 8 pairs to the FMA pipe.
+    auto exps_half = [&](auto poly_tag, int half) {
+      constexpr bool kPoly = decltype(poly_tag)::value;
+      uint32_t pk[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int e = half * 64 + 2 * i;
+        const float2 x = ffma2(make_float2(s[e], s[e + 1]), c2, nmc2);
+        const float2 pp = (kPoly && (i & 7) >= 8 - kPolyPairsPer8)
+                              ? exp2_poly2(x)
+                              : make_float2(ex2(x.x), ex2(x.y));
+        rs[i & 3] = fadd2(rs[i & 3], pp);
+        pk[i] = pack_bf16x2(pp.x, pp.y);
+      }
+      tmem_st32(tS + half * 32, pk);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_p + 8 * half);
+    };
+    if (tile_masked) {
+      exps_half(std::false_type{}, 0);
+      exps_half(std::false_type{}, 1);
+    } else {
+      exps_half(std::true_type{}, 0);
+      exps_half(std::true_type{}, 1);
+    }
+    {
+      const float2 t2 = fadd2(fadd2(rs[0], rs[1]), fadd2(rs[2], rs[3]));
+      l += t2.x + t2.y;
+    }
   }
 
   // epilogue: O / l -> bf16, LSE = m*scale + ln l
@@ -298,14 +358,23 @@ __device__ __forceinline__ void prefill_mma(const PrefillParams& p, uint32_t sba
   };
   // O_w += P_w V: A = P_w in TMEM (bf16, 8 columns per 16 keys), B = V tile
   // (keys x D, D contiguous: MN-major; 64-element column blocks 16 KB apart).
-  auto issue_pv = [&](int w, int stage, bool accumulate) {
+  // Issued per half of the keys, each after its half of P is announced.
+  auto issue_pv_half = [&](int w, int stage, int half, bool accumulate) {
     const uint32_t va = sbase + L::kRingOff + stage * L::kTileBytes;
 #pragma unroll
-    for (int kk = 0; kk < kBN / 16; ++kk) {
+    for (int k4 = 0; k4 < kBN / 32; ++k4) {
+      const int kk = half * (kBN / 32) + k4;
       mma_ts(tmem + 256 + w * D, tmem + w * 128 + kk * 8,
              sw128_desc(va + kk * 16 * 128, kSwzBytes, 1024), kIdPV,
              (accumulate || kk > 0) ? 1u : 0u);
     }
+  };
+  auto wait_p = [&](int w, int half, int j) -> bool {
+    if (!mbar_wait(bars + 8 * (L::kBarPFull + 2 * w + half), static_cast<uint32_t>(j & 1),
+                   abort_flag, p.wait_limit_ns))
+      return false;
+    tc_fence_after();
+    return true;
   };
 
   if (!mbar_wait(bars + 8 * L::kBarQ, 0u, abort_flag, p.wait_limit_ns)) goto done;
@@ -322,11 +391,10 @@ __device__ __forceinline__ void prefill_mma(const PrefillParams& p, uint32_t sba
     if (!kv_wait(iv)) goto done;
     tc_fence_after();
     if (j < n_t[0]) {
-      if (!mbar_wait(bars + 8 * (L::kBarPFull + 0), static_cast<uint32_t>(j & 1), abort_flag,
-                     p.wait_limit_ns))
-        goto done;
-      tc_fence_after();
-      issue_pv(0, kv_stage(iv), j > 0);
+      if (!wait_p(0, 0, j)) goto done;
+      issue_pv_half(0, kv_stage(iv), 0, j > 0);
+      if (!wait_p(0, 1, j)) goto done;
+      issue_pv_half(0, kv_stage(iv), 1, j > 0);
       if (j == n_t[0] - 1) mma_commit(bars + 8 * (L::kBarOFull + 0));
     }
     const bool next = (j + 1 < n_max);
@@ -336,11 +404,10 @@ __device__ __forceinline__ void prefill_mma(const PrefillParams& p, uint32_t sba
       if (j + 1 < n_t[0]) { issue_s(0, kv_stage(ik)); mma_commit(bars + 8 * (L::kBarSFull + 0)); }
     }
     if (j < n_t[1]) {
-      if (!mbar_wait(bars + 8 * (L::kBarPFull + 1), static_cast<uint32_t>(j & 1), abort_flag,
-                     p.wait_limit_ns))
-        goto done;
-      tc_fence_after();
-      issue_pv(1, kv_stage(iv), j > 0);
+      if (!wait_p(1, 0, j)) goto done;
+      issue_pv_half(1, kv_stage(iv), 0, j > 0);
+      if (!wait_p(1, 1, j)) goto done;
+      issue_pv_half(1, kv_stage(iv), 1, j > 0);
       if (j == n_t[1] - 1) mma_commit(bars + 8 * (L::kBarOFull + 1));
     }
     mma_commit(bars + 8 * (L::kBarKvEmpty + kv_stage(iv)));
@@ -392,7 +459,8 @@ fa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(bars + 8 * (L::kBarSFull + w), 1);
-      mbar_init(bars + 8 * (L::kBarPFull + w), 128);
+      mbar_init(bars + 8 * (L::kBarPFull + 2 * w), 128);
+      mbar_init(bars + 8 * (L::kBarPFull + 2 * w + 1), 128);
       mbar_init(bars + 8 * (L::kBarOFull + w), 1);
     }
     mbar_init(bars + 8 * L::kBarDone, 1);
@@ -409,15 +477,19 @@ fa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlotOff);
 
   if (warp < 8) {
+    warpgroup_reg_alloc<kSoftmaxRegs>();
     const int w = warp >> 2;
-    prefill_softmax<D>(p, tmem, bars + 8 * (L::kBarSFull + w), bars + 8 * (L::kBarPFull + w),
+    prefill_softmax<D>(p, tmem, bars + 8 * (L::kBarSFull + w), bars + 8 * (L::kBarPFull + 2 * w),
                        bars + 8 * (L::kBarOFull + w), w, n_t[w], (2 * pair + w) * kBM, b, h,
                        abort_flag);
-  } else if (warp == 8) {
-    if (lane == 0)
-      prefill_producer<D>(&tm_q, &tm_k, &tm_v, p, sbase, pair, b, h, g, n_max, abort_flag);
-  } else if (warp == 9) {
-    if (lane == 0) prefill_mma<D>(p, sbase, tmem, n_t, n_max, abort_flag);
+  } else {
+    warpgroup_reg_dealloc<kControlRegs>();
+    if (warp == 8) {
+      if (lane == 0)
+        prefill_producer<D>(&tm_q, &tm_k, &tm_v, p, sbase, pair, b, h, g, n_max, abort_flag);
+    } else if (warp == 9) {
+      if (lane == 0) prefill_mma<D>(p, sbase, tmem, n_t, n_max, abort_flag);
+    }
   }
 
   tc_fence_before();
