@@ -53,9 +53,11 @@ bool encode_bhsd(CUtensorMap* map, const void* base, int d, int rows, long long 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// One-time per-device opt-in to the prefill kernels' dynamic shared memory.
+// One-time per-device opt-in to the prefill kernels' dynamic shared memory,
+// and the device's SM count (the persistent grid size).
 std::once_flag g_attr_once[kMaxDevices];
 cudaError_t g_attr_err[kMaxDevices];
+int g_prefill_sms[kMaxDevices];
 
 // The prefill kernel moves registers between its warpgroups (setmaxnreg);
 // that is only safe when every thread was launched with the register count
@@ -72,7 +74,8 @@ cudaError_t check_prefill_regs() {
 cudaError_t prepare_prefill(int dev) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::call_once(g_attr_once[dev], [dev] {
-    cudaError_t e = check_prefill_regs<64>();
+    cudaError_t e = cudaDeviceGetAttribute(&g_prefill_sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = check_prefill_regs<64>();
     if (e == cudaSuccess) e = check_prefill_regs<128>();
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(fa::fa_prefill_kernel<64>,
@@ -112,11 +115,13 @@ fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, f
   p.causal = causal ? 1 : 0;
   const int q_tiles = (Sq + fa::kBM - 1) / fa::kBM;
   p.n_qpairs = (q_tiles + 1) / 2;
+  p.n_items = p.n_qpairs * B * Hq;
   p.n_kv_tiles = (Skv + fa::kBN - 1) / fa::kBN;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_limit_ns = kWaitLimitNs;
-  const long long grid = static_cast<long long>(p.n_qpairs) * B * Hq;
+  const int sms = g_prefill_sms[dev] > 0 ? g_prefill_sms[dev] : 1;
+  const int grid = p.n_items < sms ? p.n_items : sms;  // persistent: one CTA per SM
   fa::fa_prefill_kernel<D><<<static_cast<unsigned>(grid), fa::kPrefillThreads,
                              fa::PrefillLayout<D>::kBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;

@@ -1,12 +1,16 @@
 // prefill_sm100.cuh -- fused exact-attention forward for sm_100a.
 //
-// One CTA owns two 128-row query tiles of one (batch, query head) and streams
-// the key/value tiles of that head's key/value head past them, so the score
-// matrix never leaves the SM ("I/O-Aware Kernels", section "FlashAttention":
+// A work item is two 128-row query tiles of one (batch, query head); the
+// key/value tiles of that head's key/value head stream past them, so the
+// score matrix never leaves the SM ("I/O-Aware Kernels", section "FlashAttention":
 // query blocks stay resident while K and V blocks stream through; "Tracing
 // Tiled QKV Data Movement in FlashAttention's Memory Hierarchy", section 2,
 // tiling plus online softmax).  The loop order is query-stationary: the
-// output tile is accumulated on chip and written to HBM once.
+// output tile is accumulated on chip and written to HBM once.  The kernel is
+// persistent: one CTA per SM walks the items longest first (under a causal
+// mask the last query tiles have the most keys), in a snake order over the
+// CTAs, so the next item's query load and first score MMAs overlap the
+// current item's last tiles and epilogue.
 //
 // Roles (384 threads, three warpgroups):
 //   warps 0-3  softmax warpgroup for query tile 0 (thread = row = TMEM lane)
@@ -15,7 +19,7 @@
 //   warp  9    MMA issuer: S_w = Q_w K_j^T and O_w += P_w V_j on tcgen05
 //   warps 10-11 idle
 // Registers are moved from the third warpgroup to the softmax warpgroups
-// (setmaxnreg): 224 + 224 + 56 per SM sub-partition = 3 x 168 at launch.
+// (setmaxnreg): 208 + 208 + 88 per SM sub-partition = 3 x 168 at launch.
 // Tensor memory (512 columns x 128 lanes x 32 bit):
 //   [0,128)   S_0 (fp32 scores); P_0 (bf16) overwrites its first 64 columns
 //   [128,256) S_1 / P_1
@@ -40,8 +44,8 @@ constexpr int kBM = 128;       // query rows per tile (= TMEM lanes)
 constexpr int kBN = 128;       // keys per key/value tile
 constexpr int kPrefillThreads = 384;
 constexpr int kPrefillLaunchRegs = 168;   // 65536 / 384, rounded down to a multiple of 8
-constexpr int kSoftmaxRegs = 224;
-constexpr int kControlRegs = 56;
+constexpr int kSoftmaxRegs = 208;
+constexpr int kControlRegs = 88;
 static_assert(2 * kSoftmaxRegs + kControlRegs <= 3 * kPrefillLaunchRegs,
               "register split exceeds the launch budget");
 constexpr int kSwzBytes = 128 * 128;  // one 128-row x 64-element bf16 box, 128B swizzled
@@ -80,6 +84,7 @@ struct PrefillParams {
   int B, Hq, Hkv, Sq, Skv, group;
   int causal;
   int n_qpairs;    // ceil(ceil(Sq / 128) / 2)
+  int n_items;     // n_qpairs * B * Hq
   int n_kv_tiles;  // ceil(Skv / 128)
   float scale;     // natural units
   float scale_log2;
@@ -93,7 +98,8 @@ struct PrefillLayout {
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = 2 * kTileBytes;
   static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
-  // q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2][2 halves], o_full[2], mma_done
+  // q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2][2 halves], o_full[2], mma_done,
+  // q_empty
   static constexpr int kBarQ = 0;
   static constexpr int kBarKvFull = 1;
   static constexpr int kBarKvEmpty = 1 + kStages;
@@ -101,7 +107,8 @@ struct PrefillLayout {
   static constexpr int kBarPFull = kBarSFull + 2;
   static constexpr int kBarOFull = kBarPFull + 4;
   static constexpr int kBarDone = kBarOFull + 2;
-  static constexpr int kNumBars = kBarDone + 1;
+  static constexpr int kBarQEmpty = kBarDone + 1;
+  static constexpr int kNumBars = kBarQEmpty + 1;
   static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kAbortOff = kTmemSlotOff + 4;
   static constexpr int kBytes = kAbortOff + 4 + 1024;  // + slack for 1024-byte alignment
@@ -117,22 +124,57 @@ __device__ __forceinline__ int prefill_tiles_for(const PrefillParams& p, int r0)
   return min(p.n_kv_tiles, static_cast<int>(last_key / kBN) + 1);
 }
 
+struct PrefillItem {
+  int pair, b, h, g, n0, n1;
+};
+
+// Item k in longest-first order: pairs of query tiles in descending order
+// under a causal mask, heads of one key/value group adjacent.
+__device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int k) {
+  PrefillItem it;
+  const int bh_count = p.B * p.Hq;
+  it.pair = k / bh_count;
+  if (p.causal) it.pair = p.n_qpairs - 1 - it.pair;
+  const int bh = k % bh_count;
+  it.b = bh / p.Hq;
+  it.h = bh % p.Hq;
+  it.g = it.h / p.group;
+  it.n0 = prefill_tiles_for(p, (2 * it.pair) * kBM);
+  it.n1 = prefill_tiles_for(p, (2 * it.pair + 1) * kBM);
+  return it;
+}
+
+// The item this CTA takes in round r (snake order over the CTAs), or -1.
+__device__ __forceinline__ int prefill_item_index(const PrefillParams& p, int r) {
+  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  const long long k = static_cast<long long>(r) * G + ((r & 1) ? (G - 1 - c) : c);
+  return k < p.n_items ? static_cast<int>(k) : -1;
+}
+
 // ---------------------------------------------------------------------------
 // Softmax warpgroup: one thread per query row.
 // ---------------------------------------------------------------------------
 template <int D>
 __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t tmem,
                                                 uint32_t bar_s, uint32_t bar_p, uint32_t bar_o,
-                                                int w, int n_tiles, int q_row0, int b, int h,
-                                                volatile int* abort_flag) {
+                                                int w, volatile int* abort_flag) {
   const int warp_in_wg = (threadIdx.x >> 5) & 3;
   const int row_in_tile = warp_in_wg * 32 + (threadIdx.x & 31);
-  const int row = q_row0 + row_in_tile;
   const uint32_t lane_off = static_cast<uint32_t>(warp_in_wg * 32) << 16;
   const uint32_t tS = tmem + lane_off + static_cast<uint32_t>(w * 128);
   const uint32_t tO = tmem + lane_off + static_cast<uint32_t>(256 + w * D);
   const float c = p.scale_log2;
   const int off = p.Skv - p.Sq;
+  uint32_t tcount = 0;  // tiles this warpgroup has processed (phase of s_full / p_full)
+  uint32_t ocount = 0;  // items this warpgroup has finished with tiles (phase of o_full)
+
+  for (int r = 0;; ++r) {
+  const int k_item = prefill_item_index(p, r);
+  if (k_item < 0) break;
+  const PrefillItem item = prefill_item(p, k_item);
+  const int n_tiles = w ? item.n1 : item.n0;
+  const int q_row0 = (2 * item.pair + w) * kBM;
+  const int row = q_row0 + row_in_tile;
   // keys with index > last_key are masked for this row
   const long long last_key_ll = p.causal ? static_cast<long long>(row) + off
                                          : static_cast<long long>(p.Skv) - 1;
@@ -140,7 +182,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
 
   float m = -INFINITY;
   float l = 0.f;
-  const size_t row_index = (static_cast<size_t>(b) * p.Hq + h) * p.Sq + row;
+  const size_t row_index = (static_cast<size_t>(item.b) * p.Hq + item.h) * p.Sq + row;
 
   if (n_tiles == 0) {
     if (row < p.Sq) {
@@ -149,11 +191,11 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
       for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
       p.lse[row_index] = -INFINITY;
     }
-    return;
+    continue;
   }
 
-  for (int j = 0; j < n_tiles; ++j) {
-    bool ok = mbar_wait(bar_s, static_cast<uint32_t>(j & 1), abort_flag, p.wait_limit_ns);
+  for (int j = 0; j < n_tiles; ++j, ++tcount) {
+    bool ok = mbar_wait(bar_s, tcount & 1u, abort_flag, p.wait_limit_ns);
     if (!__all_sync(0xffffffffu, ok)) return;
     tc_fence_after();
 
@@ -257,7 +299,8 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
   }
 
   // epilogue: O / l -> bf16, LSE = m*scale + ln l
-  bool ok = mbar_wait(bar_o, 0u, abort_flag, p.wait_limit_ns);
+  bool ok = mbar_wait(bar_o, ocount & 1u, abort_flag, p.wait_limit_ns);
+  ++ocount;
   if (!__all_sync(0xffffffffu, ok)) return;
   tc_fence_after();
   const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
@@ -279,6 +322,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
     }
   }
   if (row < p.Sq) p.lse[row_index] = (l > 0.f) ? m * p.scale + logf(l) : -INFINITY;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -287,45 +331,56 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
 template <int D>
 __device__ __forceinline__ void prefill_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                                                  const CUtensorMap* tm_v, const PrefillParams& p,
-                                                 uint32_t sbase, int pair, int b, int h, int g,
-                                                 int n_max, volatile int* abort_flag) {
+                                                 uint32_t sbase, volatile int* abort_flag) {
   using L = PrefillLayout<D>;
   const uint32_t bars = sbase + L::kBarOff;
   tma_prefetch_desc(tm_q);
   tma_prefetch_desc(tm_k);
   tma_prefetch_desc(tm_v);
-
   const uint32_t bar_q = bars + 8 * L::kBarQ;
-  mbar_arrive_expect_tx(bar_q, 2 * L::kTileBytes);
-#pragma unroll
-  for (int w = 0; w < 2; ++w)
-#pragma unroll
-    for (int kb = 0; kb < D / 64; ++kb)
-      tma_load_3d(sbase + L::kQOff + w * L::kTileBytes + kb * kSwzBytes, tm_q, bar_q, kb * 64,
-                  (2 * pair + w) * kBM, b * p.Hq + h);
-
-  int issued = 0;
-  for (int idx = 0; idx < 2 * n_max; ++idx) {
-    const int stage = idx % L::kStages;
-    const uint32_t round = static_cast<uint32_t>(idx / L::kStages);
-    if (!mbar_wait(bars + 8 * (L::kBarKvEmpty + stage), (round & 1u) ^ 1u, abort_flag,
-                   p.wait_limit_ns))
+  uint32_t nq = 0;  // query loads issued (one per item)
+  uint32_t ld = 0;  // key/value tile loads issued
+  bool stop = false;
+  for (int r = 0; !stop; ++r) {
+    const int k_item = prefill_item_index(p, r);
+    if (k_item < 0) break;
+    const PrefillItem item = prefill_item(p, k_item);
+    // The query buffer is free once the previous item's last score MMA is done.
+    if (nq > 0 && !mbar_wait(bars + 8 * L::kBarQEmpty, (nq - 1) & 1u, abort_flag,
+                             p.wait_limit_ns))
       break;
-    const uint32_t bar_full = bars + 8 * (L::kBarKvFull + stage);
-    mbar_arrive_expect_tx(bar_full, L::kTileBytes);
-    const CUtensorMap* tm = (idx & 1) ? tm_v : tm_k;
+    mbar_arrive_expect_tx(bar_q, 2 * L::kTileBytes);
 #pragma unroll
-    for (int kb = 0; kb < D / 64; ++kb)
-      tma_load_3d(sbase + L::kRingOff + stage * L::kTileBytes + kb * kSwzBytes, tm, bar_full,
-                  kb * 64, (idx >> 1) * kBN, b * p.Hkv + g);
-    issued = idx + 1;
+    for (int w = 0; w < 2; ++w)
+#pragma unroll
+      for (int kb = 0; kb < D / 64; ++kb)
+        tma_load_3d(sbase + L::kQOff + w * L::kTileBytes + kb * kSwzBytes, tm_q, bar_q, kb * 64,
+                    (2 * item.pair + w) * kBM, item.b * p.Hq + item.h);
+    ++nq;
+    const int n_max = max(item.n0, item.n1);
+    for (int idx = 0; idx < 2 * n_max; ++idx) {
+      const uint32_t stage = ld % L::kStages;
+      if (!mbar_wait(bars + 8 * (L::kBarKvEmpty + stage), ((ld / L::kStages) & 1u) ^ 1u,
+                     abort_flag, p.wait_limit_ns)) {
+        stop = true;
+        break;
+      }
+      const uint32_t bar_full = bars + 8 * (L::kBarKvFull + stage);
+      mbar_arrive_expect_tx(bar_full, L::kTileBytes);
+      const CUtensorMap* tm = (idx & 1) ? tm_v : tm_k;
+#pragma unroll
+      for (int kb = 0; kb < D / 64; ++kb)
+        tma_load_3d(sbase + L::kRingOff + stage * L::kTileBytes + kb * kSwzBytes, tm, bar_full,
+                    kb * 64, (idx >> 1) * kBN, item.b * p.Hkv + item.g);
+      ++ld;
+    }
   }
 
   // Drain: no copy may still be in flight when the CTA exits.
-  mbar_wait(bar_q, 0u, nullptr, p.wait_limit_ns);
-  for (int idx = (issued > L::kStages ? issued - L::kStages : 0); idx < issued; ++idx)
-    mbar_wait(bars + 8 * (L::kBarKvFull + idx % L::kStages),
-              static_cast<uint32_t>(idx / L::kStages) & 1u, nullptr, p.wait_limit_ns);
+  if (nq > 0) mbar_wait(bar_q, (nq - 1) & 1u, nullptr, p.wait_limit_ns);
+  const uint32_t S = static_cast<uint32_t>(L::kStages);
+  for (uint32_t k = (ld > S ? ld - S : 0u); k < ld; ++k)
+    mbar_wait(bars + 8 * (L::kBarKvFull + k % S), (k / S) & 1u, nullptr, p.wait_limit_ns);
 }
 
 // ---------------------------------------------------------------------------
@@ -333,15 +388,14 @@ __device__ __forceinline__ void prefill_producer(const CUtensorMap* tm_q, const 
 // ---------------------------------------------------------------------------
 template <int D>
 __device__ __forceinline__ void prefill_mma(const PrefillParams& p, uint32_t sbase, uint32_t tmem,
-                                            const int (&n_t)[2], int n_max,
                                             volatile int* abort_flag) {
   using L = PrefillLayout<D>;
   const uint32_t bars = sbase + L::kBarOff;
   constexpr uint32_t kIdS = idesc_bf16_f32(kBM, kBN, false);
   constexpr uint32_t kIdPV = idesc_bf16_f32(kBM, D, true);
 
-  auto kv_stage = [](int idx) { return idx % L::kStages; };
-  auto kv_wait = [&](int idx) -> bool {
+  auto kv_stage = [](uint32_t idx) { return static_cast<int>(idx % L::kStages); };
+  auto kv_wait = [&](uint32_t idx) -> bool {
     return mbar_wait(bars + 8 * (L::kBarKvFull + kv_stage(idx)),
                      static_cast<uint32_t>(idx / L::kStages) & 1u, abort_flag, p.wait_limit_ns);
   };
@@ -369,51 +423,71 @@ __device__ __forceinline__ void prefill_mma(const PrefillParams& p, uint32_t sba
              (accumulate || kk > 0) ? 1u : 0u);
     }
   };
-  auto wait_p = [&](int w, int half, int j) -> bool {
-    if (!mbar_wait(bars + 8 * (L::kBarPFull + 2 * w + half), static_cast<uint32_t>(j & 1),
+  auto wait_p = [&](int w, int half, uint32_t cnt) -> bool {
+    if (!mbar_wait(bars + 8 * (L::kBarPFull + 2 * w + half), cnt & 1u,
                    abort_flag, p.wait_limit_ns))
       return false;
     tc_fence_after();
     return true;
   };
 
-  if (!mbar_wait(bars + 8 * L::kBarQ, 0u, abort_flag, p.wait_limit_ns)) goto done;
-  if (n_max == 0) goto done;
-
-  if (!kv_wait(0)) goto done;
-  tc_fence_after();
-  if (n_t[0] > 0) { issue_s(0, kv_stage(0)); mma_commit(bars + 8 * (L::kBarSFull + 0)); }
-  if (n_t[1] > 0) { issue_s(1, kv_stage(0)); mma_commit(bars + 8 * (L::kBarSFull + 1)); }
-  mma_commit(bars + 8 * (L::kBarKvEmpty + kv_stage(0)));
-
-  for (int j = 0; j < n_max; ++j) {
-    const int iv = 2 * j + 1, ik = 2 * j + 2;
-    if (!kv_wait(iv)) goto done;
-    tc_fence_after();
-    if (j < n_t[0]) {
-      if (!wait_p(0, 0, j)) goto done;
-      issue_pv_half(0, kv_stage(iv), 0, j > 0);
-      if (!wait_p(0, 1, j)) goto done;
-      issue_pv_half(0, kv_stage(iv), 1, j > 0);
-      if (j == n_t[0] - 1) mma_commit(bars + 8 * (L::kBarOFull + 0));
-    }
-    const bool next = (j + 1 < n_max);
-    if (next) {
-      if (!kv_wait(ik)) goto done;
+  {
+    uint32_t nq = 0;                 // items started (phase of q_full / q_empty)
+    uint32_t base = 0;               // ring index of the current item's first K tile
+    uint32_t pc[2] = {0u, 0u};       // tiles of each query tile consumed (phase of p_full)
+    for (int r = 0;; ++r) {
+      const int k_item = prefill_item_index(p, r);
+      if (k_item < 0) break;
+      const PrefillItem item = prefill_item(p, k_item);
+      if (!mbar_wait(bars + 8 * L::kBarQ, nq & 1u, abort_flag, p.wait_limit_ns)) goto done;
+      ++nq;
+      const int n0 = item.n0, n1 = item.n1;
+      const int n_max = max(n0, n1);
+      if (n_max == 0) {
+        mma_commit(bars + 8 * L::kBarQEmpty);
+        continue;
+      }
+      if (!kv_wait(base)) goto done;
       tc_fence_after();
-      if (j + 1 < n_t[0]) { issue_s(0, kv_stage(ik)); mma_commit(bars + 8 * (L::kBarSFull + 0)); }
-    }
-    if (j < n_t[1]) {
-      if (!wait_p(1, 0, j)) goto done;
-      issue_pv_half(1, kv_stage(iv), 0, j > 0);
-      if (!wait_p(1, 1, j)) goto done;
-      issue_pv_half(1, kv_stage(iv), 1, j > 0);
-      if (j == n_t[1] - 1) mma_commit(bars + 8 * (L::kBarOFull + 1));
-    }
-    mma_commit(bars + 8 * (L::kBarKvEmpty + kv_stage(iv)));
-    if (next) {
-      if (j + 1 < n_t[1]) { issue_s(1, kv_stage(ik)); mma_commit(bars + 8 * (L::kBarSFull + 1)); }
-      mma_commit(bars + 8 * (L::kBarKvEmpty + kv_stage(ik)));
+      if (n0 > 0) { issue_s(0, kv_stage(base)); mma_commit(bars + 8 * (L::kBarSFull + 0)); }
+      if (n1 > 0) { issue_s(1, kv_stage(base)); mma_commit(bars + 8 * (L::kBarSFull + 1)); }
+      mma_commit(bars + 8 * (L::kBarKvEmpty + kv_stage(base)));
+      if (n_max == 1) mma_commit(bars + 8 * L::kBarQEmpty);  // last score MMA of the item
+
+      for (int j = 0; j < n_max; ++j) {
+        const uint32_t iv = base + 2 * j + 1, ik = base + 2 * j + 2;
+        if (!kv_wait(iv)) goto done;
+        tc_fence_after();
+        if (j < n0) {
+          if (!wait_p(0, 0, pc[0])) goto done;
+          issue_pv_half(0, kv_stage(iv), 0, j > 0);
+          if (!wait_p(0, 1, pc[0])) goto done;
+          issue_pv_half(0, kv_stage(iv), 1, j > 0);
+          ++pc[0];
+          if (j == n0 - 1) mma_commit(bars + 8 * (L::kBarOFull + 0));
+        }
+        const bool next = (j + 1 < n_max);
+        if (next) {
+          if (!kv_wait(ik)) goto done;
+          tc_fence_after();
+          if (j + 1 < n0) { issue_s(0, kv_stage(ik)); mma_commit(bars + 8 * (L::kBarSFull + 0)); }
+        }
+        if (j < n1) {
+          if (!wait_p(1, 0, pc[1])) goto done;
+          issue_pv_half(1, kv_stage(iv), 0, j > 0);
+          if (!wait_p(1, 1, pc[1])) goto done;
+          issue_pv_half(1, kv_stage(iv), 1, j > 0);
+          ++pc[1];
+          if (j == n1 - 1) mma_commit(bars + 8 * (L::kBarOFull + 1));
+        }
+        mma_commit(bars + 8 * (L::kBarKvEmpty + kv_stage(iv)));
+        if (next) {
+          if (j + 1 < n1) { issue_s(1, kv_stage(ik)); mma_commit(bars + 8 * (L::kBarSFull + 1)); }
+          mma_commit(bars + 8 * (L::kBarKvEmpty + kv_stage(ik)));
+          if (j + 2 == n_max) mma_commit(bars + 8 * L::kBarQEmpty);  // last score MMA
+        }
+      }
+      base += 2 * static_cast<uint32_t>(n_max);
     }
   }
 done:
@@ -435,20 +509,6 @@ fa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Work item: the query-tile pair index is reversed under a causal mask so
-  // the longest items start first.
-  const int bh_count = p.B * p.Hq;
-  int pair = static_cast<int>(blockIdx.x) / bh_count;
-  const int bh = static_cast<int>(blockIdx.x) % bh_count;
-  if (p.causal) pair = p.n_qpairs - 1 - pair;
-  const int b = bh / p.Hq;
-  const int h = bh % p.Hq;
-  const int g = h / p.group;
-  int n_t[2];
-  n_t[0] = prefill_tiles_for(p, (2 * pair) * kBM);
-  n_t[1] = prefill_tiles_for(p, (2 * pair + 1) * kBM);
-  const int n_max = max(n_t[0], n_t[1]);
-
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbortOff);
   const uint32_t bars = sbase + L::kBarOff;
   if (threadIdx.x == 0) {
@@ -464,6 +524,7 @@ fa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       mbar_init(bars + 8 * (L::kBarOFull + w), 1);
     }
     mbar_init(bars + 8 * L::kBarDone, 1);
+    mbar_init(bars + 8 * L::kBarQEmpty, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -480,15 +541,14 @@ fa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     warpgroup_reg_alloc<kSoftmaxRegs>();
     const int w = warp >> 2;
     prefill_softmax<D>(p, tmem, bars + 8 * (L::kBarSFull + w), bars + 8 * (L::kBarPFull + 2 * w),
-                       bars + 8 * (L::kBarOFull + w), w, n_t[w], (2 * pair + w) * kBM, b, h,
-                       abort_flag);
+                       bars + 8 * (L::kBarOFull + w), w, abort_flag);
   } else {
     warpgroup_reg_dealloc<kControlRegs>();
     if (warp == 8) {
       if (lane == 0)
-        prefill_producer<D>(&tm_q, &tm_k, &tm_v, p, sbase, pair, b, h, g, n_max, abort_flag);
+        prefill_producer<D>(&tm_q, &tm_k, &tm_v, p, sbase, abort_flag);
     } else if (warp == 9) {
-      if (lane == 0) prefill_mma<D>(p, sbase, tmem, n_t, n_max, abort_flag);
+      if (lane == 0) prefill_mma<D>(p, sbase, tmem, abort_flag);
     }
   }
 
