@@ -178,12 +178,24 @@ def dist_setup(args):
 
 
 def max_over_ranks(values, world):
+    """Element-wise max of per-rank timings (the slowest rank sets the time)."""
     if world == 1:
         return list(values)
     import torch.distributed as dist
-    t = torch.tensor(values, dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor(values, dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return t.tolist()
+
+
+def rank_seed(seed, rank):
+    """Each rank draws its own inputs (independent replicas, weak scaling)."""
+    return seed + 1000 * rank
+
+
+def aggregate_rate(world, work_per_step, steps, max_ms):
+    """Whole-job throughput: the work all ranks did over the slowest rank's time."""
+    return world * work_per_step * steps / (max_ms * 1e-3)
 
 
 def barrier(world):
@@ -285,9 +297,8 @@ def run_ours(args, world, rank, local):
 
     c = CONFIGS[args.workload]
     cd = CONFIGS[DECODE_WORKLOAD]
-    seed_off = 1000 * rank
-    q, k, v = prefill_inputs(c.B, c.Hq, c.Hkv, c.Sq, c.Skv, c.d, c.seed + seed_off, c.q_mult,
-                             device=dev)
+    q, k, v = prefill_inputs(c.B, c.Hq, c.Hkv, c.Sq, c.Skv, c.d, rank_seed(c.seed, rank),
+                             c.q_mult, device=dev)
     o = torch.empty_like(q)
     lse = torch.empty((c.B, c.Hq, c.Sq), device=dev, dtype=torch.float32)
     if do_dec:
@@ -296,7 +307,7 @@ def run_ours(args, world, rank, local):
             cd = dataclasses.replace(cd, B=args.decode_batch,
                                      name="%s_b%d" % (cd.name, args.decode_batch))
         qd, kc, vc, sl = decode_inputs(cd.B, cd.Hq, cd.Hkv, cd.Lmin, cd.Lmax, cd.d,
-                                       cd.seed + seed_off, device=dev)
+                                       rank_seed(cd.seed, rank), device=dev)
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
         n_split = args.decode_splits or fa.decode_default_splits(cd.B, cd.Hkv, cd.Lmax, sms)
         op = torch.empty((cd.B, cd.Hq, n_split, cd.d), device=dev, dtype=torch.float32)
@@ -339,8 +350,8 @@ def run_ours(args, world, rank, local):
     pre_ms, dec_ms, tot_ms = max_over_ranks([pre_ms, dec_ms, pre_ms + dec_ms], world)
     K = args.steps
     flops = c.flops()
-    prefill_tflops = world * flops * K / (pre_ms * 1e-3) / 1e12 if do_pre else None
-    dec_gbs = world * dec_bytes * K / (dec_ms * 1e-3) / 1e9 if do_dec else None
+    prefill_tflops = aggregate_rate(world, flops, K, pre_ms) / 1e12 if do_pre else None
+    dec_gbs = aggregate_rate(world, dec_bytes, K, dec_ms) / 1e9 if do_dec else None
 
     # e2e: the user-level call with pinned host buffers, copies inside the region
     e2e = None
@@ -363,7 +374,7 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize(dev)
         barrier(world)
         e2e_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in e2e_evs)], world)[0]
-        e2e = {"value": world * flops * K / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": aggregate_rate(world, flops, K, e2e_ms) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": int((q.numel() + k.numel() + v.numel()) * 2),
                "d2h_bytes_per_step": int(o.numel() * 2 + lse.numel() * 4),
                "api": "io_aware_exact_flashattention_b200.flash_attention (host tensors)"}

@@ -150,6 +150,15 @@ fa_status fa_get_device_status(void);
 fa_status fa_debug_timeout_probe(unsigned int limit_us, fa_stream_t stream);
 
 /*
+ * Test hook for the polynomial 2^x that the prefill kernel evaluates on the
+ * FMA pipe for part of its softmax (the rest uses the hardware exp2):
+ * y[i] = 2^n * p(x[i] - n), n = round(x[i]), p the degree-3 minimax fit of
+ * 2^f on [-1/2, 1/2] (arguments clamped to >= -126).  x and y are device
+ * arrays of n floats (16-byte aligned); n >= 0.  Enqueued on stream.
+ */
+fa_status fa_debug_exp2_poly(const float *x, float *y, int n, fa_stream_t stream);
+
+/*
  * fa_decode_noalloc -- single-query decode that allocates nothing.
  *
  * The pages have no counterpart to this call.  It computes exactly what

@@ -273,6 +273,17 @@ cudaError_t noalloc_scratch_address(int dev, void** addr) {
   return cudaSuccess;
 }
 
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const float2 r = fa::exp2_poly2(make_float2(x[i], x[i + 1]));
+    y[i] = r.x;
+    y[i + 1] = r.y;
+  } else if (i < n) {
+    y[i] = fa::exp2_poly2(make_float2(x[i], 0.f)).x;
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -395,6 +406,16 @@ fa_status fa_get_device_status(void) {
       return FA_ERR_CUDA;
   }
   return static_cast<fa_status>(v);
+}
+
+fa_status fa_debug_exp2_poly(const float* x, float* y, int n, fa_stream_t stream) {
+  if (n < 0) return FA_ERR_INVALID_ARG;
+  if (n == 0) return FA_OK;
+  if (x == nullptr || y == nullptr) return FA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return FA_ERR_ALIGNMENT;
+  const int pairs = (n + 1) / 2;
+  exp2_poly_kernel<<<(pairs + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 fa_status fa_debug_timeout_probe(unsigned int limit_us, fa_stream_t stream) {

@@ -39,6 +39,7 @@ SIGNATURES = {
     "fa_get_device_status": (_I, []),
     "fa_debug_timeout_probe": (_I, [ctypes.c_uint, _VP]),
     "fa_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP]),
+    "fa_debug_exp2_poly": (_I, [_VP, _VP, _I, _VP]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -159,6 +160,15 @@ def decode_default_splits(B: int, Hkv: int, Lmax: int, num_sms: int) -> int:
 def get_device_status() -> int:
     """Read and clear the device status word (synchronises the device)."""
     return int(lib().fa_get_device_status())
+
+
+def debug_exp2_poly(x: torch.Tensor) -> torch.Tensor:
+    """The prefill kernel's polynomial 2^x on device (test hook)."""
+    _need(x, torch.float32, "x")
+    y = torch.empty_like(x)
+    _check("fa_debug_exp2_poly", lib().fa_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(),
+                                                           _stream_ptr(None)))
+    return y
 
 
 def debug_timeout_probe(limit_us: int, stream: Optional[torch.cuda.Stream] = None) -> None:
