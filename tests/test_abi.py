@@ -24,7 +24,7 @@ def lib():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(fa_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_expected_calls():
@@ -37,7 +37,7 @@ def test_header_declares_expected_calls():
 def test_library_exports_every_declared_symbol(lib):
     out = subprocess.run(["nm", "-D", "--defined-only", fa.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
-    exported = set(re.findall(r"\bT (fa_[a-z_]+)\b", out))
+    exported = set(re.findall(r"\bT (fa_[a-z0-9_]+)\b", out))
     missing = set(declared_functions()) - exported
     assert not missing, "not exported: %s" % sorted(missing)
 
