@@ -105,6 +105,7 @@ fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, f
 
   fa::PrefillParams p;
   p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_align32 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0;
   p.lse = lse;
   p.B = B;
   p.Hq = Hq;

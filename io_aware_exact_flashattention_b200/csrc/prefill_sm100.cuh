@@ -27,10 +27,12 @@
 // Online softmax ("FlashAttention & IO-aware attention", section "Direct
 // answer"): each row keeps a running max m and sum l; when the max grows the
 // accumulated l and O are multiplied by e^(m - m_new).  Here the reference max
-// only moves when it grows by more than 2^8 in the exponent, so the rescale
-// of O is rare; the result is unchanged because the final O / l and LSE use
-// the same reference max.  Exponentials are 2^x on scores pre-multiplied by
-// scale*log2(e).
+// only moves when it grows by more than 2^24 in the exponent, so the rescale
+// of O (a round trip of O through registers) is rare even for logits spread
+// over tens of binades; the result is unchanged because the final O / l and
+// LSE use the same reference max.  p <= 2^24 loses nothing: bf16 P and the
+// fp32 l and O round relative to magnitude and have ~2^100 of headroom.
+// Exponentials are 2^x on scores pre-multiplied by scale*log2(e).
 #pragma once
 
 #include <climits>
@@ -49,14 +51,14 @@ constexpr int kControlRegs = 88;
 static_assert(2 * kSoftmaxRegs + kControlRegs <= 3 * kPrefillLaunchRegs,
               "register split exceeds the launch budget");
 constexpr int kSwzBytes = 128 * 128;  // one 128-row x 64-element bf16 box, 128B swizzled
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr float kRescaleThreshold = 24.0f;  // log2 units
 
 // 2^x for part of the softmax on the FMA pipe instead of the MUFU: with
 // n = round(x) and f = x - n in [-1/2, 1/2], 2^x = 2^n * p(f) where p is the
 // degree-3 minimax fit of 2^f below (max relative error 7.5e-5; derived by
 // exp2_poly_fit.py next to this file).  2^n is applied by adding n to the
-// exponent field.  Arguments are clamped to >= -126; larger ones stay <= 8
-// because the reference max is never more than 2^8 below the row max.
+// exponent field.  Arguments are clamped to >= -126; larger ones stay <= 24
+// because the reference max is never more than 2^24 below the row max.
 constexpr float kExp2C0 = 9.999280572e-01f;
 constexpr float kExp2C1 = 6.932609677e-01f;
 constexpr float kExp2C2 = 2.426111251e-01f;
@@ -89,6 +91,7 @@ struct PrefillParams {
   float scale;     // natural units
   float scale_log2;
   unsigned long long wait_limit_ns;
+  int o_align32;   // o is 32-byte aligned: 32-byte stores in the epilogue
 };
 
 template <int D>
@@ -304,20 +307,27 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
   if (!__all_sync(0xffffffffu, ok)) return;
   tc_fence_after();
   const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-  uint4* dst = reinterpret_cast<uint4*>(p.o + row_index * D);
-#pragma unroll
-  for (int q4 = 0; q4 < D / 32; ++q4) {
-    uint32_t r[32];
-    tmem_ld32(tO + q4 * 32, r);
+  {
+    uint32_t r[D];
+    tmem_ld_row<D>(tO, r);
     if (row < p.Sq) {
+      uint8_t* dst = reinterpret_cast<uint8_t*>(p.o + row_index * D);
+      const float2 il = make_float2(inv_l, inv_l);
 #pragma unroll
-      for (int v4 = 0; v4 < 4; ++v4) {
-        uint4 pkt;
-        pkt.x = pack_bf16x2(__uint_as_float(r[v4 * 8 + 0]) * inv_l, __uint_as_float(r[v4 * 8 + 1]) * inv_l);
-        pkt.y = pack_bf16x2(__uint_as_float(r[v4 * 8 + 2]) * inv_l, __uint_as_float(r[v4 * 8 + 3]) * inv_l);
-        pkt.z = pack_bf16x2(__uint_as_float(r[v4 * 8 + 4]) * inv_l, __uint_as_float(r[v4 * 8 + 5]) * inv_l);
-        pkt.w = pack_bf16x2(__uint_as_float(r[v4 * 8 + 6]) * inv_l, __uint_as_float(r[v4 * 8 + 7]) * inv_l);
-        dst[q4 * 4 + v4] = pkt;
+      for (int c = 0; c < D / 16; ++c) {
+        uint32_t w8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float2 x = fmul2(make_float2(__uint_as_float(r[16 * c + 2 * e]),
+                                             __uint_as_float(r[16 * c + 2 * e + 1])), il);
+          w8[e] = pack_bf16x2(x.x, x.y);
+        }
+        if (p.o_align32) {
+          st_global_v8(dst + 32 * c, w8);
+        } else {
+          reinterpret_cast<uint4*>(dst + 32 * c)[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+          reinterpret_cast<uint4*>(dst + 32 * c)[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+        }
       }
     }
   }

@@ -140,6 +140,25 @@ def test_guard_bytes_untouched_and_deterministic():
     assert torch.equal(o1, o) and torch.equal(l1, lse), "two runs differ"
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_output_only_16_byte_aligned(d):
+    """O rows are written with 32-byte stores when o is 32-byte aligned and
+    with 16-byte stores otherwise; both give the same bytes and stay inside
+    the output."""
+    q, k, v = prefill_inputs(1, 4, 2, 300, 300, d, 15, device="cuda")
+    n = q.numel()
+    guard = 4096
+    o32, l32 = run_fa(q, k, v, True, 0.1)
+    obuf = torch.full((n + 2 * guard,), 3.0, device="cuda", dtype=torch.bfloat16)
+    o16 = obuf[guard + 8:guard + 8 + n].view(q.shape)  # 16 bytes past a 32-byte boundary
+    assert o16.data_ptr() % 32 == 16
+    l16 = torch.empty_like(l32)
+    fa.fa_fwd(q, k, v, o16, l16, True, 0.1)
+    torch.cuda.synchronize()
+    assert torch.equal(o32, o16) and torch.equal(l32, l16)
+    assert (obuf[:guard + 8] == 3.0).all() and (obuf[guard + 8 + n:] == 3.0).all()
+
+
 def test_non_default_stream():
     q, k, v = prefill_inputs(2, 4, 4, 256, 256, 64, 9, device="cuda")
     s = torch.cuda.Stream()
