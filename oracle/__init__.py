@@ -9,7 +9,9 @@ that file with gcc and marshals numpy arrays through ctypes.
 What it computes (see ``attn_oracle.c`` for the per-function citations):
 the one-shot, materialising softmax attention of "I/O-Aware Kernels", section
 "The Memory Bottleneck", with scores scaled as in "FlashAttention & IO-aware
-attention", section "Code", and LSE = max + ln(sum of exp).
+attention", section "Code", and LSE = max + ln(sum of exp).  A paged cache is
+read through its block table by ``paged_gather`` (plain index loops, no
+arithmetic) and then decoded like a contiguous one.
 
 Parity pins (tests/test_oracle_pins.py): closed-form golden cases, an
 independent online-softmax recurrence, invariants, torch fp64 SDPA on small
@@ -69,6 +71,9 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_split_partials.argtypes = ([_D, _D, _D, _I32, _D, _D] + [ci] * 6
                                           + [ctypes.c_double])
     lib.oracle_split_partials.restype = ci
+    lib.oracle_split_partials_aligned.argtypes = ([_D, _D, _D, _I32, _D, _D] + [ci] * 7
+                                                  + [ctypes.c_double])
+    lib.oracle_split_partials_aligned.restype = ci
     lib.oracle_combine.argtypes = [_D, _D, _D, _D] + [ci] * 4
     lib.oracle_combine.restype = ci
     lib.oracle_num_threads.argtypes = []
@@ -157,6 +162,61 @@ def split_partials(q, k_cache, v_cache, seqlens, num_splits: int, scale: float,
     if rc != 0:
         raise ValueError("oracle_split_partials rejected its arguments")
     return o, lse
+
+
+def split_partials_aligned(q, k_cache, v_cache, seqlens, num_splits: int, align: int,
+                           scale: float, lib: Optional[ctypes.CDLL] = None):
+    """Split partials with chunk sizes rounded up to a multiple of ``align``."""
+    lib = lib or load()
+    q, kc, vc = _f64(q), _f64(k_cache), _f64(v_cache)
+    sl = np.ascontiguousarray(np.asarray(
+        seqlens.cpu().numpy() if hasattr(seqlens, "cpu") else seqlens, dtype=np.int32))
+    B, Hq, d = q.shape
+    _, Hkv, Lmax, _ = kc.shape
+    o = np.zeros((B, Hq, num_splits, d))
+    lse = np.zeros((B, Hq, num_splits))
+    rc = lib.oracle_split_partials_aligned(_p(q), _p(kc), _p(vc), _p(sl, _I32), _p(o), _p(lse),
+                                           B, Hq, Hkv, Lmax, d, int(num_splits), int(align),
+                                           float(scale))
+    if rc != 0:
+        raise ValueError("oracle_split_partials_aligned rejected its arguments")
+    return o, lse
+
+
+def paged_gather(k_pages, v_pages, block_table, seqlens):
+    """Contiguous caches [B,Hkv,max_pages*P,d] (float64) from paged caches.
+
+    k_pages, v_pages: [num_pages, Hkv, P, d]; block_table: [B, max_pages] int.
+    Key t of sequence b is row t % P of physical page block_table[b, t // P]
+    (the block-table indirection of paged KV management, which "I/O-Aware
+    Kernels", section "FlashAttention", names through PagedAttention).  Rows
+    at or past seqlens[b] are NaN: nothing may read them.  Data movement
+    only: plain loops, no arithmetic."""
+    kp, vp = _f64(k_pages), _f64(v_pages)
+    bt = np.asarray(block_table.cpu().numpy() if hasattr(block_table, "cpu") else block_table)
+    sl = np.asarray(seqlens.cpu().numpy() if hasattr(seqlens, "cpu") else seqlens)
+    num_pages, Hkv, P, d = kp.shape
+    B, max_pages = bt.shape
+    kc = np.full((B, Hkv, max_pages * P, d), np.nan)
+    vc = np.full((B, Hkv, max_pages * P, d), np.nan)
+    for b in range(B):
+        L = int(sl[b])
+        if L < 0 or L > max_pages * P:
+            raise ValueError("sequence length outside the block table")
+        for t in range(L):
+            page = int(bt[b, t // P])
+            if not 0 <= page < num_pages:
+                raise ValueError("block table names a page that does not exist")
+            kc[b, :, t] = kp[page, :, t % P]
+            vc[b, :, t] = vp[page, :, t % P]
+    return kc, vc
+
+
+def decode_paged(q, k_pages, v_pages, block_table, seqlens, scale: float,
+                 lib: Optional[ctypes.CDLL] = None):
+    """Single-query decode over a paged cache: the decode of the gathered cache."""
+    kc, vc = paged_gather(k_pages, v_pages, block_table, seqlens)
+    return decode(q, kc, vc, seqlens, scale, lib=lib)
 
 
 def combine(o_part, lse_part, lib: Optional[ctypes.CDLL] = None):

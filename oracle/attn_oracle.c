@@ -235,6 +235,53 @@ int oracle_split_partials(const double *q, const double *kc, const double *vc,
     return err ? -1 : 0;
 }
 
+/* Split-KV partials with chunk boundaries on multiples of `align` keys:
+ * cs = ceil(ceil(L_b / num_splits) / align) * align and chunk c covers
+ * [c*cs, min(L_b, (c+1)*cs)); otherwise as oracle_split_partials (align = 1
+ * is that function's rule).  A decode over a paged cache uses align = 128 so
+ * that every 128-key tile of a chunk starts on a tile boundary.
+ * Outputs: o_part [B,Hq,num_splits,d], lse_part [B,Hq,num_splits]. */
+int oracle_split_partials_aligned(const double *q, const double *kc, const double *vc,
+                                  const int32_t *seqlens, double *o_part, double *lse_part,
+                                  int B, int Hq, int Hkv, int Lmax, int d, int num_splits,
+                                  int align, double scale)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || num_splits < 1 ||
+        align < 1)
+        return -1;
+    for (int b = 0; b < B; ++b)
+        if (seqlens[b] < 0 || seqlens[b] > Lmax) return -1;
+    const int group = Hq / Hkv;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Lmax > 0 ? Lmax : 1));
+        if (!s) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < (int64_t)B * Hq * num_splits; ++r) {
+                const int64_t c = r % num_splits;
+                const int64_t bh = r / num_splits;
+                const int64_t b = bh / Hq, h = bh % Hq, g = h / group;
+                const int64_t L = seqlens[b];
+                const int64_t cs0 = (L + num_splits - 1) / num_splits;
+                const int64_t cs = (cs0 + align - 1) / align * align;
+                int64_t lo = c * cs, hi = lo + cs;
+                if (lo > L) lo = L;
+                if (hi > L) hi = L;
+                const double *kh = kc + ((b * Hkv + g) * (int64_t)Lmax + lo) * d;
+                const double *vh = vc + ((b * Hkv + g) * (int64_t)Lmax + lo) * d;
+                attn_one_row(q + bh * d, kh, vh, hi - lo, d, scale, s,
+                             o_part + r * d, lse_part + r);
+            }
+            free(s);
+        }
+    }
+    return err ? -1 : 0;
+}
+
 /* Merge of split partials.  With M = max_c lse_c the merged statistics are
  * LSE = M + ln sum_c exp(lse_c - M) and O = sum_c exp(lse_c - LSE) * o_c: the
  * e^(m - m_new) rescale rule of the online softmax ("FlashAttention &

@@ -340,6 +340,81 @@ def pin_split_combine_equals_unsplit(lib):
                     _close(lp[b, :, c], l3[0, :, 0], 1e-12, f"chunk {b},{c} LSE")
 
 
+def pin_paged_gather_by_hand(lib):
+    """Block-table indirection on a case worked by hand: page size 2, three
+    physical pages, one sequence of 5 keys whose logical pages are physical
+    pages 2, 0, 1."""
+    kp = np.zeros((3, 1, 2, 1))
+    vp = np.zeros((3, 1, 2, 1))
+    for page in range(3):
+        for row in range(2):
+            kp[page, 0, row, 0] = 10 * page + row      # key value names its page and row
+            vp[page, 0, row, 0] = -(10 * page + row)
+    bt = np.array([[2, 0, 1]])
+    kc, vc = oracle.paged_gather(kp, vp, bt, np.array([5]))
+    # logical keys 0,1 <- page 2 rows 0,1; keys 2,3 <- page 0; key 4 <- page 1 row 0
+    assert kc[0, 0, :5, 0].tolist() == [20, 21, 0, 1, 10], kc[0, 0, :, 0]
+    assert vc[0, 0, :5, 0].tolist() == [-20, -21, 0, -1, -10]
+    assert np.isnan(kc[0, 0, 5:]).all(), "rows past the sequence must stay unread (NaN)"
+
+
+def pin_paged_decode_equals_contiguous(lib):
+    """A contiguous cache cut into pages, scattered by a random permutation and
+    read back through the block table, decodes exactly as the contiguous one."""
+    rng = np.random.default_rng(19)
+    B, Hq, Hkv, P, d = 3, 4, 2, 4, 8
+    max_pages = 6
+    q = _rand((B, Hq, d), rng)
+    kc = _rand((B, Hkv, max_pages * P, d), rng)
+    vc = _rand((B, Hkv, max_pages * P, d), rng)
+    sl = np.array([24, 1, 13], dtype=np.int32)
+    perm = rng.permutation(B * max_pages)
+    kp = np.zeros((B * max_pages, Hkv, P, d))
+    vp = np.zeros((B * max_pages, Hkv, P, d))
+    bt = np.zeros((B, max_pages), dtype=np.int32)
+    for b in range(B):
+        for j in range(max_pages):
+            phys = int(perm[b * max_pages + j])
+            bt[b, j] = phys
+            kp[phys] = kc[b, :, j * P:(j + 1) * P]
+            vp[phys] = vc[b, :, j * P:(j + 1) * P]
+    o, lse = oracle.decode(q, kc, vc, sl, 0.3, lib=lib)
+    o2, lse2 = oracle.decode_paged(q, kp, vp, bt, sl, 0.3, lib=lib)
+    _close(o2, o, 0.0, "paged O")
+    _close(lse2, lse, 0.0, "paged LSE")
+
+
+def pin_aligned_split(lib):
+    """Chunk sizes rounded up to a multiple of align: partials merge to the
+    unsplit decode, every chunk is the one-shot softmax over its own keys,
+    and align = 1 is the plain split rule."""
+    rng = np.random.default_rng(20)
+    q, kc, vc, sl = _decode_case(rng, Lmax=40, lens=(40, 3, 17))
+    o, lse = oracle.decode(q, kc, vc, sl, 0.25, lib=lib)
+    for n in (1, 2, 3, 7):
+        a1 = oracle.split_partials_aligned(q, kc, vc, sl, n, 1, 0.25, lib=lib)
+        a0 = oracle.split_partials(q, kc, vc, sl, n, 0.25, lib=lib)
+        _close(a1[0], a0[0], 0.0, "align 1 O")
+        _close(a1[1], a0[1], 0.0, "align 1 LSE")
+        for align in (4, 8, 16):
+            op, lp = oracle.split_partials_aligned(q, kc, vc, sl, n, align, 0.25, lib=lib)
+            o2, lse2 = oracle.combine(op, lp, lib=lib)
+            _close(o2, o, 1e-12, f"aligned split {n}/{align} O")
+            _close(lse2, lse, 1e-12, f"aligned split {n}/{align} LSE")
+            for b, L in enumerate(sl):
+                cs = -(-(-(-int(L) // n)) // align) * align
+                assert cs % align == 0
+                for c in range(n):
+                    lo, hi = min(L, c * cs), min(L, (c + 1) * cs)
+                    if hi <= lo:
+                        assert np.isneginf(lp[b, :, c]).all() and (op[b, :, c] == 0).all()
+                    else:
+                        o3, l3 = oracle.attn_fwd(q[b:b + 1, :, None], kc[b:b + 1, :, lo:hi],
+                                                 vc[b:b + 1, :, lo:hi], False, 0.25, lib=lib)
+                        _close(op[b, :, c], o3[0, :, 0], 1e-12, f"chunk {b},{c} O")
+                        _close(lp[b, :, c], l3[0, :, 0], 1e-12, f"chunk {b},{c} LSE")
+
+
 ALL_PINS = [
     pin_golden_prefill,
     pin_golden_combine,
@@ -351,4 +426,7 @@ ALL_PINS = [
     pin_gqa_equals_repeated_mha,
     pin_decode_equals_prefill,
     pin_split_combine_equals_unsplit,
+    pin_paged_gather_by_hand,
+    pin_paged_decode_equals_contiguous,
+    pin_aligned_split,
 ]

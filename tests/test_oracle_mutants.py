@@ -30,6 +30,10 @@ MUTANTS = [
     ("combine_lse_missing_max", "const double l = m + log(z);\n        for (int c = 0;",
      "const double l = log(z);\n        for (int c = 0;"),
     ("decode_reads_lmax", "attn_one_row(q + r * d, kh, vh, seqlens[b],", "attn_one_row(q + r * d, kh, vh, Lmax,"),
+    ("aligned_chunk_rounds_down", "const int64_t cs = (cs0 + align - 1) / align * align;",
+     "const int64_t cs = cs0 / align * align;"),
+    ("aligned_chunk_ignores_align", "const int64_t cs = (cs0 + align - 1) / align * align;",
+     "const int64_t cs = cs0;"),
 ]
 
 
