@@ -65,6 +65,10 @@ def parse_args():
                     help="override the decode split count (default: fa_decode_default_splits)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-paged", action="store_true",
+                    help="skip the paged-cache decode measurement")
+    ap.add_argument("--page-size", type=int, default=16,
+                    help="page size of the paged-cache decode measurement")
     return ap.parse_args()
 
 
@@ -379,6 +383,48 @@ def run_ours(args, world, rank, local):
                "d2h_bytes_per_step": int(o.numel() * 2 + lse.numel() * 4),
                "api": "io_aware_exact_flashattention_b200.flash_attention (host tensors)"}
 
+    # Paged cache: the same decode workload stored in page_size-key pages
+    # scattered over a pool, read through a block table.  Measured on its own,
+    # outside the step.
+    paged = None
+    if do_dec and not args.no_paged:
+        from io_aware_exact_flashattention_b200.inputs import paginate
+        kp, vp, bt = paginate(kc, vc, sl, args.page_size, rank_seed(cd.seed, rank))
+        del kc, vc
+        torch.cuda.empty_cache()
+        ps_bytes = dec_bytes + int(sum((int(L) + args.page_size - 1) // args.page_size
+                                       for L in sl.tolist())) * 4
+        for _ in range(max(args.warmup, 1)):
+            fa.fa_decode_paged_splitkv(qd, kp, vp, bt, sl, op, lp, cd.scale, stream=stream)
+            fa.fa_combine(op, lp, od, lsed, stream=stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        pevs = []
+        for _ in range(K):
+            flush.fill_(1.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fa.fa_decode_paged_splitkv(qd, kp, vp, bt, sl, op, lp, cd.scale, stream=stream)
+            fa.fa_combine(op, lp, od, lsed, stream=stream)
+            b.record(stream)
+            pevs.append((a, b))
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        pg_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in pevs)], world)[0]
+        pg_gbs = aggregate_rate(world, ps_bytes, K, pg_ms) / 1e9
+        per_gbs = ps_bytes / (pg_ms * 1e-3 / K) / 1e9
+        paged = {"value": pg_gbs, "unit": "GB/s", "page_size": args.page_size,
+                 "ms_per_call": pg_ms / K,
+                 "frac_of_measured_copy": per_gbs / float(peaks["hbm_gbs"]),
+                 "frac_of_8TBs": per_gbs / NOMINAL_HBM_GBS,
+                 "bytes_per_call": ps_bytes, "gpu_launches": 2 * K,
+                 "traffic": (profiled_traffic("decode_paged_b64_p16_d128.md", DECODE_SOURCES)
+                             if args.page_size == 16 else None),
+                 "kernels": "fa_decode_split_kernel<128,4> (paged loads) + fa_combine_kernel<128>",
+                 "algorithmic": "K,V visible rows + q + O + LSE + block-table entries read",
+                 "note": "same workload, pages scattered over the pool by a seeded permutation; "
+                         "measured outside the step"}
+
     if rank != 0:
         return
     cpu = None
@@ -443,6 +489,8 @@ def run_ours(args, world, rank, local):
         line["roofline"] = line.pop("roofline_decode")
     elif do_dec and not do_pre:
         line["roofline"] = line.pop("roofline_decode")
+    if paged is not None:
+        line["decode_paged"] = paged
     if cpu is not None:
         line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)

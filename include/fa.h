@@ -105,6 +105,48 @@ fa_status fa_decode_splitkv(const void *q, const void *k_cache, const void *v_ca
                             int d, int num_splits, float scale, fa_stream_t stream);
 
 /*
+ * fa_decode_paged_splitkv -- fa_decode_splitkv over a paged key/value cache.
+ *
+ * "I/O-Aware Kernels", section "FlashAttention", names paged KV management
+ * (PagedAttention) as what inference kernels built on FlashAttention read
+ * from; the pages fix no layout.  Here the cache is a pool of fixed-size
+ * pages and each sequence owns a row of a block table: key t of sequence b
+ * (and its value) is row t % page_size of physical page
+ * block_table[b, t / page_size].
+ *
+ *   q            [B, Hq, d]                           bf16
+ *   k_pages,
+ *   v_pages      [num_pages, Hkv, page_size, d]       bf16 (a page holds every
+ *                                                     key/value head's rows)
+ *   block_table  [B, max_pages]   int32, device (4-byte aligned); entries
+ *                t / page_size for t < L_b must name pages in [0, num_pages);
+ *                later entries are never read
+ *   seqlens_k    [B]  int32, device; 0 <= L_b <= max_pages * page_size
+ *                (values outside that range are clamped)
+ *   o_partial    [B, Hq, num_splits, d] fp32 (written; caller-owned scratch)
+ *   lse_partial  [B, Hq, num_splits]    fp32 (written; caller-owned scratch)
+ *
+ * Chunks differ from fa_decode_splitkv in one way: the chunk size
+ * ceil(L_b / num_splits) is rounded up to a multiple of 128, so chunk c covers
+ * keys [c*cs, min(L_b, (c+1)*cs)) with cs = 128 * ceil(ceil(L_b/num_splits)/128)
+ * (key tiles then start on tile boundaries and never straddle pages).  Chunks
+ * past L_b are empty (o_partial = 0, lse_partial = -inf); fa_combine merges
+ * the partials exactly as for the contiguous cache.  Rows of a page past L_b
+ * may be read but never contribute.  An out-of-range page index reads zeros
+ * or another page (never outside the cache), so the result is then
+ * meaningless but memory stays safe.
+ *
+ * Supported: page_size a power of two in [16, 256]; d in {64, 128};
+ * Hq / Hkv in {1, 2, 4, 8}; 1 <= num_splits <= 256.  Errors as for
+ * fa_decode_splitkv; FA_ERR_UNSUPPORTED for another page size.
+ */
+fa_status fa_decode_paged_splitkv(const void *q, const void *k_pages, const void *v_pages,
+                                  const int32_t *block_table, const int32_t *seqlens_k,
+                                  float *o_partial, float *lse_partial, int B, int Hq,
+                                  int Hkv, int num_pages, int page_size, int max_pages,
+                                  int d, int num_splits, float scale, fa_stream_t stream);
+
+/*
  * fa_combine -- second half of decode: merge split partials by their LSE.
  *
  * With M = max_c lse_partial[b,h,c]:

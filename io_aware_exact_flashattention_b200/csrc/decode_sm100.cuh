@@ -22,6 +22,13 @@
 //   warp  4    TMA producer: q of each item, then K and V tiles into a ring
 //              (full tiles in one 128-row box, the last tile of a chunk in
 //              32-row boxes so at most 31 rows past the chunk are fetched)
+// A paged cache ([num_pages, Hkv, page_size, d] with a block table per
+// sequence; paged KV management is named in "I/O-Aware Kernels", section
+// "FlashAttention") changes only the producer: chunks start on multiples of
+// 128 keys, so a tile covers whole pages (page_size <= 128) or lies inside
+// one, and it is loaded as boxes of min(page_size, 128) rows (min(page_size,
+// 32) for a chunk's last tile), each from the physical page the block table
+// names.  The MMA and softmax roles see the same shared-memory tiles.
 //   warp  5    MMA issuer
 // The online softmax keeps a per-head reference max m that only moves when
 // the max grows by more than 2^8; exp2 on scores times scale*log2(e).
@@ -36,6 +43,7 @@ constexpr int kDecBN = 128;       // keys per tile (= TMEM lanes of S^T)
 constexpr int kDecNPad = 16;      // head columns of S^T / O^T (G real, rest zero)
 constexpr int kDecSubRows = 32;   // rows per box of a chunk's last tile
 constexpr int kDecThreads = 192;
+constexpr int kDecMaxPagesPerTile = kDecBN / 16;  // pages of the smallest size in a tile
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kDecRescaleThreshold = 8.0f;  // log2 units
 
@@ -81,6 +89,13 @@ struct DecodeParams {
   int B, Hq, Hkv, Lmax, n_splits, n_items;
   float scale, scale_log2;
   unsigned long long wait_limit_ns;
+  // paged cache (block_table == nullptr: contiguous [B, Hkv, Lmax, d] cache)
+  const int* block_table;  // [B, max_pages]
+  int max_pages;
+  int page_shift;          // log2(page_size)
+  int rows_main;           // rows per box of a full tile: min(page_size, 128)
+  int rows_tail;           // rows per box of a chunk's last tile: min(page_size, 32)
+  int chunk_align;         // chunk sizes are rounded up to a multiple of this
 };
 
 // Chunk [lo, hi) of the keys of sequence b for split c (see fa.h).
@@ -88,7 +103,8 @@ __device__ __forceinline__ void decode_chunk(const DecodeParams& p, int b, int c
                                              int& hi) {
   int L = p.seqlens[b];
   L = max(0, min(L, p.Lmax));
-  const int cs = (L + p.n_splits - 1) / p.n_splits;
+  const int cs0 = (L + p.n_splits - 1) / p.n_splits;
+  const int cs = (cs0 + p.chunk_align - 1) / p.chunk_align * p.chunk_align;
   lo = min(L, c * cs);
   hi = min(L, lo + cs);
 }
@@ -102,20 +118,36 @@ __device__ __forceinline__ void decode_item(const DecodeParams& p, int item, int
 }
 
 // ---------------------------------------------------------------------------
-// TMA producer (one thread)
+// TMA producer (one warp).  Lane 0 waits for buffers, accounts the bytes and
+// issues the query loads and the contiguous-cache tile loads; for a paged
+// cache a tile is many small boxes (two per page of 16 rows at d=128), and
+// each lane issues one of them so their issue costs overlap.
 // ---------------------------------------------------------------------------
 template <int D, int G>
 __device__ __forceinline__ void decode_producer(const CUtensorMap* tk, const CUtensorMap* tv,
                                                 const CUtensorMap* tk32, const CUtensorMap* tv32,
                                                 const CUtensorMap* tq, const DecodeParams& p,
-                                                uint32_t sbase, volatile int* abort_flag) {
+                                                uint32_t sbase, volatile int* abort_flag,
+                                                int lane) {
   using L = DecodeLayout<D>;
+  const bool leader = (lane == 0);
+  const bool paged = (p.block_table != nullptr);
+  if (!paged && !leader) return;  // a contiguous cache needs lane 0 only
+  const unsigned mask = paged ? 0xffffffffu : 1u;
   const uint32_t bars = sbase + L::kBarOff;
-  tma_prefetch_desc(tk);
-  tma_prefetch_desc(tv);
-  tma_prefetch_desc(tk32);
-  tma_prefetch_desc(tv32);
-  tma_prefetch_desc(tq);
+  if (leader) {
+    tma_prefetch_desc(tk);
+    tma_prefetch_desc(tv);
+    tma_prefetch_desc(tk32);
+    tma_prefetch_desc(tv32);
+    tma_prefetch_desc(tq);
+  }
+  // lane 0 waits; every lane follows its verdict
+  auto leader_wait = [&](uint32_t bar, uint32_t parity) -> bool {
+    bool ok = true;
+    if (leader) ok = mbar_wait(bar, parity, abort_flag, p.wait_limit_ns);
+    return __shfl_sync(mask, ok ? 1 : 0, 0) != 0;
+  };
   uint32_t ld = 0;  // K/V tile loads issued
   int it = 0;
   bool stop = false;
@@ -124,45 +156,78 @@ __device__ __forceinline__ void decode_producer(const CUtensorMap* tk, const CUt
     decode_item(p, item, b, g, c);
     decode_chunk(p, b, c, lo, hi);
     const int slot = it & 1;
-    if (!mbar_wait(bars + 8 * (L::kBQEmpty + slot), (static_cast<uint32_t>(it >> 1) & 1u) ^ 1u,
-                   abort_flag, p.wait_limit_ns))
+    if (!leader_wait(bars + 8 * (L::kBQEmpty + slot), (static_cast<uint32_t>(it >> 1) & 1u) ^ 1u))
       break;
-    volatile int* meta =
-        reinterpret_cast<volatile int*>(__cvta_shared_to_generic(sbase + L::kMetaOff + slot * 16));
-    meta[0] = lo;
-    meta[1] = hi;
-    const uint32_t qbar = bars + 8 * (L::kBQFull + slot);
-    mbar_arrive_expect_tx(qbar, L::kQBytes);
+    if (leader) {
+      volatile int* meta = reinterpret_cast<volatile int*>(
+          __cvta_shared_to_generic(sbase + L::kMetaOff + slot * 16));
+      meta[0] = lo;
+      meta[1] = hi;
+      const uint32_t qbar = bars + 8 * (L::kBQFull + slot);
+      mbar_arrive_expect_tx(qbar, L::kQBytes);
 #pragma unroll
-    for (int kb = 0; kb < D / 64; ++kb)
-      tma_load_2d(sbase + L::kQOff + slot * L::kQBytes + kb * L::kQBoxBytes, tq, qbar, kb * 64,
-                  b * p.Hq + g * G);
+      for (int kb = 0; kb < D / 64; ++kb)
+        tma_load_2d(sbase + L::kQOff + slot * L::kQBytes + kb * L::kQBoxBytes, tq, qbar, kb * 64,
+                    b * p.Hq + g * G);
+    }
     const int plane = b * p.Hkv + g;
     for (int t0 = lo; t0 < hi && !stop; t0 += kDecBN) {
       const int ntok = min(kDecBN, hi - t0);
+      // Paged cache: the physical page of each page-sized (at most 128-row)
+      // slice of the tile, read before the ring-slot waits so the loads'
+      // latency overlaps them.
+      int pg[kDecMaxPagesPerTile];
+      if (paged) {
+        const int* bt = p.block_table + static_cast<size_t>(b) * p.max_pages;
+        const int slice = min(1 << p.page_shift, kDecBN);
+#pragma unroll
+        for (int j = 0; j < kDecMaxPagesPerTile; ++j)
+          pg[j] = (j * slice < ntok) ? __ldg(bt + ((t0 + j * slice) >> p.page_shift)) : 0;
+      }
 #pragma unroll
       for (int kv = 0; kv < 2; ++kv) {
         const int stage = static_cast<int>(ld % L::kStages);
-        if (!mbar_wait(bars + 8 * (L::kBKvEmpty + stage),
-                       ((ld / L::kStages) & 1u) ^ 1u, abort_flag, p.wait_limit_ns)) {
+        if (!leader_wait(bars + 8 * (L::kBKvEmpty + stage), ((ld / L::kStages) & 1u) ^ 1u)) {
           stop = true;
           break;
         }
         const uint32_t full = bars + 8 * (L::kBKvFull + stage);
         const uint32_t dst = sbase + L::kRingOff + stage * L::kTileBytes;
-        if (ntok == kDecBN) {
-          mbar_arrive_expect_tx(full, L::kTileBytes);
+        if (paged) {
+          // Boxes never straddle a page: t0 is a multiple of 128 and the box
+          // height divides both 128 and the page size.
+          const bool whole = (ntok == kDecBN);
+          const int rows = whole ? p.rows_main : p.rows_tail;
+          const int nsub = (ntok + rows - 1) / rows;
+          const CUtensorMap* tm = whole ? (kv ? tv : tk) : (kv ? tv32 : tk32);
+          if (leader) mbar_arrive_expect_tx(full, nsub * rows * 128 * (D / 64));
+          __syncwarp(mask);
+          if (lane < nsub * (D / 64)) {  // at most 16 boxes per tile (page size 16)
+            const int sub = lane / (D / 64), kb = lane % (D / 64);
+            const int slice = min(1 << p.page_shift, kDecBN);
+            int page = pg[0];
 #pragma unroll
-          for (int kb = 0; kb < D / 64; ++kb)
-            tma_load_3d(dst + kb * L::kBoxBytes, kv ? tv : tk, full, kb * 64, t0, plane);
-        } else {
-          const int nsub = (ntok + kDecSubRows - 1) / kDecSubRows;
-          mbar_arrive_expect_tx(full, nsub * kDecSubRows * 128 * (D / 64));
-          for (int sub = 0; sub < nsub; ++sub)
+            for (int j = 1; j < kDecMaxPagesPerTile; ++j)
+              if (sub * rows >= j * slice) page = pg[j];
+            const int prow = (t0 + sub * rows) & ((1 << p.page_shift) - 1);
+            tma_load_3d(dst + kb * L::kBoxBytes + sub * rows * 128, tm, full, kb * 64, prow,
+                        page * p.Hkv + g);
+          }
+        } else if (leader) {
+          if (ntok == kDecBN) {
+            mbar_arrive_expect_tx(full, L::kTileBytes);
 #pragma unroll
             for (int kb = 0; kb < D / 64; ++kb)
-              tma_load_3d(dst + kb * L::kBoxBytes + sub * kDecSubRows * 128, kv ? tv32 : tk32,
-                          full, kb * 64, t0 + sub * kDecSubRows, plane);
+              tma_load_3d(dst + kb * L::kBoxBytes, kv ? tv : tk, full, kb * 64, t0, plane);
+          } else {
+            const int nsub = (ntok + kDecSubRows - 1) / kDecSubRows;
+            mbar_arrive_expect_tx(full, nsub * kDecSubRows * 128 * (D / 64));
+            for (int sub = 0; sub < nsub; ++sub)
+#pragma unroll
+              for (int kb = 0; kb < D / 64; ++kb)
+                tma_load_3d(dst + kb * L::kBoxBytes + sub * kDecSubRows * 128, kv ? tv32 : tk32,
+                            full, kb * 64, t0 + sub * kDecSubRows, plane);
+          }
         }
         ++ld;
       }
@@ -170,12 +235,14 @@ __device__ __forceinline__ void decode_producer(const CUtensorMap* tk, const CUt
     if (stop) ++it;  // this item's q load was issued
   }
   // Drain: no copy may still be in flight when the CTA exits.
-  const uint32_t S = static_cast<uint32_t>(L::kStages);
-  for (uint32_t k = (ld > S ? ld - S : 0u); k < ld; ++k)
-    mbar_wait(bars + 8 * (L::kBKvFull + k % S), (k / S) & 1u, nullptr, p.wait_limit_ns);
-  for (int k = (it > 2 ? it - 2 : 0); k < it; ++k)
-    mbar_wait(bars + 8 * (L::kBQFull + (k & 1)), static_cast<uint32_t>(k >> 1) & 1u, nullptr,
-              p.wait_limit_ns);
+  if (leader) {
+    const uint32_t S = static_cast<uint32_t>(L::kStages);
+    for (uint32_t k = (ld > S ? ld - S : 0u); k < ld; ++k)
+      mbar_wait(bars + 8 * (L::kBKvFull + k % S), (k / S) & 1u, nullptr, p.wait_limit_ns);
+    for (int k = (it > 2 ? it - 2 : 0); k < it; ++k)
+      mbar_wait(bars + 8 * (L::kBQFull + (k & 1)), static_cast<uint32_t>(k >> 1) & 1u, nullptr,
+                p.wait_limit_ns);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -527,8 +594,7 @@ fa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
   if (warp < 4) {
     decode_softmax<D, G>(p, sbase, tmem, abort_flag);
   } else if (warp == 4) {
-    if (lane == 0)
-      decode_producer<D, G>(&tm_k, &tm_v, &tm_k32, &tm_v32, &tm_q, p, sbase, abort_flag);
+    decode_producer<D, G>(&tm_k, &tm_v, &tm_k32, &tm_v32, &tm_q, p, sbase, abort_flag, lane);
   } else {
     if (lane == 0) decode_mma<D, G>(p, sbase, tmem, abort_flag);
   }

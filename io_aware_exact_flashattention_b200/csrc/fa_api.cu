@@ -1,6 +1,7 @@
 // fa_api.cu -- the C ABI of libfa.so (declared in include/fa.h): argument
 // checks, TMA tensor-map encoding and kernel launches.  Every kernel of the
 // library lives in this one translation unit.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -187,16 +188,28 @@ bool encode_query(CUtensorMap* map, const void* base, int d, long long rows) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A paged cache: [num_pages, Hkv, page_size, d] plus a [B, max_pages] block table.
+struct PagedCache {
+  const int32_t* block_table;
+  int num_pages, page_size, max_pages;
+};
+
 template <int D, int G>
 fa_status launch_decode(const void* q, const void* kc, const void* vc, const int32_t* seqlens,
                         float* o_part, float* lse_part, int B, int Hq, int Hkv, int Lmax,
-                        int num_splits, float scale, int num_sms, cudaStream_t stream) {
+                        int num_splits, float scale, int num_sms, cudaStream_t stream,
+                        const PagedCache* pg) {
   CUtensorMap tk, tv, tk32, tv32, tq;
-  const long long planes = static_cast<long long>(B) * Hkv;
-  if (!encode_cache(&tk, kc, D, Lmax, planes, fa::kDecBN) ||
-      !encode_cache(&tv, vc, D, Lmax, planes, fa::kDecBN) ||
-      !encode_cache(&tk32, kc, D, Lmax, planes, fa::kDecSubRows) ||
-      !encode_cache(&tv32, vc, D, Lmax, planes, fa::kDecSubRows) ||
+  // Contiguous: planes (b, g) of Lmax rows.  Paged: planes (page, g) of page_size rows.
+  const long long planes = pg ? static_cast<long long>(pg->num_pages) * Hkv
+                              : static_cast<long long>(B) * Hkv;
+  const int rows = pg ? pg->page_size : Lmax;
+  const int box_main = pg ? std::min(pg->page_size, fa::kDecBN) : fa::kDecBN;
+  const int box_tail = pg ? std::min(pg->page_size, fa::kDecSubRows) : fa::kDecSubRows;
+  if (!encode_cache(&tk, kc, D, rows, planes, box_main) ||
+      !encode_cache(&tv, vc, D, rows, planes, box_main) ||
+      !encode_cache(&tk32, kc, D, rows, planes, box_tail) ||
+      !encode_cache(&tv32, vc, D, rows, planes, box_tail) ||
       !encode_query(&tq, q, D, static_cast<long long>(B) * Hq))
     return FA_ERR_CUDA;
   fa::DecodeParams p;
@@ -212,6 +225,14 @@ fa_status launch_decode(const void* q, const void* kc, const void* vc, const int
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_limit_ns = kWaitLimitNs;
+  p.block_table = pg ? pg->block_table : nullptr;
+  p.max_pages = pg ? pg->max_pages : 0;
+  int shift = 0;
+  while (pg && (1 << shift) < pg->page_size) ++shift;
+  p.page_shift = shift;
+  p.rows_main = box_main;
+  p.rows_tail = box_tail;
+  p.chunk_align = pg ? fa::kDecBN : 1;
   const int grid = p.n_items < num_sms ? p.n_items : num_sms;
   fa::fa_decode_split_kernel<D, G><<<grid, fa::kDecThreads, fa::DecodeLayout<D>::kBytes,
                                      stream>>>(tk, tv, tk32, tv32, tq, p);
@@ -222,12 +243,12 @@ template <int D>
 fa_status dispatch_decode_group(int G, const void* q, const void* kc, const void* vc,
                                 const int32_t* seqlens, float* o_part, float* lse_part, int B,
                                 int Hq, int Hkv, int Lmax, int num_splits, float scale,
-                                int num_sms, cudaStream_t stream) {
+                                int num_sms, cudaStream_t stream, const PagedCache* pg) {
   switch (G) {
-    case 1: return launch_decode<D, 1>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, num_sms, stream);
-    case 2: return launch_decode<D, 2>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, num_sms, stream);
-    case 4: return launch_decode<D, 4>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, num_sms, stream);
-    case 8: return launch_decode<D, 8>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, num_sms, stream);
+    case 1: return launch_decode<D, 1>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, num_sms, stream, pg);
+    case 2: return launch_decode<D, 2>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, num_sms, stream, pg);
+    case 4: return launch_decode<D, 4>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, num_sms, stream, pg);
+    case 8: return launch_decode<D, 8>(q, kc, vc, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, num_splits, scale, num_sms, stream, pg);
     default: return FA_ERR_UNSUPPORTED;
   }
 }
@@ -337,10 +358,58 @@ fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_ca
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const fa_status st =
       d == 64 ? dispatch_decode_group<64>(G, q, k_cache, v_cache, seqlens_k, o_partial,
-                                          lse_partial, B, Hq, Hkv, Lmax, num_splits, scale, sms, s)
+                                          lse_partial, B, Hq, Hkv, Lmax, num_splits, scale, sms, s,
+                                          nullptr)
               : dispatch_decode_group<128>(G, q, k_cache, v_cache, seqlens_k, o_partial,
                                            lse_partial, B, Hq, Hkv, Lmax, num_splits, scale, sms,
-                                           s);
+                                           s, nullptr);
+  if (st != FA_OK) return st;
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_decode_paged_splitkv(const void* q, const void* k_pages, const void* v_pages,
+                                  const int32_t* block_table, const int32_t* seqlens_k,
+                                  float* o_partial, float* lse_partial, int B, int Hq, int Hkv,
+                                  int num_pages, int page_size, int max_pages, int d,
+                                  int num_splits, float scale, fa_stream_t stream) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || num_pages < 1 || max_pages < 1) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (num_splits < 1 || num_splits > 256) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (page_size < 16 || page_size > 256 || (page_size & (page_size - 1)) != 0)
+    return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return FA_ERR_UNSUPPORTED;
+  const long long lmax = static_cast<long long>(max_pages) * page_size;
+  if (lmax > 0x7fffffffLL - fa::kDecBN ||
+      static_cast<long long>(num_pages) * Hkv > 0x7fffffffLL ||
+      static_cast<long long>(B) * max_pages > 0x7fffffffLL ||
+      static_cast<long long>(B) * Hkv * num_splits > 0x7fffffffLL)
+    return FA_ERR_UNSUPPORTED;
+  if (B == 0) return FA_OK;
+  if (q == nullptr || k_pages == nullptr || v_pages == nullptr || block_table == nullptr ||
+      seqlens_k == nullptr || o_partial == nullptr || lse_partial == nullptr)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) ||
+      (reinterpret_cast<uintptr_t>(seqlens_k) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3u) != 0 ||
+      !aligned16(o_partial) || !aligned16(lse_partial))
+    return FA_ERR_ALIGNMENT;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (prepare_decode(dev) != cudaSuccess) return FA_ERR_CUDA;
+  const int sms = g_num_sms[dev];
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const PagedCache pg{block_table, num_pages, page_size, max_pages};
+  const int Lmax = static_cast<int>(lmax);
+  const fa_status st =
+      d == 64 ? dispatch_decode_group<64>(G, q, k_pages, v_pages, seqlens_k, o_partial,
+                                          lse_partial, B, Hq, Hkv, Lmax, num_splits, scale, sms, s,
+                                          &pg)
+              : dispatch_decode_group<128>(G, q, k_pages, v_pages, seqlens_k, o_partial,
+                                           lse_partial, B, Hq, Hkv, Lmax, num_splits, scale, sms,
+                                           s, &pg);
   if (st != FA_OK) return st;
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

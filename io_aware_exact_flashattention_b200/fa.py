@@ -33,6 +33,7 @@ _I, _F = ctypes.c_int, ctypes.c_float
 SIGNATURES = {
     "fa_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _VP]),
     "fa_decode_splitkv": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP]),
+    "fa_decode_paged_splitkv": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP] + [_I] * 8 + [_F, _VP]),
     "fa_combine": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP]),
     "fa_decode_default_splits": (_I, [_I, _I, _I, _I]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
@@ -138,6 +139,35 @@ def fa_decode_splitkv(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Ten
         _ptr(lse_partial), B, Hq, Hkv, Lmax, d, n, float(scale), _stream_ptr(stream)))
 
 
+def fa_decode_paged_splitkv(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                            block_table: torch.Tensor, seqlens_k: torch.Tensor,
+                            o_partial: torch.Tensor, lse_partial: torch.Tensor, scale: float,
+                            stream: Optional[torch.cuda.Stream] = None) -> None:
+    """fa_decode_paged_splitkv on q [B,Hq,d], page pools [num_pages,Hkv,P,d] (bf16),
+    block_table [B,max_pages] and seqlens [B] int32; o_partial [B,Hq,n,d] and
+    lse_partial [B,Hq,n] fp32 (chunk sizes rounded up to multiples of 128)."""
+    for t, n in ((q, "q"), (k_pages, "k_pages"), (v_pages, "v_pages")):
+        _need(t, torch.bfloat16, n)
+    _need(block_table, torch.int32, "block_table")
+    _need(seqlens_k, torch.int32, "seqlens_k")
+    _need(o_partial, torch.float32, "o_partial")
+    _need(lse_partial, torch.float32, "lse_partial")
+    B, Hq, d = q.shape
+    num_pages, Hkv, P, _ = k_pages.shape
+    if tuple(v_pages.shape) != tuple(k_pages.shape):
+        raise ValueError("k_pages and v_pages must have the same shape")
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be [B, max_pages]")
+    max_pages = block_table.shape[1]
+    n = o_partial.shape[2]
+    if tuple(o_partial.shape) != (B, Hq, n, d) or tuple(lse_partial.shape) != (B, Hq, n):
+        raise ValueError("partial buffers must be [B,Hq,n,d] and [B,Hq,n]")
+    _check("fa_decode_paged_splitkv", lib().fa_decode_paged_splitkv(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seqlens_k),
+        _ptr(o_partial), _ptr(lse_partial), B, Hq, Hkv, num_pages, P, max_pages, d, n,
+        float(scale), _stream_ptr(stream)))
+
+
 def fa_combine(o_partial: torch.Tensor, lse_partial: torch.Tensor, o: torch.Tensor,
                lse: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> None:
     """fa_combine: o_partial [B,Hq,n,d], lse_partial [B,Hq,n] fp32 -> o [B,Hq,d]
@@ -231,6 +261,29 @@ def decode_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tens
     o_part = torch.empty((B, Hq, num_splits, d), device=q.device, dtype=torch.float32)
     lse_part = torch.empty((B, Hq, num_splits), device=q.device, dtype=torch.float32)
     fa_decode_splitkv(q, k_cache, v_cache, seqlens_k, o_part, lse_part, scale)
+    o = torch.empty((B, Hq, d), device=q.device, dtype=torch.bfloat16)
+    lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32)
+    fa_combine(o_part, lse_part, o, lse)
+    return o, lse
+
+
+def decode_attention_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                           block_table: torch.Tensor, seqlens_k: torch.Tensor,
+                           scale: Optional[float] = None,
+                           num_splits: Optional[int] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Single-query decode over a paged cache (pages [num_pages,Hkv,P,d], block
+    table [B,max_pages]): split-KV partials, then the LSE-weighted merge."""
+    B, Hq, d = q.shape
+    _, Hkv, P, _ = k_pages.shape
+    Lmax = block_table.shape[1] * P
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if num_splits is None:
+        sms = torch.cuda.get_device_properties(q.device).multi_processor_count
+        num_splits = decode_default_splits(B, Hkv, Lmax, sms)
+    o_part = torch.empty((B, Hq, num_splits, d), device=q.device, dtype=torch.float32)
+    lse_part = torch.empty((B, Hq, num_splits), device=q.device, dtype=torch.float32)
+    fa_decode_paged_splitkv(q, k_pages, v_pages, block_table, seqlens_k, o_part, lse_part, scale)
     o = torch.empty((B, Hq, d), device=q.device, dtype=torch.bfloat16)
     lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32)
     fa_combine(o_part, lse_part, o, lse)

@@ -124,3 +124,61 @@ def decode_inputs(B: int, Hq: int, Hkv: int, Lmin: int, Lmax: int, d: int, seed:
 def decode_inputs_for(shape: DecodeShape, device="cpu", pad_value=float("nan")):
     return decode_inputs(shape.B, shape.Hq, shape.Hkv, shape.Lmin, shape.Lmax, shape.d,
                          shape.seed, device, pad_value)
+
+
+def paginate(kc, vc, seqlens, page_size: int, seed: int,
+             pad_value: Optional[float] = float("nan")):
+    """Store contiguous caches [B,Hkv,Lmax,d] in a paged pool.
+
+    Returns k_pages/v_pages [num_pages,Hkv,page_size,d] and block_table
+    [B, ceil(Lmax/page_size)] (int32, on the caches' device).  Sequence b gets
+    ceil(L_b/page_size) pages, placed in the pool in an order drawn from the
+    seed (a scattered pool, as after many allocations and frees); the pool
+    holds exactly the used pages.  Table entries past a sequence's last page
+    are -1; rows of a last page past L_b hold pad_value."""
+    B, Hkv, Lmax, d = kc.shape
+    P = int(page_size)
+    max_pages = (Lmax + P - 1) // P
+    lens = [int(L) for L in seqlens.tolist()]
+    counts = [(L + P - 1) // P for L in lens]
+    num_pages = max(1, sum(counts))
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed) + 7919)
+    order = torch.randperm(num_pages, generator=g)
+    fill = float("nan") if pad_value is None else pad_value
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    b_idx, j_idx = [], []
+    for b in range(B):
+        b_idx += [b] * counts[b]
+        j_idx += list(range(counts[b]))
+    phys = order[:len(b_idx)]
+    table[torch.tensor(b_idx, dtype=torch.long), torch.tensor(j_idx, dtype=torch.long)] = \
+        phys.to(torch.int32)
+    pages = []
+    for cache in (kc, vc):
+        padded = torch.full((B, Hkv, max_pages * P, d), fill, device=cache.device,
+                            dtype=cache.dtype)
+        padded[:, :, :Lmax] = cache
+        for b, L in enumerate(lens):  # rows past L_b: pad_value
+            padded[b, :, L:] = fill
+        blocks = padded.view(B, Hkv, max_pages, P, d).permute(0, 2, 1, 3, 4)
+        pool = torch.full((num_pages, Hkv, P, d), fill, device=cache.device, dtype=cache.dtype)
+        if b_idx:
+            bi = torch.tensor(b_idx, dtype=torch.long, device=cache.device)
+            ji = torch.tensor(j_idx, dtype=torch.long, device=cache.device)
+            pool[phys.to(cache.device)] = blocks[bi, ji]
+        pages.append(pool.contiguous())
+        del padded, blocks
+    return pages[0], pages[1], table.to(kc.device).contiguous()
+
+
+def paged_decode_inputs(B: int, Hq: int, Hkv: int, Lmin: int, Lmax: int, d: int, seed: int,
+                        page_size: int, device="cpu",
+                        pad_value: Optional[float] = float("nan")):
+    """The decode_inputs() sequences stored in a paged cache (see paginate()).
+
+    Returns q [B,Hq,d], k_pages/v_pages [num_pages,Hkv,page_size,d] (bf16),
+    block_table [B, ceil(Lmax/page_size)] and seqlens [B] (int32)."""
+    q, kc, vc, seqlens = decode_inputs(B, Hq, Hkv, Lmin, Lmax, d, seed, device, pad_value)
+    k_pages, v_pages, table = paginate(kc, vc, seqlens, page_size, seed, pad_value)
+    return q, k_pages, v_pages, table, seqlens

@@ -100,6 +100,34 @@ def test_decode_rejects_before_cuda(lib, kw, want):
     assert dec(lib, **kw) == want
 
 
+def paged(lib, *, q=A, kp=A, vp=A, bt=A, sl=A, op=A, lp=A, B=2, Hq=8, Hkv=2, pages=16, P=16,
+          max_pages=8, d=128, n=4, scale=0.1):
+    return lib.fa_decode_paged_splitkv(q, kp, vp, bt, sl, op, lp, B, Hq, Hkv, pages, P,
+                                       max_pages, d, n, scale, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(P=24), UNSUPPORTED),           # not a power of two
+    (dict(P=8), UNSUPPORTED),            # below 16
+    (dict(P=512), UNSUPPORTED),          # above 256
+    (dict(d=80), UNSUPPORTED),
+    (dict(Hq=24, Hkv=2), UNSUPPORTED),
+    (dict(Hq=8, Hkv=3), INVALID),
+    (dict(pages=0), INVALID),
+    (dict(max_pages=0), INVALID),
+    (dict(n=0), INVALID),
+    (dict(scale=float("nan")), INVALID),
+    (dict(bt=None), INVALID),
+    (dict(vp=None), INVALID),
+    (dict(bt=A + 2), ALIGNMENT),
+    (dict(kp=A + 8), ALIGNMENT),
+    (dict(max_pages=1 << 24, P=256), UNSUPPORTED),  # max_pages * P beyond int32
+    (dict(B=0, q=None, bt=None), OK),
+])
+def test_paged_decode_rejects_before_cuda(lib, kw, want):
+    assert paged(lib, **kw) == want
+
+
 @pytest.mark.parametrize("args,want", [
     ((A, A, A, A, 2, 8, 0, 128), INVALID),
     ((A, A, A, A, 2, 8, 4, 96), UNSUPPORTED),
