@@ -212,38 +212,77 @@ def debug_timeout_probe(limit_us: int, stream: Optional[torch.cuda.Stream] = Non
 
 def flash_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
                     scale: Optional[float] = None, device: Optional[torch.device] = None,
-                    out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None
-                    ) -> Tuple[torch.Tensor, torch.Tensor]:
+                    out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None,
+                    chunks: Optional[int] = None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Exact attention O = softmax(scale*QK^T [+causal mask]) V and its LSE.
 
-    CUDA inputs stay where they are; CPU inputs (ideally pinned) are copied to
-    `device` (default: the current CUDA device), and the results are copied
+    CUDA inputs stay where they are.  CPU inputs (ideally pinned) are copied
+    to `device` (default: the current CUDA device) and the results are copied
     back into `out` = (o, lse) host tensors when given, else into new pinned
-    tensors.  With host inputs the call returns after the results landed."""
-    host = not q.is_cuda
+    tensors; the call returns after the results landed.  With host inputs the
+    work is cut into `chunks` groups of key/value heads (default: about 16 MB
+    of inputs each); each group is an fa_fwd problem of its own ([n, G, S, d]
+    queries against [n, 1, S, d] keys/values), so copying group c+1 in, the
+    kernel on group c and copying group c-1 out run at the same time on
+    three streams."""
     if scale is None:
         scale = 1.0 / math.sqrt(q.shape[-1])
-    if host:
-        dev = device or torch.device("cuda", torch.cuda.current_device())
-        q, k, v = (t.to(dev, non_blocking=True) for t in (q, k, v))
-    B, Hq, Sq, d = q.shape
-    if out is not None and not host:
-        o, lse = out
-    else:
-        o = torch.empty_like(q)
-        lse = torch.empty((B, Hq, Sq), device=q.device, dtype=torch.float32)
-    fa_fwd(q, k, v, o, lse, causal, scale)
-    if host:
+    if q.is_cuda:
+        B, Hq, Sq, d = q.shape
         if out is not None:
-            o_h, lse_h = out
+            o, lse = out
         else:
-            o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-            lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
-        o_h.copy_(o, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
-        torch.cuda.current_stream().synchronize()
-        return o_h, lse_h
-    return o, lse
+            o = torch.empty_like(q)
+            lse = torch.empty((B, Hq, Sq), device=q.device, dtype=torch.float32)
+        fa_fwd(q, k, v, o, lse, causal, scale)
+        return o, lse
+
+    dev = device or torch.device("cuda", torch.cuda.current_device())
+    B, Hq, Sq, d = q.shape
+    _, Hkv, Skv, _ = k.shape
+    if Hkv < 1 or Hq % Hkv != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    G = Hq // Hkv
+    rows = B * Hkv  # key/value heads; each owns G query heads
+    if out is not None:
+        o_h, lse_h = out
+    else:
+        o_h = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        lse_h = torch.empty((B, Hq, Sq), dtype=torch.float32, pin_memory=True)
+    # [rows, G, S, d] / [rows, 1, S, d] views: a range of rows is a valid problem
+    qf, kf, vf = q.reshape(rows, G, Sq, d), k.reshape(rows, 1, Skv, d), v.reshape(rows, 1, Skv, d)
+    of, lf = o_h.view(rows, G, Sq, d), lse_h.view(rows, G, Sq)
+    qd, kd, vd = (torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (qf, kf, vf))
+    od = torch.empty(qf.shape, dtype=q.dtype, device=dev)
+    ld = torch.empty((rows, G, Sq), dtype=torch.float32, device=dev)
+    if chunks is None:
+        per_row = (G * Sq + 2 * Skv) * d * q.element_size()
+        chunks = max(1, min(rows, (rows * per_row) // (16 << 20)))
+    bounds = [rows * c // chunks for c in range(chunks + 1)]
+    compute = torch.cuda.current_stream(dev)
+    s_in = torch.cuda.Stream(dev)
+    s_out = torch.cuda.Stream(dev)
+    s_in.wait_stream(compute)    # device buffers are free for this call's copies
+    s_out.wait_stream(compute)
+    for c in range(chunks):
+        a, b = bounds[c], bounds[c + 1]
+        if a == b:
+            continue
+        with torch.cuda.stream(s_in):
+            for dst, src in ((qd, qf), (kd, kf), (vd, vf)):
+                dst[a:b].copy_(src[a:b], non_blocking=True)
+        compute.wait_stream(s_in)
+        fa_fwd(qd[a:b], kd[a:b], vd[a:b], od[a:b], ld[a:b], causal, scale, stream=compute)
+        s_out.wait_stream(compute)
+        with torch.cuda.stream(s_out):
+            of[a:b].copy_(od[a:b], non_blocking=True)
+            lf[a:b].copy_(ld[a:b], non_blocking=True)
+    compute.wait_stream(s_out)
+    compute.synchronize()
+    for t in (qd, kd, vd, od, ld):  # the caching allocator must not hand these out early
+        t.record_stream(s_in)
+        t.record_stream(s_out)
+    return o_h, lse_h
 
 
 def decode_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,

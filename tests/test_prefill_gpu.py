@@ -181,6 +181,21 @@ def test_host_buffers_round_trip():
     assert eo <= O_TOL and el <= LSE_TOL
 
 
+@pytest.mark.parametrize("chunks", [2, 3, 5])
+def test_host_buffers_in_chunks_equal_device_call(chunks):
+    """Host inputs are cut into groups of key/value heads that are copied in,
+    computed and copied out on overlapping streams; every group is its own
+    launch, and the result is bit-identical to one launch on device tensors
+    (a query tile's computation does not depend on which launch holds it)."""
+    q, k, v = prefill_inputs(2, 8, 2, 333, 333, 128, 14)  # 4 key/value heads, G=4
+    o_dev, lse_dev = run_fa(q.cuda(), k.cuda(), v.cuda(), True, 0.09)
+    torch.cuda.synchronize()
+    q, k, v = (t.pin_memory() for t in (q, k, v))
+    o_h, lse_h = fa.flash_attention(q, k, v, causal=True, scale=0.09, chunks=chunks)
+    assert not o_h.is_cuda
+    assert torch.equal(o_h, o_dev.cpu()) and torch.equal(lse_h, lse_dev.cpu())
+
+
 def sample_rows(B, Hq, Sq, n, seed):
     rng = np.random.default_rng(seed)
     rows = {(0, 0, 0), (B - 1, Hq - 1, Sq - 1), (0, Hq - 1, 127), (B - 1, 0, 128),
