@@ -74,6 +74,8 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_split_partials_aligned.argtypes = ([_D, _D, _D, _I32, _D, _D] + [ci] * 7
                                                   + [ctypes.c_double])
     lib.oracle_split_partials_aligned.restype = ci
+    lib.oracle_attn_bwd.argtypes = [_D] * 7 + [ci] * 7 + [ctypes.c_double]
+    lib.oracle_attn_bwd.restype = ci
     lib.oracle_combine.argtypes = [_D, _D, _D, _D] + [ci] * 4
     lib.oracle_combine.restype = ci
     lib.oracle_num_threads.argtypes = []
@@ -108,6 +110,22 @@ def attn_fwd(q, k, v, causal: bool, scale: float, lib: Optional[ctypes.CDLL] = N
     if rc != 0:
         raise ValueError("oracle_attn_fwd rejected its arguments")
     return o, lse
+
+
+def attn_bwd(q, k, v, d_o, causal: bool, scale: float, lib: Optional[ctypes.CDLL] = None):
+    """Gradients (dq, dk, dv) in float64 of the forward above for dL/dO = d_o."""
+    lib = lib or load()
+    q, k, v, d_o = _f64(q), _f64(k), _f64(v), _f64(d_o)
+    B, Hq, Sq, d = q.shape
+    _, Hkv, Skv, _ = k.shape
+    dq = np.zeros(q.shape)
+    dk = np.zeros(k.shape)
+    dv = np.zeros(v.shape)
+    rc = lib.oracle_attn_bwd(_p(q), _p(k), _p(v), _p(d_o), _p(dq), _p(dk), _p(dv), B, Hq, Hkv,
+                             Sq, Skv, d, int(bool(causal)), float(scale))
+    if rc != 0:
+        raise ValueError("oracle_attn_bwd rejected its arguments")
+    return dq, dk, dv
 
 
 def attn_rows(q_rows, k, v, rows: Sequence[Sequence[int]], Hq: int, Sq: int,

@@ -315,6 +315,88 @@ int oracle_combine(const double *o_part, const double *lse_part, double *o,
     return 0;
 }
 
+/* Gradients of the forward pass above for a loss L with dL/dO = dO.
+ * "Tracing Tiled QKV Data Movement in FlashAttention's Memory Hierarchy"
+ * (closing takeaways) notes that the backward pass recomputes the attention
+ * matrix instead of storing it; the pages give no formulas, so this is the
+ * derivative of the definition, written out with the full row materialised:
+ *   P_ij  = exp(s_ij - LSE_i) over the visible keys,  s_ij = scale * q_i.k_j
+ *   dP_ij = dO_i . v_j
+ *   dS_ij = P_ij * (dP_ij - sum_l P_il dP_il)       (softmax Jacobian)
+ *   dq_i  = scale * sum_j dS_ij k_j
+ *   dk_j  = scale * sum_i dS_ij q_i   (over every query head of the group)
+ *   dv_j  = sum_i P_ij dO_i           (likewise)
+ * A row with no visible key contributes nothing.  Parallel over (b, kv head)
+ * so each thread owns the dk/dv rows it accumulates.
+ * Layouts: q, dO, dq [B,Hq,Sq,d]; k, v, dk, dv [B,Hkv,Skv,d]. */
+int oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dO,
+                    double *dq, double *dk, double *dv, int B, int Hq, int Hkv, int Sq,
+                    int Skv, int d, int causal, double scale)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Sq < 0 || Skv < 0 || d <= 0) return -1;
+    const int group = Hq / Hkv;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * (size_t)(Skv > 0 ? Skv : 1));
+        double *dp = (double *)malloc(sizeof(double) * (size_t)(Skv > 0 ? Skv : 1));
+        if (!p || !dp) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t bg = 0; bg < (int64_t)B * Hkv; ++bg) {
+                const int64_t b = bg / Hkv, g = bg % Hkv;
+                const double *kh = k + bg * (int64_t)Skv * d;
+                const double *vh = v + bg * (int64_t)Skv * d;
+                double *dkh = dk + bg * (int64_t)Skv * d;
+                double *dvh = dv + bg * (int64_t)Skv * d;
+                for (int64_t t = 0; t < (int64_t)Skv * d; ++t) { dkh[t] = 0.0; dvh[t] = 0.0; }
+                for (int64_t h = g * group; h < (g + 1) * group; ++h) {
+                    const int64_t bh = b * Hq + h;
+                    for (int64_t i = 0; i < Sq; ++i) {
+                        const double *qi = q + (bh * Sq + i) * d;
+                        const double *doi = dO + (bh * Sq + i) * d;
+                        double *dqi = dq + (bh * Sq + i) * d;
+                        for (int t = 0; t < d; ++t) dqi[t] = 0.0;
+                        const int64_t n = visible_keys(i, Sq, Skv, causal);
+                        if (n <= 0) continue;
+                        double m = -INFINITY;
+                        for (int64_t j = 0; j < n; ++j) {
+                            double acc = 0.0;
+                            for (int t = 0; t < d; ++t) acc += qi[t] * kh[j * d + t];
+                            p[j] = scale * acc;
+                            if (p[j] > m) m = p[j];
+                        }
+                        double z = 0.0;
+                        for (int64_t j = 0; j < n; ++j) z += exp(p[j] - m);
+                        const double lse = m + log(z);
+                        double dsum = 0.0;
+                        for (int64_t j = 0; j < n; ++j) {
+                            p[j] = exp(p[j] - lse);
+                            double acc = 0.0;
+                            for (int t = 0; t < d; ++t) acc += doi[t] * vh[j * d + t];
+                            dp[j] = acc;
+                            dsum += p[j] * acc;
+                        }
+                        for (int64_t j = 0; j < n; ++j) {
+                            const double ds = p[j] * (dp[j] - dsum);
+                            for (int t = 0; t < d; ++t) {
+                                dqi[t] += scale * ds * kh[j * d + t];
+                                dkh[j * d + t] += scale * ds * qi[t];
+                                dvh[j * d + t] += p[j] * doi[t];
+                            }
+                        }
+                    }
+                }
+            }
+        }
+        free(p);
+        free(dp);
+    }
+    return err ? -1 : 0;
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

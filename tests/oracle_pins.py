@@ -415,6 +415,86 @@ def pin_aligned_split(lib):
                         _close(lp[b, :, c], l3[0, :, 0], 1e-12, f"chunk {b},{c} LSE")
 
 
+def _loss(q, k, v, d_o, causal, scale, lib):
+    o, _ = oracle.attn_fwd(q, k, v, causal, scale, lib=lib)
+    return float(np.sum(o * d_o))
+
+
+def pin_bwd_finite_differences(lib):
+    """Each gradient the backward oracle returns matches a central finite
+    difference of L = sum(O * dO) through the forward oracle (a different
+    code path: only the forward definition is shared)."""
+    rng = np.random.default_rng(21)
+    for (B, Hq, Hkv, Sq, Skv, d, causal) in ((1, 4, 2, 7, 9, 5, True), (1, 2, 2, 6, 6, 4, False),
+                                             (2, 2, 1, 5, 3, 3, True)):
+        q = _rand((B, Hq, Sq, d), rng, 1.5)
+        k = _rand((B, Hkv, Skv, d), rng)
+        v = _rand((B, Hkv, Skv, d), rng)
+        d_o = _rand((B, Hq, Sq, d), rng)
+        scale = 0.7
+        grads = oracle.attn_bwd(q, k, v, d_o, causal, scale, lib=lib)
+        eps = 1e-5
+        for which, (x, g) in enumerate(zip((q, k, v), grads)):
+            flat = x.reshape(-1)
+            for idx in rng.choice(flat.size, size=min(12, flat.size), replace=False):
+                keep = flat[idx]
+                flat[idx] = keep + eps
+                lp = _loss(q, k, v, d_o, causal, scale, lib)
+                flat[idx] = keep - eps
+                lm = _loss(q, k, v, d_o, causal, scale, lib)
+                flat[idx] = keep
+                fd = (lp - lm) / (2 * eps)
+                got = g.reshape(-1)[idx]
+                assert abs(fd - got) <= 1e-7 * (1 + abs(fd)), \
+                    f"grad {'qkv'[which]}[{idx}] {got} vs finite difference {fd}"
+
+
+def pin_bwd_torch_autograd(lib):
+    """torch fp64 autograd through scaled_dot_product_attention (K/V repeated
+    per group, explicit bottom-right mask) gives the same gradients."""
+    rng = np.random.default_rng(22)
+    for (B, Hq, Hkv, Sq, Skv, d, causal) in ((2, 4, 4, 17, 17, 8, True), (1, 8, 2, 20, 20, 8, True),
+                                             (1, 4, 2, 19, 7, 8, True), (1, 2, 2, 12, 30, 16, False),
+                                             (1, 4, 1, 7, 19, 8, True)):
+        q = _rand((B, Hq, Sq, d), rng, 2.0)
+        k = _rand((B, Hkv, Skv, d), rng)
+        v = _rand((B, Hkv, Skv, d), rng)
+        d_o = _rand((B, Hq, Sq, d), rng)
+        scale = 1.0 / math.sqrt(d)
+        dq, dk, dv = oracle.attn_bwd(q, k, v, d_o, causal, scale, lib=lib)
+        tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+        grp = Hq // Hkv
+        mask = None
+        if causal:
+            i = torch.arange(Sq).unsqueeze(1)
+            j = torch.arange(Skv).unsqueeze(0)
+            mask = j <= i + (Skv - Sq)
+        s = (tq @ tk.repeat_interleave(grp, 1).transpose(-1, -2)) * scale
+        if mask is not None:
+            s = s.masked_fill(~mask, -math.inf)
+        pr = torch.softmax(s, dim=-1)
+        pr = torch.nan_to_num(pr, nan=0.0)  # rows with no visible key contribute nothing
+        o = pr @ tv.repeat_interleave(grp, 1)
+        o.backward(torch.tensor(d_o))
+        _close(dq, tq.grad.numpy(), 1e-10, "dq vs autograd")
+        _close(dk, tk.grad.numpy(), 1e-10, "dk vs autograd")
+        _close(dv, tv.grad.numpy(), 1e-10, "dv vs autograd")
+
+
+def pin_bwd_single_key(lib):
+    """One visible key: O = v_0 whatever q and k are, so dq = dk = 0 and
+    dv_0 = sum over query rows of dO."""
+    rng = np.random.default_rng(23)
+    q = _rand((1, 3, 4, 5), rng)
+    k = _rand((1, 1, 1, 5), rng)
+    v = _rand((1, 1, 1, 5), rng)
+    d_o = _rand((1, 3, 4, 5), rng)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, d_o, False, 0.9, lib=lib)
+    _close(dq, np.zeros_like(dq), 1e-14, "dq single key")
+    _close(dk, np.zeros_like(dk), 1e-14, "dk single key")
+    _close(dv[0, 0, 0], d_o.sum(axis=(0, 1, 2)), 1e-13, "dv single key")
+
+
 ALL_PINS = [
     pin_golden_prefill,
     pin_golden_combine,
@@ -429,4 +509,7 @@ ALL_PINS = [
     pin_paged_gather_by_hand,
     pin_paged_decode_equals_contiguous,
     pin_aligned_split,
+    pin_bwd_finite_differences,
+    pin_bwd_torch_autograd,
+    pin_bwd_single_key,
 ]

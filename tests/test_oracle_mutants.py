@@ -34,6 +34,11 @@ MUTANTS = [
      "const int64_t cs = cs0 / align * align;"),
     ("aligned_chunk_ignores_align", "const int64_t cs = (cs0 + align - 1) / align * align;",
      "const int64_t cs = cs0;"),
+    ("bwd_drops_softmax_jacobian_term", "const double ds = p[j] * (dp[j] - dsum);",
+     "const double ds = p[j] * dp[j];"),
+    ("bwd_dk_missing_scale", "dkh[j * d + t] += scale * ds * qi[t];", "dkh[j * d + t] += ds * qi[t];"),
+    ("bwd_dv_uses_dp", "dvh[j * d + t] += p[j] * doi[t];", "dvh[j * d + t] += dp[j] * doi[t];"),
+    ("bwd_dq_uses_query", "dqi[t] += scale * ds * kh[j * d + t];", "dqi[t] += scale * ds * qi[t];"),
 ]
 
 
