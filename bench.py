@@ -67,6 +67,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-paged", action="store_true",
                     help="skip the paged-cache decode measurement")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the backward measurement on the prefill workload")
     ap.add_argument("--page-size", type=int, default=16,
                     help="page size of the paged-cache decode measurement")
     return ap.parse_args()
@@ -383,6 +385,42 @@ def run_ours(args, world, rank, local):
                "d2h_bytes_per_step": int(o.numel() * 2 + lse.numel() * 4),
                "api": "io_aware_exact_flashattention_b200.flash_attention (host tensors)"}
 
+    # Backward on the prefill workload (dq, dk, dv from the forward's O and
+    # LSE), measured on its own after the step.
+    backward = None
+    if do_pre and not args.no_backward:
+        from io_aware_exact_flashattention_b200.inputs import grad_output
+        d_o = grad_output(q.shape, rank_seed(c.seed, rank), device=dev)
+        fa.fa_fwd(q, k, v, o, lse, c.causal, c.scale, stream=stream)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(fa.bwd_workspace_bytes(c.B, c.Hq, c.Sq, c.d), dtype=torch.uint8,
+                         device=dev)
+        for _ in range(max(args.warmup, 1)):
+            fa.fa_bwd(q, k, v, o, lse, d_o, dq, dk, dv, ws, c.causal, c.scale, stream=stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        bevs = []
+        for _ in range(K):
+            flush.fill_(1.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fa.fa_bwd(q, k, v, o, lse, d_o, dq, dk, dv, ws, c.causal, c.scale, stream=stream)
+            b.record(stream)
+            bevs.append((a, b))
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        bw_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in bevs)], world)[0]
+        bw_flops = 2.5 * flops
+        bw_tf = bw_flops / (bw_ms * 1e-3 / K) / 1e12
+        backward = {"value": aggregate_rate(world, bw_flops, K, bw_ms) / 1e12, "unit": "TFLOP/s",
+                    "ms_per_call": bw_ms / K, "frac_of_measured_burst": bw_tf / float(peaks["bf16_tflops"]),
+                    "frac_of_nominal_2250": bw_tf / NOMINAL_BF16_TFLOPS,
+                    "algorithmic": "%.4g FLOP per call (2.5 x the forward's: five products)" % bw_flops,
+                    "kernels": "fa_bwd_dsum_kernel + fa_bwd_kernel<128> + fa_bwd_dq_kernel (and a memset)",
+                    "gpu_launches": 3 * K,
+                    "note": "dq, dk, dv from the forward's O and LSE; measured outside the step"}
+        del dq, dk, dv, ws, d_o
+
     # Paged cache: the same decode workload stored in page_size-key pages
     # scattered over a pool, read through a block table.  Measured on its own,
     # outside the step.
@@ -491,6 +529,8 @@ def run_ours(args, world, rank, local):
         line["roofline"] = line.pop("roofline_decode")
     if paged is not None:
         line["decode_paged"] = paged
+    if backward is not None:
+        line["backward"] = backward
     if cpu is not None:
         line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)

@@ -30,6 +30,7 @@
 #ifndef FA_H_
 #define FA_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -74,6 +75,39 @@ typedef enum {
 fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
                  int B, int Hq, int Hkv, int Sq, int Skv, int d, int causal,
                  float scale, fa_stream_t stream);
+
+/*
+ * fa_bwd -- gradients of fa_fwd by recomputation.
+ *
+ * "Tracing Tiled QKV Data Movement in FlashAttention's Memory Hierarchy"
+ * (closing takeaways) notes that the backward pass recomputes the attention
+ * matrix from the inputs instead of storing it.  With the forward's LSE,
+ * P_ij = exp(scale * q_i.k_j - LSE_i) over the visible keys, D_i = dO_i . O_i
+ * and dS_ij = P_ij * (dO_i . v_j - D_i):
+ *
+ *   dq_i = scale * sum_j dS_ij k_j
+ *   dk_j = scale * sum_i dS_ij q_i   (summed over the query heads of j's group)
+ *   dv_j = sum_i P_ij dO_i           (likewise)
+ *
+ *   q, o, d_o, dq [B, Hq, Sq, d] bf16     k, v, dk, dv [B, Hkv, Skv, d] bf16
+ *   lse           [B, Hq, Sq] fp32 (natural log, as fa_fwd writes it)
+ *   workspace     fa_bwd_workspace_bytes(B, Hq, Sq, d) bytes, 16-byte aligned,
+ *                 caller-owned scratch (fp32 dq accumulator, then D); its
+ *                 contents on entry do not matter
+ *   causal, scale: as passed to fa_fwd.
+ *
+ * dq, dk, dv are written (dk = dv = 0 for keys no query sees).  P and dS
+ * enter the tensor-core products as bf16; accumulation is fp32.
+ * Supported: d in {64, 128}; Hq % Hkv == 0.  All pointers 16-byte aligned.
+ * Errors as for fa_fwd.
+ */
+fa_status fa_bwd(const void *q, const void *k, const void *v, const void *o,
+                 const float *lse, const void *d_o, void *dq, void *dk, void *dv,
+                 float *workspace, int B, int Hq, int Hkv, int Sq, int Skv, int d,
+                 int causal, float scale, fa_stream_t stream);
+
+/* Bytes of scratch fa_bwd needs: B * Hq * Sq * (d + 1) floats (0 for empty). */
+size_t fa_bwd_workspace_bytes(int B, int Hq, int Sq, int d);
 
 /*
  * fa_decode_splitkv -- first half of single-query decode (Sq = 1, no mask).

@@ -15,6 +15,7 @@
 #include "sm100.cuh"
 #include "prefill_sm100.cuh"
 #include "decode_sm100.cuh"
+#include "backward_sm100.cuh"
 
 namespace {
 
@@ -308,7 +309,117 @@ __global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict_
 
 }  // namespace
 
+// Backward: per-device shared-memory opt-in.
+std::once_flag g_bwd_once[kMaxDevices];
+cudaError_t g_bwd_err[kMaxDevices];
+
+cudaError_t prepare_backward(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::call_once(g_bwd_once[dev], [dev] {
+    cudaError_t e = cudaFuncSetAttribute(fa::fa_bwd_kernel<64>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         fa::BwdLayout<64>::kBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fa::fa_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::BwdLayout<128>::kBytes);
+    g_bwd_err[dev] = e;
+  });
+  return g_bwd_err[dev];
+}
+
+template <int D>
+fa_status launch_backward(const void* q, const void* k, const void* v, const void* o,
+                          const float* lse, const void* d_o, void* dq, void* dk, void* dv,
+                          float* workspace, int B, int Hq, int Hkv, int Sq, int Skv, int causal,
+                          float scale, cudaStream_t stream) {
+  const long long q_rows = static_cast<long long>(B) * Hq * Sq;
+  float* dq_acc = workspace;
+  float* dsum = workspace + q_rows * D;
+  if (cudaMemsetAsync(dq_acc, 0, static_cast<size_t>(q_rows) * D * sizeof(float), stream) !=
+      cudaSuccess)
+    return FA_ERR_CUDA;
+  fa::fa_bwd_dsum_kernel<D><<<static_cast<unsigned>((q_rows + 7) / 8), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o), dsum, q_rows);
+  const int n_kv_tiles = (Skv + fa::kBwdBM - 1) / fa::kBwdBM;
+  if (n_kv_tiles > 0) {
+    CUtensorMap tq, tk, tv, tdo;
+    if (!encode_bhsd(&tq, q, D, Sq, static_cast<long long>(B) * Hq) ||
+        !encode_bhsd(&tdo, d_o, D, Sq, static_cast<long long>(B) * Hq) ||
+        !encode_bhsd(&tk, k, D, Skv, static_cast<long long>(B) * Hkv) ||
+        !encode_bhsd(&tv, v, D, Skv, static_cast<long long>(B) * Hkv))
+      return FA_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+    if (prepare_backward(dev) != cudaSuccess) return FA_ERR_CUDA;
+    fa::BwdParams p;
+    p.dq_acc = dq_acc;
+    p.lse = lse;
+    p.dsum = dsum;
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Sq = Sq;
+    p.Skv = Skv;
+    p.group = Hq / Hkv;
+    p.causal = causal ? 1 : 0;
+    p.n_kv_tiles = n_kv_tiles;
+    p.n_q_tiles = (Sq + fa::kBwdBN - 1) / fa::kBwdBN;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.wait_limit_ns = kWaitLimitNs;
+    const unsigned grid = static_cast<unsigned>(static_cast<long long>(B) * Hkv * n_kv_tiles);
+    fa::fa_bwd_kernel<D><<<grid, fa::kBwdThreads, fa::BwdLayout<D>::kBytes, stream>>>(tq, tk, tv,
+                                                                                      tdo, p);
+  }
+  const long long n = q_rows * D;
+  fa::fa_bwd_dq_kernel<<<static_cast<unsigned>((n / 4 + 255) / 256), 256, 0, stream>>>(
+      dq_acc, static_cast<__nv_bfloat16*>(dq), n);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 extern "C" {
+
+size_t fa_bwd_workspace_bytes(int B, int Hq, int Sq, int d) {
+  if (B <= 0 || Hq <= 0 || Sq <= 0 || d <= 0) return 0;
+  return static_cast<size_t>(B) * Hq * Sq * (static_cast<size_t>(d) + 1) * sizeof(float);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* d_o, void* dq, void* dk, void* dv, float* workspace, int B, int Hq,
+                 int Hkv, int Sq, int Skv, int d, int causal, float scale, fa_stream_t stream) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || Sq < 0 || Skv < 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || (Sq == 0 && Skv == 0)) return FA_OK;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr ||
+      d_o == nullptr || dq == nullptr || dk == nullptr || dv == nullptr || workspace == nullptr)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(d_o) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      !aligned16(workspace))
+    return FA_ERR_ALIGNMENT;
+  const long long n_kv_tiles = (static_cast<long long>(Skv) + fa::kBwdBM - 1) / fa::kBwdBM;
+  const long long q_elems = static_cast<long long>(B) * Hq * Sq * d;
+  if (static_cast<long long>(B) * Hkv * n_kv_tiles > 0x7fffffffLL ||
+      static_cast<long long>(B) * Hq > 0x7fffffffLL || q_elems / 4 / 256 > 0x7fffffffLL ||
+      static_cast<long long>(B) * Hkv > 0x7fffffffLL)
+    return FA_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (Sq == 0) {  // no query rows: every key gets zero gradients
+    const size_t kv_bytes = static_cast<size_t>(B) * Hkv * Skv * d * 2;
+    if (cudaMemsetAsync(dk, 0, kv_bytes, s) != cudaSuccess ||
+        cudaMemsetAsync(dv, 0, kv_bytes, s) != cudaSuccess)
+      return FA_ERR_CUDA;
+    return FA_OK;
+  }
+  return d == 64 ? launch_backward<64>(q, k, v, o, lse, d_o, dq, dk, dv, workspace, B, Hq, Hkv,
+                                       Sq, Skv, causal, scale, s)
+                 : launch_backward<128>(q, k, v, o, lse, d_o, dq, dk, dv, workspace, B, Hq, Hkv,
+                                        Sq, Skv, causal, scale, s);
+}
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                  int Hkv, int Sq, int Skv, int d, int causal, float scale, fa_stream_t stream) {

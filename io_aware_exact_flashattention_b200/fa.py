@@ -35,6 +35,8 @@ SIGNATURES = {
     "fa_decode_splitkv": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP]),
     "fa_decode_paged_splitkv": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP] + [_I] * 8 + [_F, _VP]),
     "fa_combine": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP]),
+    "fa_bwd": (_I, [_VP] * 10 + [_I] * 7 + [_F, _VP]),
+    "fa_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "fa_decode_default_splits": (_I, [_I, _I, _I, _I]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_get_device_status": (_I, []),
@@ -116,6 +118,55 @@ def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
         raise ValueError("output shapes do not match q")
     _check("fa_fwd", lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Sq,
                                   Skv, d, int(bool(causal)), float(scale), _stream_ptr(stream)))
+
+
+def bwd_workspace_bytes(B: int, Hq: int, Sq: int, d: int) -> int:
+    return int(lib().fa_bwd_workspace_bytes(B, Hq, Sq, d))
+
+
+def fa_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+           lse: torch.Tensor, d_o: torch.Tensor, dq: torch.Tensor, dk: torch.Tensor,
+           dv: torch.Tensor, workspace: torch.Tensor, causal: bool, scale: float,
+           stream: Optional[torch.cuda.Stream] = None) -> None:
+    """fa_bwd: gradients dq [B,Hq,Sq,d], dk/dv [B,Hkv,Skv,d] (bf16) from q, k, v,
+    the forward's o and lse, and d_o; workspace is a uint8/float tensor of at
+    least bwd_workspace_bytes() bytes."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (d_o, "d_o"), (dq, "dq"), (dk, "dk"),
+                 (dv, "dv")):
+        _need(t, torch.bfloat16, n)
+    _need(lse, torch.float32, "lse")
+    B, Hq, Sq, d = q.shape
+    _, Hkv, Skv, _ = k.shape
+    for t, shp, n in ((o, q.shape, "o"), (d_o, q.shape, "d_o"), (dq, q.shape, "dq"),
+                      (v, k.shape, "v"), (dk, k.shape, "dk"), (dv, k.shape, "dv")):
+        if tuple(t.shape) != tuple(shp):
+            raise ValueError("%s must have shape %s" % (n, tuple(shp)))
+    if tuple(lse.shape) != (B, Hq, Sq):
+        raise ValueError("lse must be [B,Hq,Sq]")
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    if workspace.numel() * workspace.element_size() < bwd_workspace_bytes(B, Hq, Sq, d):
+        raise ValueError("workspace too small")
+    _check("fa_bwd", lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(d_o),
+                                  _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), B, Hq, Hkv, Sq,
+                                  Skv, d, int(bool(causal)), float(scale), _stream_ptr(stream)))
+
+
+def attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                       lse: torch.Tensor, d_o: torch.Tensor, causal: bool = False,
+                       scale: Optional[float] = None
+                       ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """(dq, dk, dv) for CUDA tensors, allocating the outputs and the workspace."""
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    B, Hq, Sq, d = q.shape
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    ws = torch.empty(max(16, bwd_workspace_bytes(B, Hq, Sq, d)), dtype=torch.uint8,
+                     device=q.device)
+    fa_bwd(q, k, v, o, lse, d_o, dq, dk, dv, ws, causal, scale)
+    return dq, dk, dv
 
 
 def fa_decode_splitkv(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,

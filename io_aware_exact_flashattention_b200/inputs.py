@@ -182,3 +182,11 @@ def paged_decode_inputs(B: int, Hq: int, Hkv: int, Lmin: int, Lmax: int, d: int,
     q, kc, vc, seqlens = decode_inputs(B, Hq, Hkv, Lmin, Lmax, d, seed, device, pad_value)
     k_pages, v_pages, table = paginate(kc, vc, seqlens, page_size, seed, pad_value)
     return q, k_pages, v_pages, table, seqlens
+
+
+def grad_output(shape, seed: int, device="cpu"):
+    """dL/dO for backward tests and benchmarks: N(0,1), bf16, its own seed."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed) + 104729)
+    return torch.randn(tuple(shape), generator=g, device=device,
+                       dtype=torch.float32).to(torch.bfloat16).contiguous()

@@ -128,6 +128,32 @@ def test_paged_decode_rejects_before_cuda(lib, kw, want):
     assert paged(lib, **kw) == want
 
 
+def bwd(lib, *, q=A, k=A, v=A, o=A, lse=A, do=A, dq=A, dk=A, dv=A, ws=A, B=1, Hq=4, Hkv=2,
+        Sq=128, Skv=128, d=128, causal=1, scale=0.1):
+    return lib.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, B, Hq, Hkv, Sq, Skv, d, causal, scale,
+                      None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(d=96), UNSUPPORTED),
+    (dict(Hq=4, Hkv=3), INVALID),
+    (dict(Sq=-1), INVALID),
+    (dict(scale=float("nan")), INVALID),
+    (dict(ws=None), INVALID),
+    (dict(do=None), INVALID),
+    (dict(dk=A + 8), ALIGNMENT),
+    (dict(ws=A + 4), ALIGNMENT),
+    (dict(B=0, q=None), OK),
+])
+def test_bwd_rejects_before_cuda(lib, kw, want):
+    assert bwd(lib, **kw) == want
+
+
+def test_bwd_workspace_bytes(lib):
+    assert fa.bwd_workspace_bytes(2, 4, 100, 128) == 2 * 4 * 100 * 129 * 4
+    assert fa.bwd_workspace_bytes(0, 4, 100, 128) == 0
+
+
 @pytest.mark.parametrize("args,want", [
     ((A, A, A, A, 2, 8, 0, 128), INVALID),
     ((A, A, A, A, 2, 8, 4, 96), UNSUPPORTED),

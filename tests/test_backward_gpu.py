@@ -1,0 +1,89 @@
+"""fa_bwd (through the C ABI) against the fp64 oracle's exact gradients on a
+B200.  The kernel gets the forward's own O and LSE (from fa_fwd), as a
+training step would; the oracle recomputes everything from q, k, v and dO.
+
+Tolerance.  P and dS enter the tensor-core products as bf16 (relative
+rounding 2^-9 each), D = dO . O uses the bf16-rounded forward output, and
+dq, dk, dv are rounded to bf16 (2^-9 relative); sums over up to Sq or Skv
+terms accumulate in fp32.  Errors are therefore relative to each gradient's
+scale: max |d - ref| <= GRAD_TOL * max |ref| for each of dq, dk, dv, with
+GRAD_TOL = 2e-2 (a few 2^-9 roundings, with margin for the cancellation in
+dP - D), and the Frobenius norm of the error within 1e-2 of the reference's.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from io_aware_exact_flashattention_b200 import fa
+from io_aware_exact_flashattention_b200.inputs import grad_output, prefill_inputs
+
+pytestmark = pytest.mark.gpu
+
+GRAD_TOL = 2e-2
+FRO_TOL = 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    fa.lib()
+
+
+def run_bwd(B, Hq, Hkv, Sq, Skv, d, causal, seed, q_mult=1.0, scale=None):
+    q, k, v = prefill_inputs(B, Hq, Hkv, Sq, Skv, d, seed, q_mult)
+    d_o = grad_output((B, Hq, Sq, d), seed)
+    scale = scale if scale is not None else 1.0 / math.sqrt(d)
+    qc, kc, vc, doc = (t.cuda() for t in (q, k, v, d_o))
+    o = torch.empty_like(qc)
+    lse = torch.empty((B, Hq, Sq), device="cuda", dtype=torch.float32)
+    fa.fa_fwd(qc, kc, vc, o, lse, causal, scale)
+    dq, dk, dv = fa.attention_backward(qc, kc, vc, o, lse, doc, causal, scale)
+    torch.cuda.synchronize()
+    ref = oracle.attn_bwd(q, k, v, d_o, causal, scale)
+    errs = {}
+    for name, got, want in (("dq", dq, ref[0]), ("dk", dk, ref[1]), ("dv", dv, ref[2])):
+        g = got.float().cpu().numpy().astype(np.float64)
+        assert np.isfinite(g).all(), name + ": non-finite"
+        scale_ref = max(float(np.abs(want).max()), 1e-30)
+        e_max = float(np.abs(g - want).max()) / scale_ref if g.size else 0.0
+        e_fro = (float(np.linalg.norm(g - want)) / max(float(np.linalg.norm(want)), 1e-30)
+                 if g.size else 0.0)
+        errs[name] = (e_max, e_fro)
+    return errs
+
+
+def check(errs):
+    for name, (e_max, e_fro) in errs.items():
+        assert e_max <= GRAD_TOL and e_fro <= FRO_TOL, "%s: max %.3e fro %.3e (%s)" % (
+            name, e_max, e_fro, errs)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_square(d, causal):
+    check(run_bwd(1, 2, 2, 300, 300, d, causal, seed=40 + d + causal))
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (4, 1)])
+def test_gqa(Hq, Hkv):
+    check(run_bwd(2, Hq, Hkv, 257, 257, 128, True, seed=50 + Hq))
+
+
+@pytest.mark.parametrize("Sq,Skv", [(150, 400), (400, 150), (128, 384)])
+def test_rectangular_causal(Sq, Skv):
+    # Sq > Skv: the first Sq - Skv query rows see no key (zero gradients there)
+    check(run_bwd(1, 4, 2, Sq, Skv, 128, True, seed=60 + Sq))
+
+
+def test_large_logits_q_times_8():
+    check(run_bwd(1, 2, 2, 512, 512, 128, True, seed=70, q_mult=8.0))
+
+
+def test_headline_shape_sampled_heads():
+    """The forward's headline shape (causal MHA, S=2048, d=128, Q*8), two heads
+    (the oracle's fp64 backward on all 64 heads would take minutes)."""
+    check(run_bwd(1, 2, 2, 2048, 2048, 128, True, seed=2, q_mult=8.0))
