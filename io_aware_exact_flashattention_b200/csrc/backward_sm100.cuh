@@ -17,13 +17,16 @@
 //   dV  += P^T dO_i       (A = P^T in TMEM, B = dO_i MN-major; TS)
 //   dK  += dS^T Q_i       (A = dS^T in TMEM, B = Q_i MN-major; TS)
 //   dQ_i = dS K_j         (A = dS from shared memory MN-major, B = K_j MN-major; SS)
-// Roles (192 threads):
-//   warps 0-3  thread = key row: P and dS from S^T, dP^T, LSE and D; the dQ
-//              partial (thread = query row) into the workspace; dK, dV out
-//   warp  4    TMA producer: K_j, V_j once, then Q_i and dO_i (two stages)
-//   warp  5    MMA issuer; allocates tensor memory
-// Tensor memory columns: dV [0,128), dK [128,256), S^T / P / dQ partial
-// [256,384), dP^T / dS [384,512).
+// Roles (320 threads):
+//   warps 0-7  two warpgroups, each half of every tile's queries: thread =
+//              key row for P and dS (from S^T, dP^T, LSE and D); thread =
+//              query row for the dQ partial (half the d-columns each) into
+//              the workspace; dK, dV out
+//   warp  8    TMA producer: K_j, V_j once, then Q_i and dO_i (two stages)
+//   warp  9    MMA issuer; allocates tensor memory
+// Tensor memory columns: dV [0,128), dK [128,256), S^T / P [256,384),
+// dP^T / dS / dQ partial [384,512).  The next tile's S^T is issued as soon as
+// dQ_i is, so it runs while dQ_i is read out; its dP^T waits for the read-out.
 #pragma once
 
 #include <cuda.h>
@@ -32,7 +35,7 @@
 
 namespace fa {
 
-constexpr int kBwdThreads = 192;
+constexpr int kBwdThreads = 320;
 constexpr int kBwdBM = 128;  // keys per CTA (TMEM lanes)
 constexpr int kBwdBN = 128;  // queries per tile
 
@@ -51,10 +54,10 @@ struct BwdLayout {
   static constexpr int kBQEmpty = 3;   // [2]
   static constexpr int kBSFull = 5;
   static constexpr int kBDpFull = 6;
-  static constexpr int kBPFull = 7;    // 128 arrivals
-  static constexpr int kBDsFull = 8;   // 128 arrivals
+  static constexpr int kBPFull = 7;    // 256 arrivals
+  static constexpr int kBDsFull = 8;   // 256 arrivals
   static constexpr int kBDqFull = 9;
-  static constexpr int kBSFree = 10;   // 128 arrivals: dQ partial read out of the S columns
+  static constexpr int kBSFree = 10;   // 256 arrivals: dQ partial read out of the dP columns
   static constexpr int kBDone = 11;
   static constexpr int kNumBars = 12;
   static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
@@ -203,6 +206,12 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, uint32_t sbase, uint
   const int i0 = bwd_first_q_tile(p, j);
   const int per_head = p.n_q_tiles - i0;
   const uint32_t total = per_head > 0 ? static_cast<uint32_t>(per_head * p.group) : 0u;
+  // TMEM column of the packed bf16 pairs for queries 16*kk .. 16*kk+15: each
+  // warpgroup packs its 64 queries at the start of its own 64 columns
+  auto packed_col = [](int kk) -> uint32_t {
+    constexpr int kSteps = kBwdBN / 16;
+    return static_cast<uint32_t>(kk * 8 + (kk >= kSteps / 2 ? 32 : 0));
+  };
   auto wait = [&](int bar, uint32_t parity) -> bool {
     if (!mbar_wait(bars + 8 * bar, parity, abort_flag, p.wait_limit_ns)) return false;
     tc_fence_after();
@@ -217,34 +226,46 @@ __device__ __forceinline__ void bwd_mma(const BwdParams& p, uint32_t sbase, uint
              kk > 0 ? 1u : 0u);
     }
   };
-  if (total > 0 && !wait(L::kBKv, 0u)) goto done;
+  if (total > 0) {
+    if (!wait(L::kBKv, 0u) || !wait(L::kBQFull + 0, 0u)) goto done;
+    gemm_kmajor(t_s, ka, sbase + L::kQOff);                        // S^T = K Q^T
+    mma_commit(bars + 8 * L::kBSFull);
+    gemm_kmajor(t_dp, va, sbase + L::kQOff + L::kTileBytes);       // dP^T = V dO^T
+    mma_commit(bars + 8 * L::kBDpFull);
+  }
   for (uint32_t n = 0; n < total; ++n) {
     const uint32_t s = n & 1u, ph = n & 1u;
     const uint32_t qa = sbase + L::kQOff + 2 * s * L::kTileBytes;
     const uint32_t doa = qa + L::kTileBytes;
-    if (!wait(L::kBQFull + s, (n >> 1) & 1u)) goto done;
-    // the S columns hold the previous tile's dQ partial until it is read out
-    if (n > 0 && !wait(L::kBSFree, (n - 1) & 1u)) goto done;
-    gemm_kmajor(t_s, ka, qa);                      // S^T = K Q^T
-    mma_commit(bars + 8 * L::kBSFull);
-    gemm_kmajor(t_dp, va, doa);                    // dP^T = V dO^T
-    mma_commit(bars + 8 * L::kBDpFull);
     if (!wait(L::kBPFull, ph)) goto done;
 #pragma unroll
     for (int kk = 0; kk < kBwdBN / 16; ++kk)       // dV += P^T dO
-      mma_ts(t_dv, t_s + kk * 8, sw128_desc(doa + kk * 16 * 128, L::kBoxBytes, 1024), kIdAcc,
-             (n > 0 || kk > 0) ? 1u : 0u);
+      mma_ts(t_dv, t_s + packed_col(kk), sw128_desc(doa + kk * 16 * 128, L::kBoxBytes, 1024),
+             kIdAcc, (n > 0 || kk > 0) ? 1u : 0u);
     if (!wait(L::kBDsFull, ph)) goto done;
 #pragma unroll
     for (int kk = 0; kk < kBwdBN / 16; ++kk)       // dK += dS^T Q
-      mma_ts(t_dk, t_dp + kk * 8, sw128_desc(qa + kk * 16 * 128, L::kBoxBytes, 1024), kIdAcc,
-             (n > 0 || kk > 0) ? 1u : 0u);
+      mma_ts(t_dk, t_dp + packed_col(kk), sw128_desc(qa + kk * 16 * 128, L::kBoxBytes, 1024),
+             kIdAcc, (n > 0 || kk > 0) ? 1u : 0u);
     mma_commit(bars + 8 * (L::kBQEmpty + s));     // Q_i, dO_i read by everything issued so far
+    // dQ_i = dS K (K = keys) into the dP^T / dS columns (dS already read by dK)
 #pragma unroll
-    for (int kk = 0; kk < kBwdBM / 16; ++kk)       // dQ_i = dS K (K = keys)
-      mma_ss(t_s, sw128_desc(dsa + kk * 16 * 128, L::kBoxBytes, 1024),
+    for (int kk = 0; kk < kBwdBM / 16; ++kk)
+      mma_ss(t_dp, sw128_desc(dsa + kk * 16 * 128, L::kBoxBytes, 1024),
              sw128_desc(ka + kk * 16 * 128, L::kBoxBytes, 1024), kIdDq, kk > 0 ? 1u : 0u);
     mma_commit(bars + 8 * L::kBDqFull);
+    if (n + 1 < total) {
+      // next tile's scores while dQ_i is read out (P_i was read by dV already)
+      const uint32_t s1 = (n + 1) & 1u;
+      const uint32_t qa1 = sbase + L::kQOff + 2 * s1 * L::kTileBytes;
+      if (!wait(L::kBQFull + s1, ((n + 1) >> 1) & 1u)) goto done;
+      gemm_kmajor(t_s, ka, qa1);
+      mma_commit(bars + 8 * L::kBSFull);
+      // dP^T of the next tile once dQ_i has left the dP^T columns
+      if (!wait(L::kBSFree, ph)) goto done;
+      gemm_kmajor(t_dp, va, qa1 + L::kTileBytes);
+      mma_commit(bars + 8 * L::kBDpFull);
+    }
   }
 done:
   mma_commit(bars + 8 * L::kBDone);
@@ -252,19 +273,24 @@ done:
 }
 
 // ---------------------------------------------------------------------------
-// Element-wise warpgroup (warps 0-3): thread t = key row t of the tile for P
-// and dS, query row t for the dQ partial.
+// Element-wise warpgroups (warps 0-7).  Warpgroup hf takes queries
+// [64*hf, 64*hf + 64) of each tile for P and dS (thread t = key row t, the
+// TMEM lane) and d-columns [hf*D/2, (hf+1)*D/2) for the dQ partial (thread t
+// = query row t) and for dK, dV; the two halves run side by side.
 // ---------------------------------------------------------------------------
 template <int D>
 __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, uint32_t sbase, uint8_t* smem,
                                                 uint32_t tmem, volatile int* abort_flag) {
   using L = BwdLayout<D>;
   const uint32_t bars = sbase + L::kBarOff;
-  const int t = threadIdx.x;  // 0..127
-  const int warp = t >> 5;
+  const int t = threadIdx.x & 127;
+  const int hf = threadIdx.x >> 7;  // warpgroup: query half / column half
+  const int warp = (threadIdx.x >> 5) & 3;
   const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
   const uint32_t t_dv = tmem + lane_off, t_dk = tmem + lane_off + 128;
   const uint32_t t_s = tmem + lane_off + 256, t_dp = tmem + lane_off + 384;
+  constexpr int kQH = kBwdBN / 2;   // queries per warpgroup
+  constexpr int kDH = D / 2;        // d-columns per warpgroup
   float* lse_s = reinterpret_cast<float*>(smem + L::kLseOff);
   float* d_s = lse_s + 128;
   uint8_t* ds_smem = smem + L::kDsOff;
@@ -275,7 +301,7 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, uint32_t sba
   const int i0 = bwd_first_q_tile(p, j);
   uint32_t n = 0;
   // After a failed wait a warp skips the remaining work but still takes every
-  // named barrier, so the other warps of the warpgroup can never block there.
+  // named barrier, so the other warps of its warpgroup can never block there.
   bool ok = true;
   for (int hh = 0; hh < p.group; ++hh) {
     const int h = g * p.group + hh;
@@ -283,50 +309,43 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, uint32_t sba
     for (int i = i0; i < p.n_q_tiles; ++i, ++n) {
       const uint32_t ph = n & 1u;
       const int q0 = i * kBwdBN;
-      // LSE (in log2 units) and D of this tile's queries, shared by the warpgroup
-      named_barrier(1, 128);
-      {
-        const int q = q0 + t;
-        lse_s[t] = (q < p.Sq) ? p.lse[row_base + q] * 1.4426950408889634f : INFINITY;
-        d_s[t] = (q < p.Sq) ? p.dsum[row_base + q] : 0.f;
+      // LSE (in log2 units) and D of this warpgroup's 64 queries
+      named_barrier(1 + hf, 128);
+      if (t < kQH) {
+        const int c = hf * kQH + t;
+        const int q = q0 + c;
+        lse_s[c] = (q < p.Sq) ? p.lse[row_base + q] * 1.4426950408889634f : INFINITY;
+        d_s[c] = (q < p.Sq) ? p.dsum[row_base + q] : 0.f;
       }
-      named_barrier(1, 128);
+      named_barrier(1 + hf, 128);
 
       if (!ok) continue;
-      // P^T row of this key: p = 2^(s*scale*log2e - LSE*log2e), 0 where masked
+      // P^T for this key and the warpgroup's queries: p = 2^(s*scale*log2e - LSE*log2e)
       ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * L::kBSFull, ph, abort_flag, p.wait_limit_ns));
       if (!ok) continue;
       tc_fence_after();
-      uint32_t pk[64];
+      uint32_t pk[kQH / 2];
       {
-        uint32_t ra[64], rb[64];
-        tmem_ld64_nowait(t_s, ra);
-        tmem_ld64_nowait(t_s + 64, rb);
+        uint32_t ra[64];
+        tmem_ld64_nowait(t_s + hf * kQH, ra);
         tmem_ld_wait_hold(ra);
-        tmem_ld_wait_hold(rb);
-        // key visible to query q iff key <= q + off and key < Skv
-        const int lim = key - off;  // first visible query
+        const int lim = key - off;  // first query that sees this key
 #pragma unroll
-        for (int c2 = 0; c2 < 64; ++c2) {
+        for (int c2 = 0; c2 < kQH / 2; ++c2) {
           float pr[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int c = 2 * c2 + e;
-            const float sv = __uint_as_float(c < 64 ? ra[c] : rb[c - 64]);
+            const int c = hf * kQH + 2 * c2 + e;
             const bool vis = (key < p.Skv) && (!p.causal || q0 + c >= lim);
-            const float x = fmaf(sv, p.scale_log2, -lse_s[c]);
+            const float x = fmaf(__uint_as_float(ra[2 * c2 + e]), p.scale_log2, -lse_s[c]);
             pr[e] = vis ? ex2(x) : 0.f;
           }
           pk[c2] = pack_bf16x2(pr[0], pr[1]);
         }
       }
-      {
-        uint32_t h0[32], h1[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) { h0[e] = pk[e]; h1[e] = pk[32 + e]; }
-        tmem_st32(t_s, h0);
-        tmem_st32(t_s + 32, h1);
-      }
+      // packed pairs of queries, inside this warpgroup's own (already read)
+      // score columns: the other warpgroup's scores are never overwritten
+      tmem_st32(t_s + hf * kQH, pk);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bars + 8 * L::kBPFull);
@@ -337,24 +356,25 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, uint32_t sba
       if (!ok) continue;
       tc_fence_after();
 #pragma unroll
-      for (int hq = 0; hq < 4; ++hq) {  // 32 queries per pass
+      for (int hq = 0; hq < 2; ++hq) {  // 32 queries per pass
         uint32_t dp[32];
-        tmem_ld32(t_dp + hq * 32, dp);
+        tmem_ld32(t_dp + hf * kQH + hq * 32, dp);
         uint32_t dsk[16];
 #pragma unroll
         for (int e2 = 0; e2 < 16; ++e2) {
-          const int c = hq * 32 + 2 * e2;
-          const __nv_bfloat162 pb = *reinterpret_cast<const __nv_bfloat162*>(&pk[c >> 1]);
+          const int cl = hq * 32 + 2 * e2;  // local query index in the half
+          const __nv_bfloat162 pb = *reinterpret_cast<const __nv_bfloat162*>(&pk[cl >> 1]);
+          const int c = hf * kQH + cl;
           const float d0 = __bfloat162float(pb.x) * (__uint_as_float(dp[2 * e2]) - d_s[c]);
           const float d1 = __bfloat162float(pb.y) * (__uint_as_float(dp[2 * e2 + 1]) - d_s[c + 1]);
           dsk[e2] = pack_bf16x2(d0, d1);
         }
-        tmem_st16(t_dp + hq * 16, dsk);
-        // queries hq*32 .. +31 = box hq/2, 16-byte chunks (hq%2)*4 .. +3 of row t
+        tmem_st16(t_dp + hf * kQH + hq * 16, dsk);  // own columns, already read
+        // queries hf*64 + hq*32 .. +31: box hf, 16-byte chunks hq*4 .. +3 of row t
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
-          const int chunk = (hq & 1) * 4 + k4;
-          uint4* dst = reinterpret_cast<uint4*>(ds_smem + (hq >> 1) * L::kBoxBytes + t * 128 +
+          const int chunk = hq * 4 + k4;
+          uint4* dst = reinterpret_cast<uint4*>(ds_smem + hf * L::kBoxBytes + t * 128 +
                                                 ((chunk ^ (t & 7)) * 16));
           *dst = make_uint4(dsk[4 * k4], dsk[4 * k4 + 1], dsk[4 * k4 + 2], dsk[4 * k4 + 3]);
         }
@@ -364,17 +384,17 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, uint32_t sba
       tc_fence_before();
       mbar_arrive(bars + 8 * L::kBDsFull);
 
-      // dQ partial (thread = query row q0 + t) into the fp32 workspace
+      // dQ partial (thread = query row q0 + t, this warpgroup's d-columns)
       ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * L::kBDqFull, ph, abort_flag, p.wait_limit_ns));
       if (!ok) continue;
       tc_fence_after();
       {
         const int q = q0 + t;
-        float* dst = p.dq_acc + (row_base + q) * D;
+        float* dst = p.dq_acc + (row_base + q) * D + hf * kDH;
 #pragma unroll
-        for (int c4 = 0; c4 < D / 32; ++c4) {
+        for (int c4 = 0; c4 < kDH / 32; ++c4) {
           uint32_t r[32];
-          tmem_ld32(t_s + c4 * 32, r);
+          tmem_ld32(t_dp + hf * kDH + c4 * 32, r);
           if (q < p.Sq) {
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
@@ -390,7 +410,8 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, uint32_t sba
   }
   if (!ok) return;
 
-  // dK = scale * (dS^T Q summed), dV = P^T dO summed: thread t = key row
+  // dK = scale * (dS^T Q summed), dV = P^T dO summed: thread t = key row,
+  // this warpgroup's d-columns
   if (!__all_sync(0xffffffffu, mbar_wait(bars + 8 * L::kBDone, 0u, abort_flag, p.wait_limit_ns)))
     return;
   tc_fence_after();
@@ -401,12 +422,12 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, uint32_t sba
   const size_t krow = (static_cast<size_t>(b) * p.Hkv + g) * p.Skv + (real ? key : 0);
 #pragma unroll
   for (int which = 0; which < 2; ++which) {
-    __nv_bfloat16* out = (which == 0 ? p.dv : p.dk) + krow * D;
+    __nv_bfloat16* out = (which == 0 ? p.dv : p.dk) + krow * D + hf * kDH;
     const float mul = (which == 0) ? 1.f : p.scale;
 #pragma unroll
-    for (int c4 = 0; c4 < D / 32; ++c4) {
+    for (int c4 = 0; c4 < kDH / 32; ++c4) {
       uint32_t r[32];
-      tmem_ld32((which == 0 ? t_dv : t_dk) + c4 * 32, r);
+      tmem_ld32((which == 0 ? t_dv : t_dk) + hf * kDH + c4 * 32, r);
       if (real) {
 #pragma unroll
         for (int v4 = 0; v4 < 4; ++v4) {
@@ -445,15 +466,15 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
     mbar_init(bars + 8 * L::kBSFull, 1);
     mbar_init(bars + 8 * L::kBDpFull, 1);
-    mbar_init(bars + 8 * L::kBPFull, 128);
-    mbar_init(bars + 8 * L::kBDsFull, 128);
+    mbar_init(bars + 8 * L::kBPFull, 256);
+    mbar_init(bars + 8 * L::kBDsFull, 256);
     mbar_init(bars + 8 * L::kBDqFull, 1);
-    mbar_init(bars + 8 * L::kBSFree, 128);
+    mbar_init(bars + 8 * L::kBSFree, 256);
     mbar_init(bars + 8 * L::kBDone, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(sbase + L::kTmemSlotOff, 512);
     tmem_relinquish();
   }
@@ -462,9 +483,9 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlotOff);
 
-  if (warp < 4) {
+  if (warp < 8) {
     bwd_elementwise<D>(p, sbase, smem, tmem, abort_flag);
-  } else if (warp == 4) {
+  } else if (warp == 8) {
     if (lane == 0) bwd_producer<D>(&tm_q, &tm_k, &tm_v, &tm_do, p, sbase, abort_flag);
   } else {
     if (lane == 0) bwd_mma<D>(p, sbase, tmem, abort_flag);
@@ -472,7 +493,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
