@@ -47,6 +47,8 @@ PREFILL_SOURCES = ["io_aware_exact_flashattention_b200/csrc/prefill_sm100.cuh",
                    "io_aware_exact_flashattention_b200/csrc/sm100.cuh"]
 DECODE_SOURCES = ["io_aware_exact_flashattention_b200/csrc/decode_sm100.cuh",
                   "io_aware_exact_flashattention_b200/csrc/sm100.cuh"]
+BACKWARD_SOURCES = ["io_aware_exact_flashattention_b200/csrc/backward_sm100.cuh",
+                    "io_aware_exact_flashattention_b200/csrc/sm100.cuh"]
 
 
 def parse_args():
@@ -417,6 +419,8 @@ def run_ours(args, world, rank, local):
                     "frac_of_nominal_2250": bw_tf / NOMINAL_BF16_TFLOPS,
                     "algorithmic": "%.4g FLOP per call (2.5 x the forward's: five products)" % bw_flops,
                     "kernels": "fa_bwd_dsum_kernel + fa_bwd_kernel<128> + fa_bwd_dq_kernel (and a memset)",
+                    "traffic_main_kernel": profiled_traffic("backward_causal_mha_s2048_d128.md",
+                                                            BACKWARD_SOURCES),
                     "gpu_launches": 3 * K,
                     "note": "dq, dk, dv from the forward's O and LSE; measured outside the step"}
         del dq, dk, dv, ws, d_o
