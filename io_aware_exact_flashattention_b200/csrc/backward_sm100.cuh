@@ -10,7 +10,7 @@
 // shared memory and dK_j, dV_j accumulate in tensor memory while the query
 // tiles of every query head of the group stream past (key-stationary loop, so
 // dK and dV are written once; dQ rows collect contributions from every key
-// tile and are added into an fp32 workspace with vector reductions).  Per
+// tile and are added into an fp32 workspace by bulk tensor reductions).  Per
 // query tile, all on tcgen05 with fp32 accumulators in TMEM:
 //   S^T  = K_j Q_i^T      (M=128 keys, N=128 queries; SS)
 //   dP^T = V_j dO_i^T     (M=128 keys, N=128 queries; SS)
@@ -96,10 +96,27 @@ __device__ __forceinline__ void bwd_cta(const BwdParams& p, int& b, int& g, int&
   g = bg % p.Hkv;
 }
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
+// Element-wise add of a shared-memory box into global memory (bulk reduction
+// in L2), tracked by the issuing thread's bulk-async group.
+__device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, uint32_t src, int c0, int c1,
+                                                  int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
+      " [%0, {%2, %3, %4}], [%1];"
+      ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(src), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until every committed bulk operation of this thread has completed.
+__device__ __forceinline__ void bulk_wait_group0() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Wait until every committed bulk operation of this thread has finished
+// reading its shared-memory source.
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -279,8 +296,9 @@ done:
 // = query row t) and for dK, dV; the two halves run side by side.
 // ---------------------------------------------------------------------------
 template <int D>
-__device__ __forceinline__ void bwd_elementwise(const BwdParams& p, uint32_t sbase, uint8_t* smem,
-                                                uint32_t tmem, volatile int* abort_flag) {
+__device__ __forceinline__ void bwd_elementwise(const BwdParams& p, const CUtensorMap* tm_dq,
+                                                uint32_t sbase, uint8_t* smem, uint32_t tmem,
+                                                volatile int* abort_flag) {
   using L = BwdLayout<D>;
   const uint32_t bars = sbase + L::kBarOff;
   const int t = threadIdx.x & 127;
@@ -384,30 +402,44 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, uint32_t sba
       tc_fence_before();
       mbar_arrive(bars + 8 * L::kBDsFull);
 
-      // dQ partial (thread = query row q0 + t, this warpgroup's d-columns)
+      // dQ partial (thread = query row q0 + t, this warpgroup's d-columns),
+      // scaled, staged 32 columns at a time in this warpgroup's half of the
+      // dS buffer (free: the dQ MMA that read dS is complete) and added into
+      // the fp32 workspace by one bulk tensor reduction per 128 x 32 box.
       ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * L::kBDqFull, ph, abort_flag, p.wait_limit_ns));
       if (!ok) continue;
       tc_fence_after();
       {
-        const int q = q0 + t;
-        float* dst = p.dq_acc + (row_base + q) * D + hf * kDH;
+        uint8_t* stage = ds_smem + hf * L::kBoxBytes;  // 128 rows x 128 B, 128B swizzle
+        const uint32_t stage_s = sbase + L::kDsOff + hf * L::kBoxBytes;
 #pragma unroll
         for (int c4 = 0; c4 < kDH / 32; ++c4) {
           uint32_t r[32];
           tmem_ld32(t_dp + hf * kDH + c4 * 32, r);
-          if (q < p.Sq) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              red_add_v4(dst + c4 * 32 + e, __uint_as_float(r[e]) * p.scale,
-                         __uint_as_float(r[e + 1]) * p.scale, __uint_as_float(r[e + 2]) * p.scale,
-                         __uint_as_float(r[e + 3]) * p.scale);
+          for (int k4 = 0; k4 < 8; ++k4) {
+            float4 v4 = make_float4(__uint_as_float(r[4 * k4]) * p.scale,
+                                    __uint_as_float(r[4 * k4 + 1]) * p.scale,
+                                    __uint_as_float(r[4 * k4 + 2]) * p.scale,
+                                    __uint_as_float(r[4 * k4 + 3]) * p.scale);
+            *reinterpret_cast<float4*>(stage + t * 128 + ((k4 ^ (t & 7)) * 16)) = v4;
           }
+          fence_proxy_async_smem();
+          named_barrier(1 + hf, 128);
+          if (t == 0) {
+            tma_reduce_add_3d(tm_dq, stage_s, hf * kDH + c4 * 32, q0, static_cast<int>(
+                static_cast<size_t>(b) * p.Hq + h));
+            bulk_commit_group();
+            bulk_wait_group_read0();  // the box has been read: the buffer is free again
+          }
+          named_barrier(1 + hf, 128);
         }
       }
       tc_fence_before();
       mbar_arrive(bars + 8 * L::kBSFree);
     }
   }
+  if (t == 0) bulk_wait_group0();  // this thread's reductions have landed
   if (!ok) return;
 
   // dK = scale * (dS^T Q summed), dV = P^T dO summed: thread t = key row,
@@ -448,7 +480,7 @@ template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-              const BwdParams p) {
+              const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using L = BwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
@@ -484,7 +516,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlotOff);
 
   if (warp < 8) {
-    bwd_elementwise<D>(p, sbase, smem, tmem, abort_flag);
+    bwd_elementwise<D>(p, &tm_dq, sbase, smem, tmem, abort_flag);
   } else if (warp == 8) {
     if (lane == 0) bwd_producer<D>(&tm_q, &tm_k, &tm_v, &tm_do, p, sbase, abort_flag);
   } else {

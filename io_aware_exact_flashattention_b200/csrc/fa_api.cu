@@ -55,6 +55,21 @@ bool encode_bhsd(CUtensorMap* map, const void* base, int d, int rows, long long 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [planes, rows, d] fp32 rows (the backward's dq accumulator) as a 3-D map with
+// 32 x 128 x 1 boxes, 128B swizzle: the target of bulk tensor reductions.
+bool encode_f32_rows(CUtensorMap* map, void* base, int d, int rows, long long planes) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t r = static_cast<cuuint64_t>(rows > 0 ? rows : 1);
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), r, static_cast<cuuint64_t>(planes)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4, r * static_cast<cuuint64_t>(d) * 4};
+  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // One-time per-device opt-in to the prefill kernels' dynamic shared memory,
 // and the device's SM count (the persistent grid size).
 std::once_flag g_attr_once[kMaxDevices];
@@ -342,9 +357,10 @@ fa_status launch_backward(const void* q, const void* k, const void* v, const voi
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o), dsum, q_rows);
   const int n_kv_tiles = (Skv + fa::kBwdBM - 1) / fa::kBwdBM;
   if (n_kv_tiles > 0) {
-    CUtensorMap tq, tk, tv, tdo;
+    CUtensorMap tq, tk, tv, tdo, tdq;
     if (!encode_bhsd(&tq, q, D, Sq, static_cast<long long>(B) * Hq) ||
         !encode_bhsd(&tdo, d_o, D, Sq, static_cast<long long>(B) * Hq) ||
+        !encode_f32_rows(&tdq, dq_acc, D, Sq, static_cast<long long>(B) * Hq) ||
         !encode_bhsd(&tk, k, D, Skv, static_cast<long long>(B) * Hkv) ||
         !encode_bhsd(&tv, v, D, Skv, static_cast<long long>(B) * Hkv))
       return FA_ERR_CUDA;
@@ -371,7 +387,7 @@ fa_status launch_backward(const void* q, const void* k, const void* v, const voi
     p.wait_limit_ns = kWaitLimitNs;
     const unsigned grid = static_cast<unsigned>(static_cast<long long>(B) * Hkv * n_kv_tiles);
     fa::fa_bwd_kernel<D><<<grid, fa::kBwdThreads, fa::BwdLayout<D>::kBytes, stream>>>(tq, tk, tv,
-                                                                                      tdo, p);
+                                                                                      tdo, tdq, p);
   }
   const long long n = q_rows * D;
   fa::fa_bwd_dq_kernel<<<static_cast<unsigned>((n / 4 + 255) / 256), 256, 0, stream>>>(
