@@ -418,7 +418,7 @@ def run_ours(args, world, rank, local):
                     "ms_per_call": bw_ms / K, "frac_of_measured_burst": bw_tf / float(peaks["bf16_tflops"]),
                     "frac_of_nominal_2250": bw_tf / NOMINAL_BF16_TFLOPS,
                     "algorithmic": "%.4g FLOP per call (2.5 x the forward's: five products)" % bw_flops,
-                    "kernels": "fa_bwd_dsum_kernel + fa_bwd_kernel<128> + fa_bwd_dq_kernel (and a memset)",
+                    "kernels": "fa_bwd_dsum_kernel (also zeroes the dq workspace) + fa_bwd_kernel<128> + fa_bwd_dq_kernel",
                     "traffic_main_kernel": profiled_traffic("backward_causal_mha_s2048_d128.md",
                                                             BACKWARD_SOURCES),
                     "gpu_launches": 3 * K,

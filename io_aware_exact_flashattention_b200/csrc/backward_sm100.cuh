@@ -120,15 +120,21 @@ __device__ __forceinline__ void bulk_wait_group_read0() {
 }
 
 // ---------------------------------------------------------------------------
-// D = rowsum(dO * O) for every query row (one warp per row).
+// D = rowsum(dO * O) for every query row (one warp per row); the row's fp32
+// dq accumulator is zeroed on the way.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_dsum_kernel(const __nv_bfloat16* __restrict__ o,
                                                           const __nv_bfloat16* __restrict__ d_o,
-                                                          float* __restrict__ dsum, long long rows) {
+                                                          float* __restrict__ dsum,
+                                                          float* __restrict__ dq_acc,
+                                                          long long rows) {
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
+#pragma unroll
+  for (int c = lane * 4; c < D; c += 128)
+    *reinterpret_cast<float4*>(dq_acc + row * D + c) = make_float4(0.f, 0.f, 0.f, 0.f);
   float acc = 0.f;
 #pragma unroll
   for (int c = lane * 2; c < D; c += 64) {

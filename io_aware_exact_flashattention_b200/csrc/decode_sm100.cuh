@@ -49,7 +49,7 @@ constexpr float kDecRescaleThreshold = 8.0f;  // log2 units
 
 template <int D>
 struct DecodeLayout {
-  static constexpr int kStages = (D == 128) ? 5 : 8;  // ring of K or V tiles
+  static constexpr int kStages = (D == 128) ? 6 : 8;  // ring of K or V tiles
   static constexpr int kTileBytes = kDecBN * D * 2;
   static constexpr int kBoxBytes = kDecBN * 128;       // one 64-wide column block of a tile
   static constexpr int kRingOff = 0;

@@ -350,11 +350,9 @@ fa_status launch_backward(const void* q, const void* k, const void* v, const voi
   const long long q_rows = static_cast<long long>(B) * Hq * Sq;
   float* dq_acc = workspace;
   float* dsum = workspace + q_rows * D;
-  if (cudaMemsetAsync(dq_acc, 0, static_cast<size_t>(q_rows) * D * sizeof(float), stream) !=
-      cudaSuccess)
-    return FA_ERR_CUDA;
   fa::fa_bwd_dsum_kernel<D><<<static_cast<unsigned>((q_rows + 7) / 8), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o), dsum, q_rows);
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o), dsum, dq_acc,
+      q_rows);
   const int n_kv_tiles = (Skv + fa::kBwdBM - 1) / fa::kBwdBM;
   if (n_kv_tiles > 0) {
     CUtensorMap tq, tk, tv, tdo, tdq;
