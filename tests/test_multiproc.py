@@ -40,7 +40,7 @@ def _worker(rank, world, port, out):
 
 def test_two_gloo_ranks_reduce_and_seed():
     world, port = 2, _free_port()
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()  # no fork of a threaded process
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
     for rank in range(world):
         got, same_inputs = out[rank]
