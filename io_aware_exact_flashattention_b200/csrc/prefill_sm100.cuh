@@ -63,7 +63,11 @@ constexpr float kExp2C0 = 9.999280572e-01f;
 constexpr float kExp2C1 = 6.932609677e-01f;
 constexpr float kExp2C2 = 2.426111251e-01f;
 constexpr float kExp2C3 = 5.517166853e-02f;
-constexpr int kPolyPairsPer8 = 3;  // of every 8 pairs of scores, this many use the polynomial
+// Of every 8 pairs of scores, this many use the polynomial.  Off: on B200,
+// with the other choices in this kernel, every share tried (1 to 4 of 8)
+// took more cycles than the MUFU alone (2-7 %); the polynomial stays as a
+// tested option (fa_debug_exp2_poly checks it against the MUFU).
+constexpr int kPolyPairsPer8 = 0;
 
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer
