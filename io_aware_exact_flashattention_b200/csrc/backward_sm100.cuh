@@ -324,24 +324,37 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, const CUtens
   const int off = p.Skv - p.Sq;
   const int i0 = bwd_first_q_tile(p, j);
   uint32_t n = 0;
+  // LSE (in log2 units) and D of this thread's query for a tile: loaded one
+  // tile ahead, so the load latency hides behind the previous tile's work.
+  auto load_ld = [&](int hh_, int i_, float& lse_v, float& d_v) {
+    const int c = hf * kQH + t;
+    const int q = i_ * kBwdBN + c;
+    const size_t rb = (static_cast<size_t>(b) * p.Hq + g * p.group + hh_) * p.Sq;
+    lse_v = (t < kQH && q < p.Sq) ? p.lse[rb + q] * 1.4426950408889634f : INFINITY;
+    d_v = (t < kQH && q < p.Sq) ? p.dsum[rb + q] : 0.f;
+  };
+  float lse_next = INFINITY, d_next = 0.f;
+  if (i0 < p.n_q_tiles) load_ld(0, i0, lse_next, d_next);
   // After a failed wait a warp skips the remaining work but still takes every
   // named barrier, so the other warps of its warpgroup can never block there.
   bool ok = true;
   for (int hh = 0; hh < p.group; ++hh) {
     const int h = g * p.group + hh;
-    const size_t row_base = (static_cast<size_t>(b) * p.Hq + h) * p.Sq;
     for (int i = i0; i < p.n_q_tiles; ++i, ++n) {
       const uint32_t ph = n & 1u;
       const int q0 = i * kBwdBN;
-      // LSE (in log2 units) and D of this warpgroup's 64 queries
+      // this warpgroup's 64 queries: LSE and D into shared memory
       named_barrier(1 + hf, 128);
       if (t < kQH) {
-        const int c = hf * kQH + t;
-        const int q = q0 + c;
-        lse_s[c] = (q < p.Sq) ? p.lse[row_base + q] * 1.4426950408889634f : INFINITY;
-        d_s[c] = (q < p.Sq) ? p.dsum[row_base + q] : 0.f;
+        lse_s[hf * kQH + t] = lse_next;
+        d_s[hf * kQH + t] = d_next;
       }
       named_barrier(1 + hf, 128);
+      {  // next tile's values (same head, or the next head's first tile)
+        const bool more_i = (i + 1 < p.n_q_tiles);
+        if (more_i) load_ld(hh, i + 1, lse_next, d_next);
+        else if (hh + 1 < p.group) load_ld(hh + 1, i0, lse_next, d_next);
+      }
 
       if (!ok) continue;
       // P^T for this key and the warpgroup's queries: p = 2^(s*scale*log2e - LSE*log2e)
