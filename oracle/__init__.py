@@ -15,7 +15,9 @@ arithmetic) and then decoded like a contiguous one.
 
 Parity pins (tests/test_oracle_pins.py): closed-form golden cases, an
 independent online-softmax recurrence, invariants, torch fp64 SDPA on small
-shapes, GQA/decode/split reductions.  Every function here is pinned.
+shapes, GQA/decode/split reductions, the E4M3 decoding by hand and against
+torch's float8 conversion, and the per-head dequantisation in closed form.
+Every function here is pinned.
 """
 from __future__ import annotations
 
@@ -34,6 +36,7 @@ _lib: Optional[ctypes.CDLL] = None
 _D = ctypes.POINTER(ctypes.c_double)
 _I32 = ctypes.POINTER(ctypes.c_int32)
 _I64 = ctypes.POINTER(ctypes.c_int64)
+_U8 = ctypes.POINTER(ctypes.c_uint8)
 
 
 def build(src: str = _SRC, out: str = _LIB_PATH, force: bool = False) -> str:
@@ -78,6 +81,10 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_attn_bwd.restype = ci
     lib.oracle_combine.argtypes = [_D, _D, _D, _D] + [ci] * 4
     lib.oracle_combine.restype = ci
+    lib.oracle_e4m3_decode.argtypes = [_U8, ctypes.c_int64, _D]
+    lib.oracle_e4m3_decode.restype = ci
+    lib.oracle_dequant_heads.argtypes = [_U8, _D, _D] + [ci] * 5
+    lib.oracle_dequant_heads.restype = ci
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ci
     return lib
@@ -248,6 +255,59 @@ def combine(o_part, lse_part, lib: Optional[ctypes.CDLL] = None):
     if rc != 0:
         raise ValueError("oracle_combine rejected its arguments")
     return o, lse
+
+
+def _codes(a) -> np.ndarray:
+    """E4M3 codes as a contiguous uint8 array (torch float8 tensors are viewed
+    as bytes, never converted)."""
+    if hasattr(a, "detach"):
+        import torch
+        a = a.detach().to("cpu").contiguous()
+        if a.element_size() != 1:
+            raise TypeError("expected one byte per element")
+        a = a.view(torch.uint8).numpy()
+    a = np.asarray(a)
+    if a.dtype != np.uint8:
+        raise TypeError("expected uint8 codes")
+    return np.ascontiguousarray(a)
+
+
+def e4m3_decode(codes, lib: Optional[ctypes.CDLL] = None) -> np.ndarray:
+    """float64 values of E4M3 codes (any shape)."""
+    lib = lib or load()
+    c = _codes(codes)
+    out = np.zeros(c.shape)
+    if lib.oracle_e4m3_decode(_p(c, _U8), c.size, _p(out)) != 0:
+        raise ValueError("oracle_e4m3_decode rejected its arguments")
+    return out
+
+
+def dequant_heads(x8, descale, Hkv: int, lib: Optional[ctypes.CDLL] = None) -> np.ndarray:
+    """Real values [B,H,S,d] of E4M3 codes x8 [B,H,S,d]: head h of batch b is
+    scaled by descale[b, h // (H // Hkv)]; descale None means 1."""
+    lib = lib or load()
+    c = _codes(x8)
+    B, H, S, d = c.shape
+    out = np.zeros(c.shape)
+    ds = None if descale is None else _f64(descale).reshape(-1)
+    if ds is not None and ds.size != B * Hkv:
+        raise ValueError("descale must hold B * Hkv factors")
+    rc = lib.oracle_dequant_heads(_p(c, _U8), None if ds is None else _p(ds), _p(out), B, H,
+                                  Hkv, S, d)
+    if rc != 0:
+        raise ValueError("oracle_dequant_heads rejected its arguments")
+    return out
+
+
+def attn_fwd_fp8(q8, k8, v8, descale_q, descale_k, descale_v, causal: bool, scale: float,
+                 lib: Optional[ctypes.CDLL] = None):
+    """O and LSE (float64) of the attention of the dequantised E4M3 inputs."""
+    lib = lib or load()
+    Hkv = int(k8.shape[1])
+    q = dequant_heads(q8, descale_q, Hkv, lib)
+    k = dequant_heads(k8, descale_k, Hkv, lib)
+    v = dequant_heads(v8, descale_v, Hkv, lib)
+    return attn_fwd(q, k, v, causal, scale, lib=lib)
 
 
 def num_threads(lib: Optional[ctypes.CDLL] = None) -> int:

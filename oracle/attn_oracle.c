@@ -397,6 +397,60 @@ int oracle_attn_bwd(const double *q, const double *k, const double *v, const dou
     return err ? -1 : 0;
 }
 
+/* --- 8-bit floating-point inputs ------------------------------------------
+ * "FlashAttention & IO-aware attention", section "Deep dive", names
+ * FlashAttention-3's FP8 variant and says nothing more.  The reading used
+ * here: Q, K and V arrive as E4M3 codes (the OCP 8-bit format with 4 exponent
+ * bits, bias 7, 3 mantissa bits, no infinities, NaN = S.1111.111) with one
+ * fp32 dequantisation factor per (batch, key/value head) for each of Q, K and
+ * V; the real input is factor * value(code).  The attention of those real
+ * inputs is then the one-shot definition above, unchanged. */
+
+/* Value of one E4M3 code, written out from the format's definition. */
+static double e4m3_value(uint8_t c)
+{
+    const int sign = (c >> 7) & 1;
+    const int e = (c >> 3) & 15;
+    const int m = c & 7;
+    double mag;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        mag = ldexp((double)m / 8.0, -6);          /* subnormal: 0.m * 2^(1-7) */
+    else
+        mag = ldexp(1.0 + (double)m / 8.0, e - 7); /* normal: 1.m * 2^(e-7) */
+    return sign ? -mag : mag;
+}
+
+int oracle_e4m3_decode(const uint8_t *codes, int64_t n, double *out)
+{
+    if (n < 0 || (n > 0 && (codes == NULL || out == NULL)))
+        return -1;
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = e4m3_value(codes[i]);
+    return 0;
+}
+
+/* x8 [B,H,S,d] E4M3 codes -> out [B,H,S,d] real values: head h of batch b is
+ * scaled by descale[b * Hkv + h / (H / Hkv)] (H = Hq for queries, H = Hkv for
+ * keys and values, where the map is the identity).  descale == NULL means 1. */
+int oracle_dequant_heads(const uint8_t *x8, const double *descale, double *out, int B, int H,
+                         int Hkv, int S, int d)
+{
+    if (B < 0 || H < 1 || Hkv < 1 || S < 0 || d < 1 || H % Hkv != 0)
+        return -1;
+    const int group = H / Hkv;
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t h = 0; h < H; ++h) {
+            const int64_t g = h / group;
+            const double f = descale ? descale[b * Hkv + g] : 1.0;
+            const int64_t base = ((b * H + h) * (int64_t)S) * d;
+            for (int64_t i = 0; i < (int64_t)S * d; ++i)
+                out[base + i] = f * e4m3_value(x8[base + i]);
+        }
+    return 0;
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -12,7 +12,9 @@ oracle disagrees with:
   * invariants of softmax attention;
   * torch's fp64 scaled_dot_product_attention (an independent implementation);
   * reductions: GQA == MHA with repeated K/V, decode == prefill with one query,
-    split + combine == unsplit.
+    split + combine == unsplit;
+  * for E4M3 inputs: code values derived by hand (tests/golden/e4m3_codes.json),
+    torch's float8_e4m3fn decoding, and a one-key closed form per head.
 """
 from __future__ import annotations
 
@@ -495,6 +497,72 @@ def pin_bwd_single_key(lib):
     _close(dv[0, 0, 0], d_o.sum(axis=(0, 1, 2)), 1e-13, "dv single key")
 
 
+# --------------------------------------------------------------------------
+# E4M3 inputs
+E4M3_GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "e4m3_codes.json")
+
+
+def _torch_e4m3(codes):
+    """torch's own float8_e4m3fn decoding (an independent implementation)."""
+    c = torch.as_tensor(np.asarray(codes, dtype=np.uint8))
+    return c.view(torch.float8_e4m3fn).double().numpy()
+
+
+def pin_e4m3_golden(lib):
+    """Single codes whose values were derived by hand from the E4M3 definition."""
+    table = json.load(open(E4M3_GOLDEN))["codes"]
+    codes = np.array([c for c, _ in table], dtype=np.uint8)
+    got = oracle.e4m3_decode(codes, lib=lib)
+    for (c, want), g in zip(table, got):
+        if want is None:
+            assert np.isnan(g), f"code {c}: {g} is not NaN"
+        else:
+            assert g == want and math.copysign(1.0, g) == math.copysign(1.0, want), \
+                f"code {c}: {g} != {want}"
+
+
+def pin_e4m3_matches_torch(lib):
+    """All 256 codes agree with torch's float8_e4m3fn conversion (NaN with NaN)."""
+    codes = np.arange(256, dtype=np.uint8)
+    got = oracle.e4m3_decode(codes, lib=lib)
+    want = _torch_e4m3(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(want)), "NaN codes differ"
+    ok = ~np.isnan(want)
+    assert np.array_equal(got[ok], want[ok]), "E4M3 values differ from torch"
+
+
+def pin_e4m3_order_and_sign(lib):
+    """Codes 0..126 are strictly increasing and setting bit 7 negates."""
+    pos = oracle.e4m3_decode(np.arange(127, dtype=np.uint8), lib=lib)
+    neg = oracle.e4m3_decode(np.arange(128, 255, dtype=np.uint8), lib=lib)
+    assert np.all(np.diff(pos) > 0), "E4M3 codes not monotone"
+    assert np.array_equal(neg, -pos), "sign bit does not negate"
+
+
+def pin_fp8_one_key_closed_form(lib):
+    """One key per head: O = dv * v_0 and LSE = scale * dq * dk * (q . k_0), with
+    the factors of the query's key/value head (GQA group) in its own batch."""
+    rng = np.random.default_rng(31)
+    B, Hq, Hkv, Sq, d = 2, 4, 2, 3, 5
+
+    def codes(shape):  # finite codes of either sign
+        c = rng.integers(0, 127, size=shape).astype(np.uint8)
+        return np.where(rng.random(shape) < 0.5, c | 0x80, c).astype(np.uint8)
+
+    q8, k8, v8 = codes((B, Hq, Sq, d)), codes((B, Hkv, 1, d)), codes((B, Hkv, 1, d))
+    dq, dk, dv = (rng.uniform(0.25, 4.0, size=(B, Hkv)) for _ in range(3))
+    scale = 0.3
+    o, lse = oracle.attn_fwd_fp8(q8, k8, v8, dq, dk, dv, False, scale, lib=lib)
+    qv, kv, vv = _torch_e4m3(q8), _torch_e4m3(k8), _torch_e4m3(v8)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // (Hq // Hkv)
+            for i in range(Sq):
+                want_l = scale * dq[b, g] * dk[b, g] * float(qv[b, h, i] @ kv[b, g, 0])
+                _close(lse[b, h, i], want_l, 1e-12 * max(1.0, abs(want_l)), "fp8 one-key LSE")
+                _close(o[b, h, i], dv[b, g] * vv[b, g, 0], 1e-12, "fp8 one-key O")
+
+
 ALL_PINS = [
     pin_golden_prefill,
     pin_golden_combine,
@@ -512,4 +580,8 @@ ALL_PINS = [
     pin_bwd_finite_differences,
     pin_bwd_torch_autograd,
     pin_bwd_single_key,
+    pin_e4m3_golden,
+    pin_e4m3_matches_torch,
+    pin_e4m3_order_and_sign,
+    pin_fp8_one_key_closed_form,
 ]

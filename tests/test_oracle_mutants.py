@@ -39,6 +39,16 @@ MUTANTS = [
     ("bwd_dk_missing_scale", "dkh[j * d + t] += scale * ds * qi[t];", "dkh[j * d + t] += ds * qi[t];"),
     ("bwd_dv_uses_dp", "dvh[j * d + t] += p[j] * doi[t];", "dvh[j * d + t] += dp[j] * doi[t];"),
     ("bwd_dq_uses_query", "dqi[t] += scale * ds * kh[j * d + t];", "dqi[t] += scale * ds * qi[t];"),
+    ("e4m3_bias_8", "mag = ldexp(1.0 + (double)m / 8.0, e - 7);",
+     "mag = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    ("e4m3_subnormal_implicit_one", "mag = ldexp((double)m / 8.0, -6);",
+     "mag = ldexp(1.0 + (double)m / 8.0, -6);"),
+    ("e4m3_nan_code_missed", "if (e == 15 && m == 7)\n        return NAN;",
+     "if (e == 16 && m == 7)\n        return NAN;"),
+    ("e4m3_sign_dropped", "return sign ? -mag : mag;", "return mag;"),
+    ("dequant_query_head_modulo", "const int64_t g = h / group;\n            const double f",
+     "const int64_t g = h % Hkv;\n            const double f"),
+    ("dequant_batch_ignored", "descale[b * Hkv + g]", "descale[g]"),
 ]
 
 
