@@ -71,6 +71,8 @@ def parse_args():
                     help="skip the paged-cache decode measurement")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the backward measurement on the prefill workload")
+    ap.add_argument("--no-fp8", action="store_true",
+                    help="skip the E4M3-input forward on the prefill workload")
     ap.add_argument("--page-size", type=int, default=16,
                     help="page size of the paged-cache decode measurement")
     return ap.parse_args()
@@ -425,6 +427,44 @@ def run_ours(args, world, rank, local):
                     "note": "dq, dk, dv from the forward's O and LSE; measured outside the step"}
         del dq, dk, dv, ws, d_o
 
+    # The prefill workload with E4M3 inputs (per-(batch, kv-head) factors),
+    # measured on its own after the step.
+    prefill_fp8 = None
+    if do_pre and not args.no_fp8 and c.d == 128:
+        from io_aware_exact_flashattention_b200.inputs import fp8_prefill_inputs
+        q8, k8, v8, dq8, dk8, dv8 = fp8_prefill_inputs(c.B, c.Hq, c.Hkv, c.Sq, c.Skv, c.d,
+                                                      rank_seed(c.seed, rank), c.q_mult,
+                                                      device=dev)
+        for _ in range(max(args.warmup, 1)):
+            fa.fa_fwd_fp8(q8, k8, v8, dq8, dk8, dv8, o, lse, c.causal, c.scale, stream=stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        fevs = []
+        for _ in range(K):
+            flush.fill_(1.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fa.fa_fwd_fp8(q8, k8, v8, dq8, dk8, dv8, o, lse, c.causal, c.scale, stream=stream)
+            b.record(stream)
+            fevs.append((a, b))
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        f8_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in fevs)], world)[0]
+        f8_tf = flops / (f8_ms * 1e-3 / K) / 1e12
+        f8_peak = 2.0 * float(peaks["bf16_tflops"])  # E4M3 dense rate = 2 x bf16 (4.5 / 2.25)
+        prefill_fp8 = {
+            "value": aggregate_rate(world, flops, K, f8_ms) / 1e12, "unit": "TFLOP/s",
+            "ms_per_call": f8_ms / K, "dtype": "e4m3 (fp32 accumulate)",
+            "roofline": {"bound": "tensor", "achieved": f8_tf, "peak": f8_peak,
+                         "unit": "TFLOP/s", "frac": f8_tf / f8_peak,
+                         "peak_source": "2 x measured bf16 burst (nominal e4m3:bf16 ratio 4.5:2.25)",
+                         "traffic": profiled_traffic("prefill_fp8_causal_mha_s2048_d128.md",
+                                                     PREFILL_SOURCES)},
+            "frac_of_nominal_4500": f8_tf / (2.0 * NOMINAL_BF16_TFLOPS),
+            "kernels": "fa_prefill_kernel<128, true>", "gpu_launches": K,
+            "note": "same shape and FLOP count as the bf16 prefill; measured outside the step"}
+        del q8, k8, v8, dq8, dk8, dv8
+
     # Paged cache: the same decode workload stored in page_size-key pages
     # scattered over a pool, read through a block table.  Measured on its own,
     # outside the step.
@@ -535,6 +575,8 @@ def run_ours(args, world, rank, local):
         line["decode_paged"] = paged
     if backward is not None:
         line["backward"] = backward
+    if prefill_fp8 is not None:
+        line["prefill_fp8"] = prefill_fp8
     if cpu is not None:
         line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)

@@ -65,7 +65,10 @@ typedef enum {
  *   causal != 0: key j is visible to query i iff j <= i + (Skv - Sq)
  *       (bottom-right alignment).  A query row that sees no key gets
  *       O = 0 and LSE = -inf.
- *   scale: multiplies q.k before the softmax (normally 1/sqrt(d)).
+ *   scale: multiplies q.k before the softmax (normally 1/sqrt(d)); must be
+ *       >= 0 (the kernel follows the largest raw score q.k, which is the
+ *       softmax's largest only for a non-negative scale), else
+ *       FA_ERR_UNSUPPORTED.
  *
  * Supported: d in {64, 128}; Hq % Hkv == 0; B, Hq, Hkv >= 1; Sq, Skv >= 0
  * (Sq == 0 or B == 0 is a no-op).  All five pointers 16-byte aligned.
@@ -75,6 +78,40 @@ typedef enum {
 fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
                  int B, int Hq, int Hkv, int Sq, int Skv, int d, int causal,
                  float scale, fa_stream_t stream);
+
+/*
+ * fa_fwd_fp8 -- fa_fwd on 8-bit inputs (the FP8 variant of FlashAttention-3
+ * that "FlashAttention & IO-aware attention", section "Deep dive", names; the
+ * page fixes no format or scaling, so this call defines its own):
+ *
+ *   q, k, v hold E4M3 codes (OCP 8-bit float: 4 exponent bits with bias 7,
+ *   3 mantissa bits, no infinities, NaN = S.1111.111), one byte per element,
+ *   in the layouts of fa_fwd.  descale_q, descale_k, descale_v are device
+ *   arrays of B * Hkv fp32 factors, [b * Hkv + g]; the real input of head h
+ *   of batch b is factor[b, g] * value(code) with g = h / (Hq / Hkv) for the
+ *   queries and g = h for keys and values.  A null factor pointer means 1.
+ *   Factors must be positive and finite (the kernel cannot check device
+ *   memory; a negative Q or K factor gives meaningless results, as a
+ *   negative scale would).
+ *   o and lse are those of fa_fwd on the real inputs (o bf16, lse fp32).
+ *
+ * Arithmetic: both products on the tensor cores in E4M3 with fp32
+ * accumulation; the softmax weights are quantised to E4M3 for P V (as
+ * p * 2^6, p relative to a reference max that lags the row max by at most
+ * 2^2), while the normaliser l and LSE use the unquantised fp32 weights.
+ * Per output element the error against exact attention of the real inputs is
+ * at most 2^-4 * sum_j w_j |v_j| (w = softmax weights; E4M3 keeps 3 mantissa
+ * bits) + n * 2^-16 * max|v| (n visible keys; E4M3 subnormals) + the bf16
+ * rounding of o.  LSE is as accurate as fa_fwd's.
+ *
+ * Supported: d == 128 (other d: FA_ERR_UNSUPPORTED); otherwise as fa_fwd.
+ * q, k, v, o, lse 16-byte aligned; factor arrays 4-byte aligned
+ * (FA_ERR_ALIGNMENT).  Errors as fa_fwd.
+ */
+fa_status fa_fwd_fp8(const void *q, const void *k, const void *v, const float *descale_q,
+                     const float *descale_k, const float *descale_v, void *o, float *lse,
+                     int B, int Hq, int Hkv, int Sq, int Skv, int d, int causal,
+                     float scale, fa_stream_t stream);
 
 /*
  * fa_bwd -- gradients of fa_fwd by recomputation.
@@ -131,7 +168,8 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Sq, int d);
  *   o_partial    [B, Hq, num_splits, d] fp32 (written; caller-owned scratch)
  *   lse_partial  [B, Hq, num_splits]    fp32 (written; caller-owned scratch)
  *
- * Supported: d in {64, 128}; Hq / Hkv in {1, 2, 4, 8}; 1 <= num_splits <= 256.
+ * Supported: d in {64, 128}; Hq / Hkv in {1, 2, 4, 8}; 1 <= num_splits <= 256;
+ * scale >= 0 (as for fa_fwd; a negative scale is FA_ERR_UNSUPPORTED).
  */
 fa_status fa_decode_splitkv(const void *q, const void *k_cache, const void *v_cache,
                             const int32_t *seqlens_k, float *o_partial,

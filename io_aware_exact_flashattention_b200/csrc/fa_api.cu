@@ -55,6 +55,22 @@ bool encode_bhsd(CUtensorMap* map, const void* base, int d, int rows, long long 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [planes, rows, d] E4M3 (one byte per element) tensor as a 3-D map with
+// 128 x 128 x 1 boxes (128-byte rows), 128B swizzle; rows beyond `rows` read
+// as zeros.
+bool encode_bhsd_e4m3(CUtensorMap* map, const void* base, int d, int rows, long long planes) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t r = static_cast<cuuint64_t>(rows > 0 ? rows : 1);
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), r, static_cast<cuuint64_t>(planes)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d), r * static_cast<cuuint64_t>(d)};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // [planes, rows, d] fp32 rows (the backward's dq accumulator) as a 3-D map with
 // 32 x 128 x 1 boxes, 128B swizzle: the target of bulk tensor reductions.
 bool encode_f32_rows(CUtensorMap* map, void* base, int d, int rows, long long planes) {
@@ -80,10 +96,10 @@ int g_prefill_sms[kMaxDevices];
 // that is only safe when every thread was launched with the register count
 // the split was computed for, so a build that compiled to another count is
 // refused instead of launched.
-template <int D>
+template <int D, bool kF8 = false>
 cudaError_t check_prefill_regs() {
   cudaFuncAttributes a;
-  cudaError_t e = cudaFuncGetAttributes(&a, fa::fa_prefill_kernel<D>);
+  cudaError_t e = cudaFuncGetAttributes(&a, fa::fa_prefill_kernel<D, kF8>);
   if (e != cudaSuccess) return e;
   return a.numRegs == fa::kPrefillLaunchRegs ? cudaSuccess : cudaErrorInvalidKernelImage;
 }
@@ -94,6 +110,11 @@ cudaError_t prepare_prefill(int dev) {
     cudaError_t e = cudaDeviceGetAttribute(&g_prefill_sms[dev], cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess) e = check_prefill_regs<64>();
     if (e == cudaSuccess) e = check_prefill_regs<128>();
+    if (e == cudaSuccess) e = check_prefill_regs<128, true>();
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fa::fa_prefill_kernel<128, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::PrefillLayout<128, true>::kBytes);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(fa::fa_prefill_kernel<64>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -107,14 +128,17 @@ cudaError_t prepare_prefill(int dev) {
   return g_attr_err[dev];
 }
 
-template <int D>
+template <int D, bool kF8 = false>
 fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                          int Hq, int Hkv, int Sq, int Skv, int causal, float scale,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, const float* descale_q = nullptr,
+                         const float* descale_k = nullptr, const float* descale_v = nullptr) {
   CUtensorMap tq, tk, tv;
-  if (!encode_bhsd(&tq, q, D, Sq, static_cast<long long>(B) * Hq) ||
-      !encode_bhsd(&tk, k, D, Skv, static_cast<long long>(B) * Hkv) ||
-      !encode_bhsd(&tv, v, D, Skv, static_cast<long long>(B) * Hkv))
+  auto encode = kF8 ? encode_bhsd_e4m3 : encode_bhsd;
+  if (Skv == 0) k = v = q;  // no key tile is ever loaded; any valid address will do
+  if (!encode(&tq, q, D, Sq, static_cast<long long>(B) * Hq) ||
+      !encode(&tk, k, D, Skv, static_cast<long long>(B) * Hkv) ||
+      !encode(&tv, v, D, Skv, static_cast<long long>(B) * Hkv))
     return FA_ERR_CUDA;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
@@ -138,10 +162,13 @@ fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, f
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_limit_ns = kWaitLimitNs;
+  p.descale_q = descale_q;
+  p.descale_k = descale_k;
+  p.descale_v = descale_v;
   const int sms = g_prefill_sms[dev] > 0 ? g_prefill_sms[dev] : 1;
   const int grid = p.n_items < sms ? p.n_items : sms;  // persistent: one CTA per SM
-  fa::fa_prefill_kernel<D><<<static_cast<unsigned>(grid), fa::kPrefillThreads,
-                             fa::PrefillLayout<D>::kBytes, stream>>>(tq, tk, tv, p);
+  fa::fa_prefill_kernel<D, kF8><<<static_cast<unsigned>(grid), fa::kPrefillThreads,
+                                  fa::PrefillLayout<D, kF8>::kBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -440,9 +467,12 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   if (B < 0 || Hq < 1 || Hkv < 1 || Sq < 0 || Skv < 0) return FA_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (scale < 0.f) return FA_ERR_UNSUPPORTED;  // softmax follows the largest raw score
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (B == 0 || Sq == 0) return FA_OK;  // nothing to compute
-  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr)
+  // no keys: k and v may be null (nothing is read from them)
+  if (q == nullptr || o == nullptr || lse == nullptr ||
+      (Skv > 0 && (k == nullptr || v == nullptr)))
     return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return FA_ERR_ALIGNMENT;
@@ -456,6 +486,35 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  : launch_prefill<128>(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, causal, scale, s);
 }
 
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, const float* descale_q,
+                     const float* descale_k, const float* descale_v, void* o, float* lse, int B,
+                     int Hq, int Hkv, int Sq, int Skv, int d, int causal, float scale,
+                     fa_stream_t stream) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || Sq < 0 || Skv < 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (scale < 0.f) return FA_ERR_UNSUPPORTED;  // softmax follows the largest raw score
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || Sq == 0) return FA_OK;  // nothing to compute
+  // no keys: k and v may be null (nothing is read from them)
+  if (q == nullptr || o == nullptr || lse == nullptr ||
+      (Skv > 0 && (k == nullptr || v == nullptr)))
+    return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_ALIGNMENT;
+  auto aligned4 = [](const float* f) { return (reinterpret_cast<uintptr_t>(f) & 3u) == 0; };
+  if (!aligned4(descale_q) || !aligned4(descale_k) || !aligned4(descale_v))
+    return FA_ERR_ALIGNMENT;
+  const long long q_tiles = (static_cast<long long>(Sq) + fa::kBM - 1) / fa::kBM;
+  const long long grid = (q_tiles + 1) / 2 * B * static_cast<long long>(Hq);
+  if (grid > 0x7fffffffLL || static_cast<long long>(B) * Hq > 0x7fffffffLL ||
+      static_cast<long long>(B) * Hkv > 0x7fffffffLL)
+    return FA_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return launch_prefill<128, true>(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, causal, scale, s,
+                                   descale_q, descale_k, descale_v);
+}
+
 fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
                             const int32_t* seqlens_k, float* o_partial, float* lse_partial, int B,
                             int Hq, int Hkv, int Lmax, int d, int num_splits, float scale,
@@ -464,6 +523,7 @@ fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_ca
   if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (num_splits < 1 || num_splits > 256) return FA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (scale < 0.f) return FA_ERR_UNSUPPORTED;  // softmax follows the largest raw score
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   const int G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8) return FA_ERR_UNSUPPORTED;
@@ -501,6 +561,7 @@ fa_status fa_decode_paged_splitkv(const void* q, const void* k_pages, const void
   if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (num_splits < 1 || num_splits > 256) return FA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (scale < 0.f) return FA_ERR_UNSUPPORTED;  // softmax follows the largest raw score
   if (page_size < 16 || page_size > 256 || (page_size & (page_size - 1)) != 0)
     return FA_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;

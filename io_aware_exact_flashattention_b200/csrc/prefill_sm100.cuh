@@ -33,6 +33,21 @@
 // LSE use the same reference max.  p <= 2^24 loses nothing: bf16 P and the
 // fp32 l and O round relative to magnitude and have ~2^100 of headroom.
 // Exponentials are 2^x on scores pre-multiplied by scale*log2(e).
+//
+// 8-bit inputs (kF8; FlashAttention-3's FP8 variant, which "FlashAttention &
+// IO-aware attention", section "Deep dive", names): Q, K and V are E4M3 codes
+// with one fp32 dequantisation factor per (batch, key/value head) each.  Both
+// products run as tcgen05 kind::f8f6f4 MMAs (K = 32 per instruction): S from
+// Q and K in shared memory, O from P in tensor memory (E4M3, four per 32-bit
+// column, 32 columns per tile) and V in shared memory (MN-major).  A d = 128
+// tile of E4M3 is 128-byte rows, the shared-memory geometry of a bf16 d = 64
+// tile, so it takes that layout (16 KB tiles, 8 ring stages).  The factors of
+// Q and K fold into the exponent constant and that of V into the epilogue's
+// 1/l.  P is quantised as p * 2^6 with the reference max allowed to lag the
+// row max by at most 2^2, so every quantised value lies in (0, 256], inside
+// E4M3's range (448), and the row's largest one is >= 64, which keeps the
+// absolute rounding of E4M3 subnormals (<= 2^-10) below 2^-16 of l.  The
+// power of two cancels in O / l; LSE subtracts it.
 #pragma once
 
 #include <climits>
@@ -52,6 +67,8 @@ static_assert(2 * kSoftmaxRegs + kControlRegs <= 3 * kPrefillLaunchRegs,
               "register split exceeds the launch budget");
 constexpr int kSwzBytes = 128 * 128;  // one 128-row x 64-element bf16 box, 128B swizzled
 constexpr float kRescaleThreshold = 24.0f;  // log2 units
+constexpr float kRescaleThresholdF8 = 2.0f;  // log2 units, 8-bit P
+constexpr float kPOffsetF8 = 6.0f;           // 8-bit P is stored as p * 2^6
 
 // 2^x for part of the softmax on the FMA pipe instead of the MUFU: with
 // n = round(x) and f = x - n in [-1/2, 1/2], 2^x = 2^n * p(f) where p is the
@@ -84,6 +101,48 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
+// D[tmem] (+)= A[smem] * B[smem], kind::f8f6f4 (A and B both E4M3 here).
+__device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem], kind::f8f6f4; A is read from tensor memory.
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor, kind::f8f6f4: D fp32 (bits 4-5 = 1), A and B E4M3
+// (format 0 in bits 7-9 and 10-12), B major at bit 16 (1 = MN-major), N >> 3
+// at bits 17-22, M >> 4 at bits 24-28.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool b_mn_major) {
+  return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Four fp32 values -> four E4M3 codes (nearest even, saturating), a in the
+// lowest byte.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r) : "f"(a), "f"(b), "f"(c), "f"(d));
+  return r;
+}
+
 struct PrefillParams {
   __nv_bfloat16* o;
   float* lse;
@@ -96,12 +155,19 @@ struct PrefillParams {
   float scale_log2;
   unsigned long long wait_limit_ns;
   int o_align32;   // o is 32-byte aligned: 32-byte stores in the epilogue
+  // 8-bit inputs only: dequantisation factors [B, Hkv] of Q, K, V (null = 1)
+  const float* descale_q;
+  const float* descale_k;
+  const float* descale_v;
 };
 
-template <int D>
+template <int D, bool kF8 = false>
 struct PrefillLayout {
-  static constexpr int kStages = (D == 128) ? 4 : 8;
-  static constexpr int kTileBytes = kBM * D * 2;
+  static constexpr int kRowBytes = D * (kF8 ? 1 : 2);
+  static constexpr int kBoxes = kRowBytes / 128;  // 128-byte swizzle boxes per row
+  static constexpr int kBoxElems = 128 / (kF8 ? 1 : 2);
+  static constexpr int kTileBytes = kBM * kRowBytes;
+  static constexpr int kStages = (kTileBytes == 32768) ? 4 : 8;
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = 2 * kTileBytes;
   static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
@@ -161,7 +227,7 @@ __device__ __forceinline__ int prefill_item_index(const PrefillParams& p, int r)
 // ---------------------------------------------------------------------------
 // Softmax warpgroup: one thread per query row.
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool kF8>
 __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t tmem,
                                                 uint32_t bar_s, uint32_t bar_p, uint32_t bar_o,
                                                 int w, volatile int* abort_flag) {
@@ -170,7 +236,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
   const uint32_t lane_off = static_cast<uint32_t>(warp_in_wg * 32) << 16;
   const uint32_t tS = tmem + lane_off + static_cast<uint32_t>(w * 128);
   const uint32_t tO = tmem + lane_off + static_cast<uint32_t>(256 + w * D);
-  const float c = p.scale_log2;
+  constexpr float kThreshold = kF8 ? kRescaleThresholdF8 : kRescaleThreshold;
   const int off = p.Skv - p.Sq;
   uint32_t tcount = 0;  // tiles this warpgroup has processed (phase of s_full / p_full)
   uint32_t ocount = 0;  // items this warpgroup has finished with tiles (phase of o_full)
@@ -180,6 +246,15 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
   if (k_item < 0) break;
   const PrefillItem item = prefill_item(p, k_item);
   const int n_tiles = w ? item.n1 : item.n0;
+  // score-to-exponent constant, natural-unit score scale, output factor
+  float c = p.scale_log2, lse_scale = p.scale, o_factor = 1.f;
+  if constexpr (kF8) {
+    const int bg = item.b * p.Hkv + item.g;
+    const float f = (p.descale_q ? p.descale_q[bg] : 1.f) * (p.descale_k ? p.descale_k[bg] : 1.f);
+    c *= f;
+    lse_scale *= f;
+    o_factor = p.descale_v ? p.descale_v[bg] : 1.f;
+  }
   const int q_row0 = (2 * item.pair + w) * kBM;
   const int row = q_row0 + row_in_tile;
   // keys with index > last_key are masked for this row
@@ -243,7 +318,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
                            fmaxf(mx[6], mx[7]));
     const float m_new = fmaxf(m, mt);
     float alpha = 1.f;
-    if ((m_new - m) * c > kRescaleThreshold) {  // false while both are -inf (NaN)
+    if ((m_new - m) * c > kThreshold) {  // false while both are -inf (NaN)
       alpha = ex2((m - m_new) * c);              // 0 when m was -inf
       l *= alpha;
       m = m_new;
@@ -269,13 +344,34 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
     // announced on its own barrier, so P.V on the first 64 keys runs while
     // the second half is computed.
     const float2 c2 = make_float2(c, c);
-    const float2 nmc2 = make_float2(-mc, -mc);
+    const float nmc = kF8 ? kPOffsetF8 - mc : -mc;
+    const float2 nmc2 = make_float2(nmc, nmc);
     float2 rs[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                     make_float2(0.f, 0.f)};
     // Masked tiles take every exponential on the MUFU (2^-inf is exactly 0);
     // the others move kPolyPairsPer8 of every 8 pairs to the FMA pipe.
     auto exps_half = [&](auto poly_tag, int half) {
       constexpr bool kPoly = decltype(poly_tag)::value;
+      if constexpr (kF8) {
+        // four keys per 32-bit column, all exponentials on the MUFU
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int e = half * 64 + 4 * i;
+          const float2 x0 = ffma2(make_float2(s[e], s[e + 1]), c2, nmc2);
+          const float2 x1 = ffma2(make_float2(s[e + 2], s[e + 3]), c2, nmc2);
+          const float2 p0 = make_float2(ex2(x0.x), ex2(x0.y));
+          const float2 p1 = make_float2(ex2(x1.x), ex2(x1.y));
+          rs[(2 * i) & 3] = fadd2(rs[(2 * i) & 3], p0);
+          rs[(2 * i + 1) & 3] = fadd2(rs[(2 * i + 1) & 3], p1);
+          pk[i] = pack_e4m3x4(p0.x, p0.y, p1.x, p1.y);
+        }
+        tmem_st16(tS + half * 16, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar_p + 8 * half);
+        return;
+      }
       uint32_t pk[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -310,7 +406,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
   ++ocount;
   if (!__all_sync(0xffffffffu, ok)) return;
   tc_fence_after();
-  const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+  const float inv_l = (l > 0.f) ? o_factor / l : 0.f;
   {
     uint32_t r[D];
     tmem_ld_row<D>(tO, r);
@@ -335,18 +431,22 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
       }
     }
   }
-  if (row < p.Sq) p.lse[row_index] = (l > 0.f) ? m * p.scale + logf(l) : -INFINITY;
+  if (row < p.Sq) {
+    float lse = m * lse_scale + logf(l);
+    if constexpr (kF8) lse -= kPOffsetF8 * 0.69314718055994531f;  // the 2^6 of P
+    p.lse[row_index] = (l > 0.f) ? lse : -INFINITY;
+  }
   }
 }
 
 // ---------------------------------------------------------------------------
 // TMA producer (one thread).
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool kF8>
 __device__ __forceinline__ void prefill_producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                                                  const CUtensorMap* tm_v, const PrefillParams& p,
                                                  uint32_t sbase, volatile int* abort_flag) {
-  using L = PrefillLayout<D>;
+  using L = PrefillLayout<D, kF8>;
   const uint32_t bars = sbase + L::kBarOff;
   tma_prefetch_desc(tm_q);
   tma_prefetch_desc(tm_k);
@@ -367,9 +467,9 @@ __device__ __forceinline__ void prefill_producer(const CUtensorMap* tm_q, const 
 #pragma unroll
     for (int w = 0; w < 2; ++w)
 #pragma unroll
-      for (int kb = 0; kb < D / 64; ++kb)
-        tma_load_3d(sbase + L::kQOff + w * L::kTileBytes + kb * kSwzBytes, tm_q, bar_q, kb * 64,
-                    (2 * item.pair + w) * kBM, item.b * p.Hq + item.h);
+      for (int kb = 0; kb < L::kBoxes; ++kb)
+        tma_load_3d(sbase + L::kQOff + w * L::kTileBytes + kb * kSwzBytes, tm_q, bar_q,
+                    kb * L::kBoxElems, (2 * item.pair + w) * kBM, item.b * p.Hq + item.h);
     ++nq;
     const int n_max = max(item.n0, item.n1);
     for (int idx = 0; idx < 2 * n_max; ++idx) {
@@ -383,9 +483,9 @@ __device__ __forceinline__ void prefill_producer(const CUtensorMap* tm_q, const 
       mbar_arrive_expect_tx(bar_full, L::kTileBytes);
       const CUtensorMap* tm = (idx & 1) ? tm_v : tm_k;
 #pragma unroll
-      for (int kb = 0; kb < D / 64; ++kb)
+      for (int kb = 0; kb < L::kBoxes; ++kb)
         tma_load_3d(sbase + L::kRingOff + stage * L::kTileBytes + kb * kSwzBytes, tm, bar_full,
-                    kb * 64, (idx >> 1) * kBN, item.b * p.Hkv + item.g);
+                    kb * L::kBoxElems, (idx >> 1) * kBN, item.b * p.Hkv + item.g);
       ++ld;
     }
   }
@@ -400,41 +500,53 @@ __device__ __forceinline__ void prefill_producer(const CUtensorMap* tm_q, const 
 // ---------------------------------------------------------------------------
 // MMA issuer (one thread).
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool kF8>
 __device__ __forceinline__ void prefill_mma(const PrefillParams& p, uint32_t sbase, uint32_t tmem,
                                             volatile int* abort_flag) {
-  using L = PrefillLayout<D>;
+  using L = PrefillLayout<D, kF8>;
   const uint32_t bars = sbase + L::kBarOff;
-  constexpr uint32_t kIdS = idesc_bf16_f32(kBM, kBN, false);
-  constexpr uint32_t kIdPV = idesc_bf16_f32(kBM, D, true);
+  constexpr uint32_t kIdS = kF8 ? idesc_e4m3_f32(kBM, kBN, false) : idesc_bf16_f32(kBM, kBN, false);
+  constexpr uint32_t kIdPV = kF8 ? idesc_e4m3_f32(kBM, D, true) : idesc_bf16_f32(kBM, D, true);
+  constexpr int kKeysPerMma = kF8 ? 32 : 16;  // K of one MMA: 32 bytes of a row
 
   auto kv_stage = [](uint32_t idx) { return static_cast<int>(idx % L::kStages); };
   auto kv_wait = [&](uint32_t idx) -> bool {
     return mbar_wait(bars + 8 * (L::kBarKvFull + kv_stage(idx)),
                      static_cast<uint32_t>(idx / L::kStages) & 1u, abort_flag, p.wait_limit_ns);
   };
-  // S_w = Q_w K^T: M=128 rows, N=128 keys, K=D in steps of 16 (32 bytes).
+  // S_w = Q_w K^T: M=128 rows, N=128 keys, K=D in steps of 32 bytes (16 bf16
+  // or 32 E4M3 elements).
   auto issue_s = [&](int w, int stage) {
     const uint32_t qa = sbase + L::kQOff + w * L::kTileBytes;
     const uint32_t ka = sbase + L::kRingOff + stage * L::kTileBytes;
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
+    for (int kk = 0; kk < L::kRowBytes / 32; ++kk) {
       const uint32_t o = (kk >> 2) * kSwzBytes + (kk & 3) * 32;
-      mma_ss(tmem + w * 128, sw128_desc(qa + o, 16, 1024), sw128_desc(ka + o, 16, 1024), kIdS,
-             kk > 0 ? 1u : 0u);
+      if constexpr (kF8)
+        mma_ss_f8(tmem + w * 128, sw128_desc(qa + o, 16, 1024), sw128_desc(ka + o, 16, 1024),
+                  kIdS, kk > 0 ? 1u : 0u);
+      else
+        mma_ss(tmem + w * 128, sw128_desc(qa + o, 16, 1024), sw128_desc(ka + o, 16, 1024), kIdS,
+               kk > 0 ? 1u : 0u);
     }
   };
-  // O_w += P_w V: A = P_w in TMEM (bf16, 8 columns per 16 keys), B = V tile
-  // (keys x D, D contiguous: MN-major; 64-element column blocks 16 KB apart).
-  // Issued per half of the keys, each after its half of P is announced.
+  // O_w += P_w V: A = P_w in TMEM (8 columns per MMA: 16 bf16 or 32 E4M3
+  // keys), B = V tile (keys x D, D contiguous: MN-major; bf16 d = 128 has two
+  // 64-element column blocks 16 KB apart).  Issued per half of the keys, each
+  // after its half of P is announced.
   auto issue_pv_half = [&](int w, int stage, int half, bool accumulate) {
     const uint32_t va = sbase + L::kRingOff + stage * L::kTileBytes;
+    constexpr int kSteps = (kBN / 2) / kKeysPerMma;
 #pragma unroll
-    for (int k4 = 0; k4 < kBN / 32; ++k4) {
-      const int kk = half * (kBN / 32) + k4;
-      mma_ts(tmem + 256 + w * D, tmem + w * 128 + kk * 8,
-             sw128_desc(va + kk * 16 * 128, kSwzBytes, 1024), kIdPV,
-             (accumulate || kk > 0) ? 1u : 0u);
+    for (int k4 = 0; k4 < kSteps; ++k4) {
+      const int kk = half * kSteps + k4;
+      const uint64_t vd = sw128_desc(va + kk * kKeysPerMma * 128, kSwzBytes, 1024);
+      if constexpr (kF8)
+        mma_ts_f8(tmem + 256 + w * D, tmem + w * 128 + kk * 8, vd, kIdPV,
+                  (accumulate || kk > 0) ? 1u : 0u);
+      else
+        mma_ts(tmem + 256 + w * D, tmem + w * 128 + kk * 8, vd, kIdPV,
+               (accumulate || kk > 0) ? 1u : 0u);
     }
   };
   auto wait_p = [&](int w, int half, uint32_t cnt) -> bool {
@@ -510,11 +622,11 @@ done:
   mbar_wait(bars + 8 * L::kBarDone, 0u, nullptr, p.wait_limit_ns);
 }
 
-template <int D>
+template <int D, bool kF8 = false>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
 fa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
-  using L = PrefillLayout<D>;
+  using L = PrefillLayout<D, kF8>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
@@ -554,15 +666,15 @@ fa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   if (warp < 8) {
     warpgroup_reg_alloc<kSoftmaxRegs>();
     const int w = warp >> 2;
-    prefill_softmax<D>(p, tmem, bars + 8 * (L::kBarSFull + w), bars + 8 * (L::kBarPFull + 2 * w),
+    prefill_softmax<D, kF8>(p, tmem, bars + 8 * (L::kBarSFull + w), bars + 8 * (L::kBarPFull + 2 * w),
                        bars + 8 * (L::kBarOFull + w), w, abort_flag);
   } else {
     warpgroup_reg_dealloc<kControlRegs>();
     if (warp == 8) {
       if (lane == 0)
-        prefill_producer<D>(&tm_q, &tm_k, &tm_v, p, sbase, abort_flag);
+        prefill_producer<D, kF8>(&tm_q, &tm_k, &tm_v, p, sbase, abort_flag);
     } else if (warp == 9) {
-      if (lane == 0) prefill_mma<D>(p, sbase, tmem, abort_flag);
+      if (lane == 0) prefill_mma<D, kF8>(p, sbase, tmem, abort_flag);
     }
   }
 

@@ -32,6 +32,7 @@ _VP, _FP, _I32P = ctypes.c_void_p, ctypes.POINTER(ctypes.c_float), ctypes.c_void
 _I, _F = ctypes.c_int, ctypes.c_float
 SIGNATURES = {
     "fa_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _VP]),
+    "fa_fwd_fp8": (_I, [_VP] * 8 + [_I] * 7 + [_F, _VP]),
     "fa_decode_splitkv": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP]),
     "fa_decode_paged_splitkv": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP] + [_I] * 8 + [_F, _VP]),
     "fa_combine": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP]),
@@ -118,6 +119,62 @@ def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
         raise ValueError("output shapes do not match q")
     _check("fa_fwd", lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Sq,
                                   Skv, d, int(bool(causal)), float(scale), _stream_ptr(stream)))
+
+
+def _need_e4m3(t: torch.Tensor, name: str) -> None:
+    if t.dtype not in (torch.float8_e4m3fn, torch.uint8):
+        raise ValueError("%s must hold E4M3 codes (float8_e4m3fn or uint8), got %s"
+                         % (name, t.dtype))
+    _need(t, t.dtype, name)
+
+
+def fa_fwd_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+               descale_q: Optional[torch.Tensor], descale_k: Optional[torch.Tensor],
+               descale_v: Optional[torch.Tensor], o: torch.Tensor, lse: torch.Tensor,
+               causal: bool, scale: float, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """fa_fwd_fp8 on E4M3 q [B,Hq,Sq,d], k/v [B,Hkv,Skv,d] with fp32
+    dequantisation factors [B,Hkv] (None = 1); o [B,Hq,Sq,d] bf16, lse
+    [B,Hq,Sq] fp32."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need_e4m3(t, n)
+    _need(o, torch.bfloat16, "o")
+    _need(lse, torch.float32, "lse")
+    B, Hq, Sq, d = q.shape
+    _, Hkv, Skv, _ = k.shape
+    if tuple(v.shape) != tuple(k.shape) or k.shape[0] != B or k.shape[3] != d:
+        raise ValueError("k/v shapes %s/%s do not match q %s" % (tuple(k.shape), tuple(v.shape),
+                                                                 tuple(q.shape)))
+    if tuple(o.shape) != tuple(q.shape) or tuple(lse.shape) != (B, Hq, Sq):
+        raise ValueError("output shapes do not match q")
+    for t, n in ((descale_q, "descale_q"), (descale_k, "descale_k"), (descale_v, "descale_v")):
+        if t is not None:
+            _need(t, torch.float32, n)
+            if t.numel() != B * Hkv:
+                raise ValueError("%s must hold B * Hkv factors" % n)
+    _check("fa_fwd_fp8", lib().fa_fwd_fp8(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(descale_q), _ptr(descale_k), _ptr(descale_v), _ptr(o),
+        _ptr(lse), B, Hq, Hkv, Sq, Skv, d, int(bool(causal)), float(scale), _stream_ptr(stream)))
+
+
+def flash_attention_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                        descale_q: Optional[torch.Tensor] = None,
+                        descale_k: Optional[torch.Tensor] = None,
+                        descale_v: Optional[torch.Tensor] = None, causal: bool = False,
+                        scale: Optional[float] = None,
+                        out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None
+                        ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Exact attention of E4M3 inputs (CUDA tensors): returns (o bf16, lse fp32)
+    of softmax(scale * Q K^T [+causal mask]) V on the dequantised values."""
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    B, Hq, Sq, d = q.shape
+    if out is not None:
+        o, lse = out
+    else:
+        o = torch.empty((B, Hq, Sq, d), device=q.device, dtype=torch.bfloat16)
+        lse = torch.empty((B, Hq, Sq), device=q.device, dtype=torch.float32)
+    fa_fwd_fp8(q, k, v, descale_q, descale_k, descale_v, o, lse, causal, scale)
+    return o, lse
 
 
 def bwd_workspace_bytes(B: int, Hq: int, Sq: int, d: int) -> int:

@@ -9,6 +9,9 @@ Recipe (fixed so that every caller sees the same tensors for a seed):
   * ``randn`` in fp32, drawn in the order Q, K, V (shape order below);
   * Q multiplied by ``q_mult`` (a power of two, so the product is exact);
   * rounded to bf16 (round-to-nearest-even, torch's ``.to(bfloat16)``).
+  * FP8 prefill: the same fp32 draws, each of Q, K, V scaled per (batch,
+    key/value head) so its largest magnitude is 448 and rounded to E4M3
+    (quantize_e4m3); the factors are returned beside the codes;
   * decode: per-sequence KV lengths ``randint(lmin, lmax + 1)`` drawn after
     K and V from the same generator; cache positions at or beyond a
     sequence's length are filled with ``pad_value`` (NaN by default) so that
@@ -182,6 +185,48 @@ def paged_decode_inputs(B: int, Hq: int, Hkv: int, Lmin: int, Lmax: int, d: int,
     q, kc, vc, seqlens = decode_inputs(B, Hq, Hkv, Lmin, Lmax, d, seed, device, pad_value)
     k_pages, v_pages, table = paginate(kc, vc, seqlens, page_size, seed, pad_value)
     return q, k_pages, v_pages, table, seqlens
+
+
+E4M3_MAX = 448.0
+
+
+def quantize_e4m3(x: torch.Tensor, Hkv: int):
+    """E4M3 codes and per-(batch, key/value head) dequantisation factors for a
+    [B,H,S,d] tensor, the way a caller would prepare FP8 inputs: the factor of
+    (b, g) is max|x| over the heads of group g divided by 448 (1 for an all-zero
+    group), and x8 = x / factor rounded to E4M3 by torch (nearest even).
+    Returns (x8 as torch.float8_e4m3fn, factors [B, Hkv] fp32)."""
+    B, H = int(x.shape[0]), int(x.shape[1])
+    xf = x.float()
+    flat = xf.abs().reshape(B, Hkv, -1)
+    amax = (flat.amax(dim=2) if flat.shape[2] > 0
+            else torch.zeros((B, Hkv), device=x.device, dtype=torch.float32))
+    descale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
+    per_head = descale.repeat_interleave(H // Hkv, dim=1)[:, :, None, None]
+    x8 = (xf / per_head).clamp_(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn)
+    return x8.contiguous(), descale.contiguous()
+
+
+def fp8_prefill_inputs(B: int, Hq: int, Hkv: int, Sq: int, Skv: int, d: int, seed: int,
+                       q_mult: float = 1.0, device="cpu"):
+    """The prefill_inputs() draws (fp32, before any rounding) quantised to E4M3
+    with quantize_e4m3(): (q8, k8, v8, descale_q, descale_k, descale_v)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    q = torch.randn((B, Hq, Sq, d), generator=g, device=device, dtype=torch.float32)
+    k = torch.randn((B, Hkv, Skv, d), generator=g, device=device, dtype=torch.float32)
+    v = torch.randn((B, Hkv, Skv, d), generator=g, device=device, dtype=torch.float32)
+    if q_mult != 1.0:
+        q.mul_(q_mult)
+    q8, dq = quantize_e4m3(q, Hkv)
+    k8, dk = quantize_e4m3(k, Hkv)
+    v8, dv = quantize_e4m3(v, Hkv)
+    return q8, k8, v8, dq, dk, dv
+
+
+def fp8_prefill_inputs_for(shape: PrefillShape, device="cpu"):
+    return fp8_prefill_inputs(shape.B, shape.Hq, shape.Hkv, shape.Sq, shape.Skv, shape.d,
+                              shape.seed, shape.q_mult, device)
 
 
 def grad_output(shape, seed: int, device="cpu"):

@@ -29,7 +29,7 @@ def declared_functions():
 
 def test_header_declares_expected_calls():
     names = declared_functions()
-    for n in ("fa_fwd", "fa_decode_splitkv", "fa_combine", "fa_status_string"):
+    for n in ("fa_fwd", "fa_fwd_fp8", "fa_decode_splitkv", "fa_combine", "fa_status_string"):
         assert n in names
     assert set(names) == set(fa.SIGNATURES), "binding and header disagree"
 
@@ -68,6 +68,7 @@ def fwd(lib, *, q=A, k=A, v=A, o=A, lse=A, B=1, Hq=4, Hkv=4, Sq=128, Skv=128, d=
     (dict(Skv=-1), INVALID),
     (dict(scale=float("nan")), INVALID),
     (dict(scale=float("inf")), INVALID),
+    (dict(scale=-0.125), UNSUPPORTED),   # the kernel follows the largest raw score
     (dict(q=None), INVALID),
     (dict(lse=None), INVALID),
     (dict(v=A + 8), ALIGNMENT),
@@ -77,6 +78,32 @@ def fwd(lib, *, q=A, k=A, v=A, o=A, lse=A, B=1, Hq=4, Hkv=4, Sq=128, Skv=128, d=
 ])
 def test_fwd_rejects_before_cuda(lib, kw, want):
     assert fwd(lib, **kw) == want
+
+
+def fwd8(lib, *, q=A, k=A, v=A, dq=None, dk=None, dv=None, o=A, lse=A, B=1, Hq=4, Hkv=4,
+         Sq=128, Skv=128, d=128, causal=0, scale=0.125):
+    return lib.fa_fwd_fp8(q, k, v, dq, dk, dv, o, lse, B, Hq, Hkv, Sq, Skv, d, causal, scale,
+                          None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(d=64), UNSUPPORTED),          # 8-bit inputs: d = 128 only
+    (dict(d=256), UNSUPPORTED),
+    (dict(Hq=4, Hkv=3), INVALID),
+    (dict(Hkv=0), INVALID),
+    (dict(Sq=-1), INVALID),
+    (dict(scale=float("nan")), INVALID),
+    (dict(scale=-1.0), UNSUPPORTED),
+    (dict(q=None), INVALID),
+    (dict(lse=None), INVALID),
+    (dict(k=A + 8), ALIGNMENT),
+    (dict(dq=A + 2), ALIGNMENT),        # factor arrays: 4-byte aligned
+    (dict(dv=A + 1), ALIGNMENT),
+    (dict(B=0, q=None), OK),
+    (dict(Sq=0, q=None, o=None), OK),
+])
+def test_fwd_fp8_rejects_before_cuda(lib, kw, want):
+    assert fwd8(lib, **kw) == want
 
 
 def dec(lib, *, q=A, kc=A, vc=A, sl=A, op=A, lp=A, B=2, Hq=8, Hkv=2, Lmax=64, d=128, n=4,
@@ -91,6 +118,7 @@ def dec(lib, *, q=A, kc=A, vc=A, sl=A, op=A, lp=A, B=2, Hq=8, Hkv=2, Lmax=64, d=
     (dict(n=0), INVALID),
     (dict(n=257), INVALID),
     (dict(Lmax=-1), INVALID),
+    (dict(scale=-0.1), UNSUPPORTED),
     (dict(sl=None), INVALID),
     (dict(op=A + 4), ALIGNMENT),
     (dict(sl=A + 2), ALIGNMENT),
@@ -117,6 +145,7 @@ def paged(lib, *, q=A, kp=A, vp=A, bt=A, sl=A, op=A, lp=A, B=2, Hq=8, Hkv=2, pag
     (dict(max_pages=0), INVALID),
     (dict(n=0), INVALID),
     (dict(scale=float("nan")), INVALID),
+    (dict(scale=-0.1), UNSUPPORTED),
     (dict(bt=None), INVALID),
     (dict(vp=None), INVALID),
     (dict(bt=A + 2), ALIGNMENT),

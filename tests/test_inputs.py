@@ -6,8 +6,10 @@ import pytest
 import torch
 
 import oracle
-from io_aware_exact_flashattention_b200.inputs import (decode_inputs, grad_output, paginate,
-                                                       paged_decode_inputs, prefill_inputs)
+from io_aware_exact_flashattention_b200.inputs import (decode_inputs, fp8_prefill_inputs,
+                                                       grad_output, paginate,
+                                                       paged_decode_inputs, prefill_inputs,
+                                                       quantize_e4m3)
 
 
 def test_prefill_inputs_deterministic_and_scaled():
@@ -58,3 +60,34 @@ def test_paged_decode_inputs_match_decode_inputs():
     o, lse = oracle.decode_paged(q, kp, vp, bt, sl, 0.125)
     o2, lse2 = oracle.decode(q2, kc, vc, sl2, 0.125)
     assert np.array_equal(o, o2) and np.array_equal(lse, lse2)
+
+
+def test_quantiser_round_trip():
+    """quantize_e4m3's codes dequantise (through the oracle) to within E4M3
+    rounding of the input: 2^-4 relative for normal codes, 2^-10 of the
+    factor for subnormal ones; each group's largest magnitude maps to 448."""
+    x = torch.randn((2, 4, 64, 128), generator=torch.Generator().manual_seed(3))
+    x8, ds = quantize_e4m3(x, 2)
+    assert x8.dtype == torch.float8_e4m3fn and tuple(ds.shape) == (2, 2)
+    back = oracle.dequant_heads(x8, ds, 2)
+    per_head = ds.repeat_interleave(2, dim=1)[:, :, None, None].double().numpy()
+    xd = x.double().numpy()
+    assert (np.abs(back - xd) <= np.abs(xd) * 2.0 ** -4 + 2.0 ** -10 * per_head).all()
+    codes = x8.float().abs().reshape(2, 2, -1).amax(dim=2)
+    assert torch.equal(codes, torch.full((2, 2), 448.0))
+
+
+def test_fp8_inputs_deterministic():
+    a = fp8_prefill_inputs(1, 4, 2, 30, 40, 128, seed=8, q_mult=8.0)
+    b = fp8_prefill_inputs(1, 4, 2, 30, 40, 128, seed=8, q_mult=8.0)
+    for x, y in zip(a, b):
+        assert torch.equal(x.view(torch.uint8) if x.element_size() == 1 else x,
+                           y.view(torch.uint8) if y.element_size() == 1 else y)
+    q8, k8, v8, dq, dk, dv = a
+    assert q8.shape == (1, 4, 30, 128) and k8.shape == (1, 2, 40, 128)
+    assert dq.shape == dk.shape == dv.shape == (1, 2)
+
+
+def test_quantiser_empty_sequence():
+    x8, ds = quantize_e4m3(torch.zeros((2, 4, 0, 128)), 2)
+    assert x8.shape == (2, 4, 0, 128) and torch.equal(ds, torch.ones((2, 2)))

@@ -78,7 +78,7 @@ def test_gqa_groups(Hq, Hkv, causal):
     check_full(2, Hq, Hkv, 384, 384, 128, causal, seed=7 * Hq + Hkv)
 
 
-@pytest.mark.parametrize("Sq,Skv", [(100, 700), (384, 1000), (1, 900), (700, 300), (260, 129)])
+@pytest.mark.parametrize("Sq,Skv", [(100, 700), (384, 1000), (1, 900), (700, 300), (260, 129), (128, 0)])
 @pytest.mark.parametrize("causal", [False, True])
 def test_rectangular(Sq, Skv, causal):
     # causal with Sq > Skv leaves leading rows with no visible key: O = 0, LSE = -inf
