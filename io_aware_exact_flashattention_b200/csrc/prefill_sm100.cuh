@@ -85,6 +85,11 @@ constexpr float kExp2C3 = 5.517166853e-02f;
 // took more cycles than the MUFU alone (2-7 %); the polynomial stays as a
 // tested option (fa_debug_exp2_poly checks it against the MUFU).
 constexpr int kPolyPairsPer8 = 0;
+// The same share for 8-bit P.  There the E4M3 products take half the tensor
+// time, so the softmax's exponentials rather than the MMA set the key tile
+// period: on B200, 2 of 8 pairs on the polynomial took 2.6 % (S = 2048) and
+// 4.4 % (S = 8192) less time than none, 3 of 8 about the same, 4 of 8 more.
+constexpr int kPolyPairsPer8F8 = 2;
 
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer
@@ -353,15 +358,17 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
     auto exps_half = [&](auto poly_tag, int half) {
       constexpr bool kPoly = decltype(poly_tag)::value;
       if constexpr (kF8) {
-        // four keys per 32-bit column, all exponentials on the MUFU
+        // four keys per 32-bit column; pairs (2i, 2i+1) of the row
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int e = half * 64 + 4 * i;
           const float2 x0 = ffma2(make_float2(s[e], s[e + 1]), c2, nmc2);
           const float2 x1 = ffma2(make_float2(s[e + 2], s[e + 3]), c2, nmc2);
-          const float2 p0 = make_float2(ex2(x0.x), ex2(x0.y));
-          const float2 p1 = make_float2(ex2(x1.x), ex2(x1.y));
+          const float2 p0 = (kPoly && ((2 * i) & 7) >= 8 - kPolyPairsPer8F8)
+                                ? exp2_poly2(x0) : make_float2(ex2(x0.x), ex2(x0.y));
+          const float2 p1 = (kPoly && ((2 * i + 1) & 7) >= 8 - kPolyPairsPer8F8)
+                                ? exp2_poly2(x1) : make_float2(ex2(x1.x), ex2(x1.y));
           rs[(2 * i) & 3] = fadd2(rs[(2 * i) & 3], p0);
           rs[(2 * i + 1) & 3] = fadd2(rs[(2 * i + 1) & 3], p1);
           pk[i] = pack_e4m3x4(p0.x, p0.y, p1.x, p1.y);
