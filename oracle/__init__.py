@@ -85,6 +85,8 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_e4m3_decode.restype = ci
     lib.oracle_dequant_heads.argtypes = [_U8, _D, _D] + [ci] * 5
     lib.oracle_dequant_heads.restype = ci
+    lib.oracle_ffn.argtypes = [_D, _D, _D, _D, ctypes.c_int64, ci, ci]
+    lib.oracle_ffn.restype = ci
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ci
     return lib
@@ -308,6 +310,35 @@ def attn_fwd_fp8(q8, k8, v8, descale_q, descale_k, descale_v, causal: bool, scal
     k = dequant_heads(k8, descale_k, Hkv, lib)
     v = dequant_heads(v8, descale_v, Hkv, lib)
     return attn_fwd(q, k, v, causal, scale, lib=lib)
+
+
+def ffn(x, w1, w2, lib: Optional[ctypes.CDLL] = None) -> np.ndarray:
+    """y [..., D] = W2 gelu(W1 x) per token (x [..., D], w1 [F, D], w2 [D, F])."""
+    lib = lib or load()
+    x, w1, w2 = _f64(x), _f64(w1), _f64(w2)
+    F, D = w1.shape
+    if w2.shape != (D, F) or x.shape[-1] != D:
+        raise ValueError("ffn: x [..., D], w1 [F, D], w2 [D, F]")
+    xs = np.ascontiguousarray(x.reshape(-1, D))
+    y = np.zeros(xs.shape)
+    if lib.oracle_ffn(_p(xs), _p(w1), _p(w2), _p(y), xs.shape[0], D, F) != 0:
+        raise ValueError("oracle_ffn rejected its arguments")
+    return y.reshape(x.shape)
+
+
+def heads_to_tokens(o) -> np.ndarray:
+    """[B, Hq, S, d] attention output -> [B, S, Hq * d] token rows (the
+    concatenation over heads; data movement only)."""
+    o = _f64(o)
+    B, Hq, S, d = o.shape
+    return np.ascontiguousarray(o.transpose(0, 2, 1, 3).reshape(B, S, Hq * d))
+
+
+def bpt_layer(q, k, v, w1, w2, causal: bool, scale: float, lib: Optional[ctypes.CDLL] = None):
+    """Attention followed by the feed-forward network on every token:
+    y [B, S, Hq * d] (float64), plus the attention's O and LSE."""
+    o, lse = attn_fwd(q, k, v, causal, scale, lib=lib)
+    return ffn(heads_to_tokens(o), w1, w2, lib=lib), o, lse
 
 
 def num_threads(lib: Optional[ctypes.CDLL] = None) -> int:

@@ -451,6 +451,59 @@ int oracle_dequant_heads(const uint8_t *x8, const double *descale, double *out, 
     return 0;
 }
 
+/* --- Blockwise feed-forward after attention ---------------------------------
+ * "I/O-Aware Kernels", section "Blockwise Parallel Transformers": the
+ * feed-forward network acts on every token independently, so it can run on a
+ * query block as soon as that block's attention is done, and only that
+ * block's activations are ever materialised.  The result is that of the
+ * unblocked layer, which is what this oracle computes.  Reading of what the
+ * page leaves open: the network's input for token t is the concatenation over
+ * query heads of the attention output, x_t = (O[b,0,t,:], ..., O[b,Hq-1,t,:])
+ * of width D = Hq * d; the network is two bias-free linear maps with the erf
+ * form of GELU between them: y_t = W2 gelu(W1 x_t), W1 [F, D], W2 [D, F]. */
+
+static double gelu(double h)
+{
+    return 0.5 * h * (1.0 + erf(h / sqrt(2.0)));
+}
+
+/* x [n, D] -> y [n, D]; hidden [F] per token in scratch. */
+int oracle_ffn(const double *x, const double *w1, const double *w2, double *y, int64_t n,
+               int D, int F)
+{
+    if (n < 0 || D < 1 || F < 1)
+        return -1;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *hid = (double *)malloc(sizeof(double) * (size_t)F);
+        if (!hid) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t t = 0; t < n; ++t) {
+                const double *xt = x + t * D;
+                for (int f = 0; f < F; ++f) {
+                    const double *w = w1 + (int64_t)f * D;
+                    double acc = 0.0;
+                    for (int i = 0; i < D; ++i) acc += w[i] * xt[i];
+                    hid[f] = gelu(acc);
+                }
+                double *yt = y + t * D;
+                for (int i = 0; i < D; ++i) {
+                    const double *w = w2 + (int64_t)i * F;
+                    double acc = 0.0;
+                    for (int f = 0; f < F; ++f) acc += w[f] * hid[f];
+                    yt[i] = acc;
+                }
+            }
+            free(hid);
+        }
+    }
+    return err ? -1 : 0;
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -14,7 +14,10 @@ oracle disagrees with:
   * reductions: GQA == MHA with repeated K/V, decode == prefill with one query,
     split + combine == unsplit;
   * for E4M3 inputs: code values derived by hand (tests/golden/e4m3_codes.json),
-    torch's float8_e4m3fn decoding, and a one-key closed form per head.
+    torch's float8_e4m3fn decoding, and a one-key closed form per head;
+  * for the feed-forward network after attention: textbook values of the normal
+    CDF, torch's fp64 GELU network, token independence (blockwise == full) and
+    the head-to-token concatenation by hand.
 """
 from __future__ import annotations
 
@@ -563,6 +566,68 @@ def pin_fp8_one_key_closed_form(lib):
                 _close(o[b, h, i], dv[b, g] * vv[b, g, 0], 1e-12, "fp8 one-key O")
 
 
+# --------------------------------------------------------------------------
+# Feed-forward network after attention (blockwise parallel transformer)
+
+def pin_ffn_gelu_closed_forms(lib):
+    """D = F = 1 with unit weights: y = gelu(x) = x * Phi(x).  Phi(1) and
+    Phi(2) are the textbook values of the standard normal CDF; gelu(0) = 0;
+    gelu(x) - gelu(-x) = x; gelu(x) -> x for large x."""
+    xs = np.array([0.0, 1.0, -1.0, 2.0, -2.0, 10.0, 0.5, -0.5]).reshape(-1, 1)
+    y = oracle.ffn(xs, np.ones((1, 1)), np.ones((1, 1)), lib=lib).ravel()
+    phi1, phi2 = 0.8413447460685429, 0.9772498680518208
+    _close(y[0], 0.0, 1e-15, "gelu(0)")
+    _close(y[1], phi1, 1e-15, "gelu(1)")
+    _close(y[2], -(1.0 - phi1), 1e-15, "gelu(-1)")
+    _close(y[3], 2.0 * phi2, 1e-15, "gelu(2)")
+    _close(y[4], -2.0 * (1.0 - phi2), 1e-15, "gelu(-2)")
+    _close(y[5], 10.0, 1e-14, "gelu(10)")
+    _close(y[6] - y[7], 0.5, 1e-15, "gelu(x) - gelu(-x) = x")
+
+
+def pin_ffn_torch(lib):
+    """torch's fp64 GELU (erf form) between two bias-free linear maps."""
+    rng = np.random.default_rng(41)
+    for n, D, F in ((7, 16, 40), (1, 3, 5), (20, 8, 32)):
+        x = _rand((n, D), rng)
+        w1 = _rand((F, D), rng, 0.3)
+        w2 = _rand((D, F), rng, 0.3)
+        y = oracle.ffn(x, w1, w2, lib=lib)
+        tx, t1, t2 = (torch.tensor(a) for a in (x, w1, w2))
+        want = (torch.nn.functional.gelu(tx @ t1.T) @ t2.T).numpy()
+        _close(y, want, 1e-12, "ffn vs torch (n=%d D=%d F=%d)" % (n, D, F))
+
+
+def pin_ffn_tokens_independent(lib):
+    """The property blockwise scheduling rests on ("I/O-Aware Kernels",
+    section "Blockwise Parallel Transformers"): each token's output depends on
+    that token alone, so blocks of any size, in any order, give the full result."""
+    rng = np.random.default_rng(43)
+    x = _rand((2, 23, 12), rng)
+    w1, w2 = _rand((30, 12), rng, 0.4), _rand((12, 30), rng, 0.4)
+    full = oracle.ffn(x, w1, w2, lib=lib)
+    for blk in (1, 3, 7, 23):
+        parts = [oracle.ffn(x[:, s:s + blk], w1, w2, lib=lib) for s in range(0, 23, blk)]
+        _close(np.concatenate(parts, axis=1), full, 1e-15, "blockwise FFN (block %d)" % blk)
+    perm = rng.permutation(23)
+    _close(oracle.ffn(x[:, perm], w1, w2, lib=lib), full[:, perm], 1e-15, "token permutation")
+
+
+def pin_heads_to_tokens_by_hand(lib):
+    """Token t's row is (O[b,0,t,:], O[b,1,t,:], ...), written out by hand."""
+    o = np.arange(1 * 2 * 3 * 2, dtype=np.float64).reshape(1, 2, 3, 2)
+    want = np.array([[[0, 1, 6, 7], [2, 3, 8, 9], [4, 5, 10, 11]]], dtype=np.float64)
+    got = oracle.heads_to_tokens(o)
+    assert np.array_equal(got, want), got
+    y, o2, _ = oracle.bpt_layer(np.ones((1, 2, 3, 2)), np.ones((1, 1, 3, 2)),
+                                o[:, :1], np.eye(4), np.eye(4), False, 1.0, lib=lib)
+    # equal scores: every query's O is the mean of V's rows; FFN = gelu with identity weights
+    mean_v = o[0, 0].mean(axis=0)
+    _close(o2[0, 1, 2], mean_v, 1e-15, "bpt attention part")
+    phi = 0.5 * (1.0 + np.array([math.erf(m / math.sqrt(2.0)) for m in mean_v]))
+    _close(y[0, 2], np.concatenate([mean_v * phi] * 2), 1e-14, "bpt layer with identity FFN")
+
+
 ALL_PINS = [
     pin_golden_prefill,
     pin_golden_combine,
@@ -584,4 +649,8 @@ ALL_PINS = [
     pin_e4m3_matches_torch,
     pin_e4m3_order_and_sign,
     pin_fp8_one_key_closed_form,
+    pin_ffn_gelu_closed_forms,
+    pin_ffn_torch,
+    pin_ffn_tokens_independent,
+    pin_heads_to_tokens_by_hand,
 ]

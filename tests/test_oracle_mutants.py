@@ -49,6 +49,13 @@ MUTANTS = [
     ("dequant_query_head_modulo", "const int64_t g = h / group;\n            const double f",
      "const int64_t g = h % Hkv;\n            const double f"),
     ("dequant_batch_ignored", "descale[b * Hkv + g]", "descale[g]"),
+    ("gelu_missing_half", "return 0.5 * h * (1.0 + erf(h / sqrt(2.0)));",
+     "return h * (1.0 + erf(h / sqrt(2.0)));"),
+    ("gelu_erf_unscaled", "return 0.5 * h * (1.0 + erf(h / sqrt(2.0)));",
+     "return 0.5 * h * (1.0 + erf(h));"),
+    ("ffn_w1_row_frozen", "const double *w = w1 + (int64_t)f * D;", "const double *w = w1;"),
+    ("ffn_w2_row_frozen", "const double *w = w2 + (int64_t)i * F;", "const double *w = w2;"),
+    ("ffn_token_frozen", "const double *xt = x + t * D;", "const double *xt = x;"),
 ]
 
 
