@@ -85,6 +85,8 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_e4m3_decode.restype = ci
     lib.oracle_dequant_heads.argtypes = [_U8, _D, _D] + [ci] * 5
     lib.oracle_dequant_heads.restype = ci
+    lib.oracle_ffn_hidden.argtypes = [_D, _D, _D, ctypes.c_int64, ci, ci]
+    lib.oracle_ffn_hidden.restype = ci
     lib.oracle_ffn.argtypes = [_D, _D, _D, _D, ctypes.c_int64, ci, ci]
     lib.oracle_ffn.restype = ci
     lib.oracle_num_threads.argtypes = []
@@ -324,6 +326,20 @@ def ffn(x, w1, w2, lib: Optional[ctypes.CDLL] = None) -> np.ndarray:
     if lib.oracle_ffn(_p(xs), _p(w1), _p(w2), _p(y), xs.shape[0], D, F) != 0:
         raise ValueError("oracle_ffn rejected its arguments")
     return y.reshape(x.shape)
+
+
+def ffn_hidden(x, w1, lib: Optional[ctypes.CDLL] = None) -> np.ndarray:
+    """The activations between the two maps: gelu(W1 x) [..., F] per token."""
+    lib = lib or load()
+    x, w1 = _f64(x), _f64(w1)
+    F, D = w1.shape
+    if x.shape[-1] != D:
+        raise ValueError("ffn_hidden: x [..., D], w1 [F, D]")
+    xs = np.ascontiguousarray(x.reshape(-1, D))
+    h = np.zeros((xs.shape[0], F))
+    if lib.oracle_ffn_hidden(_p(xs), _p(w1), _p(h), xs.shape[0], D, F) != 0:
+        raise ValueError("oracle_ffn_hidden rejected its arguments")
+    return h.reshape(x.shape[:-1] + (F,))
 
 
 def heads_to_tokens(o) -> np.ndarray:

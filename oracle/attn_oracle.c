@@ -467,6 +467,28 @@ static double gelu(double h)
     return 0.5 * h * (1.0 + erf(h / sqrt(2.0)));
 }
 
+/* hid [F] = gelu(W1 x_t) for one token. */
+static void ffn_token_hidden(const double *xt, const double *w1, int D, int F, double *hid)
+{
+    for (int f = 0; f < F; ++f) {
+        const double *w = w1 + (int64_t)f * D;
+        double acc = 0.0;
+        for (int i = 0; i < D; ++i) acc += w[i] * xt[i];
+        hid[f] = gelu(acc);
+    }
+}
+
+/* hidden [n, F] = gelu(W1 x) per token (the activations between the two maps). */
+int oracle_ffn_hidden(const double *x, const double *w1, double *hid, int64_t n, int D, int F)
+{
+    if (n < 0 || D < 1 || F < 1)
+        return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < n; ++t)
+        ffn_token_hidden(x + t * D, w1, D, F, hid + t * F);
+    return 0;
+}
+
 /* x [n, D] -> y [n, D]; hidden [F] per token in scratch. */
 int oracle_ffn(const double *x, const double *w1, const double *w2, double *y, int64_t n,
                int D, int F)
@@ -483,13 +505,7 @@ int oracle_ffn(const double *x, const double *w1, const double *w2, double *y, i
         } else {
 #pragma omp for schedule(static)
             for (int64_t t = 0; t < n; ++t) {
-                const double *xt = x + t * D;
-                for (int f = 0; f < F; ++f) {
-                    const double *w = w1 + (int64_t)f * D;
-                    double acc = 0.0;
-                    for (int i = 0; i < D; ++i) acc += w[i] * xt[i];
-                    hid[f] = gelu(acc);
-                }
+                ffn_token_hidden(x + t * D, w1, D, F, hid);
                 double *yt = y + t * D;
                 for (int i = 0; i < D; ++i) {
                     const double *w = w2 + (int64_t)i * F;

@@ -598,6 +598,18 @@ def pin_ffn_torch(lib):
         _close(y, want, 1e-12, "ffn vs torch (n=%d D=%d F=%d)" % (n, D, F))
 
 
+def pin_ffn_hidden(lib):
+    """The hidden activations: torch's fp64 gelu(x W1^T), and the second map
+    applied to them gives the network's output."""
+    rng = np.random.default_rng(47)
+    x = _rand((9, 16), rng)
+    w1, w2 = _rand((24, 16), rng, 0.3), _rand((16, 24), rng, 0.3)
+    h = oracle.ffn_hidden(x, w1, lib=lib)
+    want = torch.nn.functional.gelu(torch.tensor(x) @ torch.tensor(w1).T).numpy()
+    _close(h, want, 1e-13, "ffn hidden vs torch")
+    _close(h @ w2.T, oracle.ffn(x, w1, w2, lib=lib), 1e-13, "ffn = W2 hidden")
+
+
 def pin_ffn_tokens_independent(lib):
     """The property blockwise scheduling rests on ("I/O-Aware Kernels",
     section "Blockwise Parallel Transformers"): each token's output depends on
@@ -651,6 +663,7 @@ ALL_PINS = [
     pin_fp8_one_key_closed_form,
     pin_ffn_gelu_closed_forms,
     pin_ffn_torch,
+    pin_ffn_hidden,
     pin_ffn_tokens_independent,
     pin_heads_to_tokens_by_hand,
 ]

@@ -55,7 +55,11 @@ MUTANTS = [
      "return 0.5 * h * (1.0 + erf(h));"),
     ("ffn_w1_row_frozen", "const double *w = w1 + (int64_t)f * D;", "const double *w = w1;"),
     ("ffn_w2_row_frozen", "const double *w = w2 + (int64_t)i * F;", "const double *w = w2;"),
-    ("ffn_token_frozen", "const double *xt = x + t * D;", "const double *xt = x;"),
+    ("ffn_token_frozen", "ffn_token_hidden(x + t * D, w1, D, F, hid);",
+     "ffn_token_hidden(x, w1, D, F, hid);"),
+    ("ffn_hidden_token_frozen", "ffn_token_hidden(x + t * D, w1, D, F, hid + t * F);",
+     "ffn_token_hidden(x, w1, D, F, hid + t * F);"),
+    ("ffn_hidden_no_gelu", "hid[f] = gelu(acc);", "hid[f] = acc;"),
 ]
 
 
