@@ -73,6 +73,10 @@ def parse_args():
                     help="skip the backward measurement on the prefill workload")
     ap.add_argument("--no-fp8", action="store_true",
                     help="skip the E4M3-input forward on the prefill workload")
+    ap.add_argument("--no-bpt", action="store_true",
+                    help="skip the blockwise feed-forward network after the prefill attention")
+    ap.add_argument("--bpt-chunk", type=int, default=16,
+                    help="query tiles per chunk of the blockwise feed-forward network")
     ap.add_argument("--page-size", type=int, default=16,
                     help="page size of the paged-cache decode measurement")
     return ap.parse_args()
@@ -465,6 +469,49 @@ def run_ours(args, world, rank, local):
             "note": "same shape and FLOP count as the bf16 prefill; measured outside the step"}
         del q8, k8, v8, dq8, dk8, dv8
 
+    # Blockwise feed-forward network (F = 4 D) on the forward's attention
+    # output, chunk by chunk; random stand-in weights.  Measured on its own.
+    bpt = None
+    if do_pre and not args.no_bpt and (c.Hq * c.d) % 256 == 0:
+        from io_aware_exact_flashattention_b200.inputs import ffn_inputs
+        D = c.Hq * c.d
+        F = 4 * D
+        _, w1, w2 = ffn_inputs(1, c.Hq, 1, c.d, F, rank_seed(c.seed, rank), device=dev)
+        chunk = max(1, args.bpt_chunk)
+        y = torch.empty((c.B, c.Sq, D), device=dev, dtype=torch.bfloat16)
+        ws = torch.empty(max(16, fa.bpt_workspace_bytes(F, chunk)), dtype=torch.uint8, device=dev)
+        fa.fa_fwd(q, k, v, o, lse, c.causal, c.scale, stream=stream)
+        for _ in range(max(args.warmup, 1)):
+            fa.fa_bpt_ffn(o, w1, w2, y, ws, chunk, stream=stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        pevs = []
+        for _ in range(K):
+            flush.fill_(1.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fa.fa_bpt_ffn(o, w1, w2, y, ws, chunk, stream=stream)
+            b.record(stream)
+            pevs.append((a, b))
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        bpt_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in pevs)], world)[0]
+        ffn_flops = 4.0 * c.B * c.Sq * D * F
+        bpt_tf = ffn_flops / (bpt_ms * 1e-3 / K) / 1e12
+        tiles = c.B * ((c.Sq + 127) // 128)
+        n_chunks = (tiles + chunk - 1) // chunk
+        bpt = {"value": aggregate_rate(world, ffn_flops, K, bpt_ms) / 1e12, "unit": "TFLOP/s",
+               "ms_per_call": bpt_ms / K,
+               "frac_of_measured_burst": bpt_tf / float(peaks["bf16_tflops"]),
+               "algorithmic": "%.4g FLOP per call (two products, 2 x 2 x tokens x D x F; "
+                              "D = %d, F = %d)" % (ffn_flops, D, F),
+               "chunk_tiles": chunk, "hidden_bytes_per_chunk": chunk * 128 * F * 2,
+               "hidden_bytes_unblocked": c.B * c.Sq * F * 2,
+               "kernels": "fa_ffn_gemm_kernel, two launches per chunk",
+               "gpu_launches": 2 * n_chunks * K, "traffic_main_kernel": None,
+               "note": "y = W2 gelu(W1 x_t) on the forward's output; measured outside the step"}
+        del y, ws, w1, w2
+
     # Paged cache: the same decode workload stored in page_size-key pages
     # scattered over a pool, read through a block table.  Measured on its own,
     # outside the step.
@@ -577,6 +624,8 @@ def run_ours(args, world, rank, local):
         line["backward"] = backward
     if prefill_fp8 is not None:
         line["prefill_fp8"] = prefill_fp8
+    if bpt is not None:
+        line["bpt_ffn"] = bpt
     if cpu is not None:
         line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)

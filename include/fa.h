@@ -147,6 +147,39 @@ fa_status fa_bwd(const void *q, const void *k, const void *v, const void *o,
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Sq, int d);
 
 /*
+ * fa_bpt_ffn -- the feed-forward network after attention, run blockwise
+ * ("I/O-Aware Kernels", section "Blockwise Parallel Transformers": the
+ * network acts on each token alone, so it runs on blocks of query rows and
+ * only one block's activations are materialised).  The page fixes no network;
+ * this call defines it:
+ *
+ *   x_t = (o[b,0,t,:], ..., o[b,Hq-1,t,:])       (concatenation over heads, D = Hq*d)
+ *   y[b,t,:] = W2 gelu(W1 x_t)                    (gelu(h) = h/2 (1 + erf(h/sqrt 2)))
+ *
+ *   o   [B, Hq, S, d] bf16 (an attention output, as fa_fwd writes it)
+ *   w1  [F, D] bf16, w2 [D, F] bf16 (row-major; no biases)
+ *   y   [B, S, D] bf16 (written)
+ *   workspace  fa_bpt_workspace_bytes(F, chunk_tiles) bytes, caller-owned
+ *
+ * The query rows are taken in chunks of chunk_tiles tiles of 128 rows (over
+ * all sequences, in order).  Per chunk, one launch writes the chunk's hidden
+ * activations gelu(X W1^T) to the workspace (chunk_tiles * 128 * F bf16) and
+ * a second writes Y = H W2^T.  So the F-wide activations exist for one chunk
+ * at a time; chunk_tiles trades that memory against launches.  Both products
+ * run on the tensor cores with fp32 accumulation; H and y are rounded to
+ * bf16 once each.
+ *
+ * Supported: d in {64, 128}; D and F multiples of 256; chunk_tiles in
+ * [1, 65535].  Pointers 16-byte aligned.  B == 0 or S == 0 is a no-op.
+ * Errors as for fa_fwd (FA_ERR_UNSUPPORTED for other sizes).
+ */
+fa_status fa_bpt_ffn(const void *o, const void *w1, const void *w2, void *y, void *workspace,
+                     int B, int Hq, int S, int d, int F, int chunk_tiles, fa_stream_t stream);
+
+/* Bytes of scratch fa_bpt_ffn needs: chunk_tiles * 128 * F bf16 values. */
+size_t fa_bpt_workspace_bytes(int F, int chunk_tiles);
+
+/*
  * fa_decode_splitkv -- first half of single-query decode (Sq = 1, no mask).
  *
  * The key/value length L_b = seqlens_k[b] of sequence b is cut into

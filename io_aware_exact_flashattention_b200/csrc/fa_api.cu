@@ -16,6 +16,7 @@
 #include "prefill_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "backward_sm100.cuh"
+#include "ffn_sm100.cuh"
 
 namespace {
 
@@ -68,6 +69,21 @@ bool encode_bhsd_e4m3(CUtensorMap* map, const void* base, int d, int rows, long 
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [rows, cols] bf16 matrix (a weight, K = cols contiguous) as a 3-D map with
+// 64 x 256 x 1 boxes, 128B swizzle.
+bool encode_rows256(CUtensorMap* map, const void* base, int cols, int rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows), 1};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 2,
+                           static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[3] = {64, 256, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -420,6 +436,20 @@ fa_status launch_backward(const void* q, const void* k, const void* v, const voi
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// Feed-forward network after attention: per-device shared-memory opt-in.
+std::once_flag g_ffn_once[kMaxDevices];
+cudaError_t g_ffn_err[kMaxDevices];
+
+cudaError_t prepare_ffn(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::call_once(g_ffn_once[dev], [dev] {
+    g_ffn_err[dev] = cudaFuncSetAttribute(fa::fa_ffn_gemm_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          fa::FfnLayout::kBytes);
+  });
+  return g_ffn_err[dev];
+}
+
 extern "C" {
 
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Sq, int d) {
@@ -513,6 +543,71 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, const float* d
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   return launch_prefill<128, true>(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, causal, scale, s,
                                    descale_q, descale_k, descale_v);
+}
+
+size_t fa_bpt_workspace_bytes(int F, int chunk_tiles) {
+  if (F < 1 || chunk_tiles < 1) return 0;
+  return static_cast<size_t>(chunk_tiles) * fa::kFfnBM * static_cast<size_t>(F) * 2;
+}
+
+fa_status fa_bpt_ffn(const void* o, const void* w1, const void* w2, void* y,
+                                void* workspace, int B, int Hq, int S, int d, int F,
+                                int chunk_tiles, fa_stream_t stream) {
+  if (B < 0 || Hq < 1 || S < 0 || F < 1 || chunk_tiles < 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const long long D = static_cast<long long>(Hq) * d;
+  if (D % fa::kFfnBN != 0 || F % fa::kFfnBN != 0 || D > (1 << 20) || F > (1 << 20))
+    return FA_ERR_UNSUPPORTED;
+  if (B == 0 || S == 0) return FA_OK;  // nothing to compute
+  if (o == nullptr || w1 == nullptr || w2 == nullptr || y == nullptr || workspace == nullptr)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned16(o) || !aligned16(w1) || !aligned16(w2) || !aligned16(y) || !aligned16(workspace))
+    return FA_ERR_ALIGNMENT;
+  const long long tiles_per_seq = (static_cast<long long>(S) + fa::kFfnBM - 1) / fa::kFfnBM;
+  const long long total_tiles = tiles_per_seq * B;
+  if (total_tiles > 0x7fffffffLL || static_cast<long long>(B) * Hq > 0x7fffffffLL ||
+      static_cast<long long>(B) * S * D > (1LL << 40) || chunk_tiles > 65535)
+    return FA_ERR_UNSUPPORTED;
+  CUtensorMap tm_o, tm_w1, tm_w2, tm_h;
+  if (!encode_bhsd(&tm_o, o, d, S, static_cast<long long>(B) * Hq) ||
+      !encode_rows256(&tm_w1, w1, static_cast<int>(D), F) ||
+      !encode_rows256(&tm_w2, w2, F, static_cast<int>(D)) ||
+      !encode_bhsd(&tm_h, workspace, F, chunk_tiles * fa::kFfnBM, 1))
+    return FA_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (prepare_ffn(dev) != cudaSuccess) return FA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  fa::FfnParams p1;  // H = gelu(X W1^T), X read from the attention output
+  p1.c = static_cast<__nv_bfloat16*>(workspace);
+  p1.N = F;
+  p1.K = static_cast<int>(D);
+  p1.S = S;
+  p1.Hq = Hq;
+  p1.d = d;
+  p1.tiles_per_seq = static_cast<int>(tiles_per_seq);
+  p1.a_heads = 1;
+  p1.c_tokens = 0;
+  p1.gelu = 1;
+  p1.wait_limit_ns = kWaitLimitNs;
+  fa::FfnParams p2 = p1;  // Y = H W2^T, rows back to their tokens
+  p2.c = static_cast<__nv_bfloat16*>(y);
+  p2.N = static_cast<int>(D);
+  p2.K = F;
+  p2.a_heads = 0;
+  p2.c_tokens = 1;
+  p2.gelu = 0;
+  for (long long mt0 = 0; mt0 < total_tiles; mt0 += chunk_tiles) {
+    const int n = static_cast<int>(std::min<long long>(chunk_tiles, total_tiles - mt0));
+    p1.mt0 = p2.mt0 = static_cast<int>(mt0);
+    fa::fa_ffn_gemm_kernel<<<dim3(static_cast<unsigned>(F / fa::kFfnBN), static_cast<unsigned>(n)),
+                             fa::kFfnThreads, fa::FfnLayout::kBytes, s>>>(tm_o, tm_w1, p1);
+    fa::fa_ffn_gemm_kernel<<<dim3(static_cast<unsigned>(D / fa::kFfnBN), static_cast<unsigned>(n)),
+                             fa::kFfnThreads, fa::FfnLayout::kBytes, s>>>(tm_h, tm_w2, p2);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
 }
 
 fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,

@@ -38,6 +38,8 @@ SIGNATURES = {
     "fa_combine": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP]),
     "fa_bwd": (_I, [_VP] * 10 + [_I] * 7 + [_F, _VP]),
     "fa_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
+    "fa_bpt_ffn": (_I, [_VP] * 5 + [_I] * 6 + [_VP]),
+    "fa_bpt_workspace_bytes": (ctypes.c_size_t, [_I, _I]),
     "fa_decode_default_splits": (_I, [_I, _I, _I, _I]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_get_device_status": (_I, []),
@@ -175,6 +177,51 @@ def flash_attention_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         lse = torch.empty((B, Hq, Sq), device=q.device, dtype=torch.float32)
     fa_fwd_fp8(q, k, v, descale_q, descale_k, descale_v, o, lse, causal, scale)
     return o, lse
+
+
+def bpt_workspace_bytes(F: int, chunk_tiles: int) -> int:
+    return int(lib().fa_bpt_workspace_bytes(F, chunk_tiles))
+
+
+def fa_bpt_ffn(o: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor, y: torch.Tensor,
+               workspace: torch.Tensor, chunk_tiles: int,
+               stream: Optional[torch.cuda.Stream] = None) -> None:
+    """fa_bpt_ffn: y [B,S,D] = W2 gelu(W1 x_t) with x_t the concatenation over
+    heads of o [B,Hq,S,d]; w1 [F,D], w2 [D,F]; all bf16 on one CUDA device."""
+    for t, n in ((o, "o"), (w1, "w1"), (w2, "w2"), (y, "y")):
+        _need(t, torch.bfloat16, n)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    B, Hq, S, d = o.shape
+    D = Hq * d
+    F = w1.shape[0]
+    if tuple(w1.shape) != (F, D) or tuple(w2.shape) != (D, F) or tuple(y.shape) != (B, S, D):
+        raise ValueError("w1 [F, D], w2 [D, F] and y [B, S, D] with D = Hq * d")
+    if workspace.numel() * workspace.element_size() < bpt_workspace_bytes(F, chunk_tiles):
+        raise ValueError("workspace smaller than fa_bpt_workspace_bytes")
+    _check("fa_bpt_ffn", lib().fa_bpt_ffn(_ptr(o), _ptr(w1), _ptr(w2), _ptr(y), _ptr(workspace),
+                                          B, Hq, S, d, F, int(chunk_tiles), _stream_ptr(stream)))
+
+
+def bpt_ffn(o: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor,
+            chunk_tiles: int = 16) -> torch.Tensor:
+    """The feed-forward network on every token of an attention output o
+    [B,Hq,S,d], run blockwise (chunk_tiles query tiles at a time): y [B,S,Hq*d]."""
+    B, Hq, S, d = o.shape
+    y = torch.empty((B, S, Hq * d), device=o.device, dtype=torch.bfloat16)
+    ws = torch.empty(max(16, bpt_workspace_bytes(w1.shape[0], chunk_tiles)), dtype=torch.uint8,
+                     device=o.device)
+    fa_bpt_ffn(o, w1, w2, y, ws, chunk_tiles)
+    return y
+
+
+def bpt_layer(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, w1: torch.Tensor,
+              w2: torch.Tensor, causal: bool = False, scale: Optional[float] = None,
+              chunk_tiles: int = 16) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Attention (fa_fwd) followed by the blockwise feed-forward network:
+    returns (y [B,S,Hq*d], o, lse)."""
+    o, lse = flash_attention(q, k, v, causal=causal, scale=scale)
+    return bpt_ffn(o, w1, w2, chunk_tiles), o, lse
 
 
 def bwd_workspace_bytes(B: int, Hq: int, Sq: int, d: int) -> int:

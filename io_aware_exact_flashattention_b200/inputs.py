@@ -12,6 +12,8 @@ Recipe (fixed so that every caller sees the same tensors for a seed):
   * FP8 prefill: the same fp32 draws, each of Q, K, V scaled per (batch,
     key/value head) so its largest magnitude is 448 and rounded to E4M3
     (quantize_e4m3); the factors are returned beside the codes;
+  * feed-forward network after attention (ffn_inputs): o ~ N(0,1),
+    w1 ~ N(0,1)/sqrt(D), w2 ~ N(0,1)/sqrt(F), bf16, from seed + 15485863;
   * decode: per-sequence KV lengths ``randint(lmin, lmax + 1)`` drawn after
     K and V from the same generator; cache positions at or beyond a
     sequence's length are filled with ``pad_value`` (NaN by default) so that
@@ -227,6 +229,20 @@ def fp8_prefill_inputs(B: int, Hq: int, Hkv: int, Sq: int, Skv: int, d: int, see
 def fp8_prefill_inputs_for(shape: PrefillShape, device="cpu"):
     return fp8_prefill_inputs(shape.B, shape.Hq, shape.Hkv, shape.Sq, shape.Skv, shape.d,
                               shape.seed, shape.q_mult, device)
+
+
+def ffn_inputs(B: int, Hq: int, S: int, d: int, F: int, seed: int, device="cpu"):
+    """Inputs of the feed-forward network after attention, random stand-ins
+    for trained weights: o [B,Hq,S,d] ~ N(0,1) (an attention output's shape),
+    w1 [F, D] ~ N(0,1)/sqrt(D), w2 [D, F] ~ N(0,1)/sqrt(F) with D = Hq*d, all
+    rounded to bf16; drawn in that order from their own seed (seed + 15485863)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed) + 15485863)
+    D = Hq * d
+    o = torch.randn((B, Hq, S, d), generator=g, device=device, dtype=torch.float32)
+    w1 = torch.randn((F, D), generator=g, device=device, dtype=torch.float32) / D ** 0.5
+    w2 = torch.randn((D, F), generator=g, device=device, dtype=torch.float32) / F ** 0.5
+    return tuple(x.to(torch.bfloat16).contiguous() for x in (o, w1, w2))
 
 
 def grad_output(shape, seed: int, device="cpu"):

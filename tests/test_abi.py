@@ -178,6 +178,34 @@ def test_bwd_rejects_before_cuda(lib, kw, want):
     assert bwd(lib, **kw) == want
 
 
+def bpt(lib, *, o=A, w1=A, w2=A, y=A, ws=A, B=1, Hq=2, S=300, d=128, F=512, chunk=2):
+    return lib.fa_bpt_ffn(o, w1, w2, y, ws, B, Hq, S, d, F, chunk, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(d=96), UNSUPPORTED),
+    (dict(Hq=1), UNSUPPORTED),           # D = 128 is not a multiple of 256
+    (dict(F=300), UNSUPPORTED),
+    (dict(chunk=0), INVALID),
+    (dict(chunk=70000), UNSUPPORTED),
+    (dict(B=-1), INVALID),
+    (dict(S=-1), INVALID),
+    (dict(o=None), INVALID),
+    (dict(ws=None), INVALID),
+    (dict(y=A + 8), ALIGNMENT),
+    (dict(w2=A + 2), ALIGNMENT),
+    (dict(B=0, o=None), OK),
+    (dict(S=0, o=None), OK),
+])
+def test_bpt_ffn_rejects_before_cuda(lib, kw, want):
+    assert bpt(lib, **kw) == want
+
+
+def test_bpt_workspace_bytes(lib):
+    assert fa.bpt_workspace_bytes(512, 3) == 3 * 128 * 512 * 2
+    assert fa.bpt_workspace_bytes(0, 3) == 0
+
+
 def test_bwd_workspace_bytes(lib):
     assert fa.bwd_workspace_bytes(2, 4, 100, 128) == 2 * 4 * 100 * 129 * 4
     assert fa.bwd_workspace_bytes(0, 4, 100, 128) == 0

@@ -1,0 +1,118 @@
+"""fa_bpt_ffn (through the C ABI) against the fp64 oracle on a B200.
+
+The network's input is a seeded bf16 stand-in for an attention output, so the
+oracle's inputs never come from the CUDA path.  Per output element the bound
+follows from the arithmetic (bf16 inputs, fp32 accumulation, H and y rounded
+to bf16 once each):
+
+  2^-8 * (|H| |W2|^T)        H rounded to bf16 (half an ulp is 2^-9 relative)
+  + F * 2^-24 * (|H| |W2|^T)  fp32 accumulation of the second product
+  + 1.13 * K * 2^-24 * ((|x| |W1|^T) |W2|^T)
+                              fp32 accumulation of the first product, through
+                              GELU (slope at most 1.13) and W2
+  + 2^-8 * |y|                y rounded to bf16
+  + 1e-6
+
+with H the oracle's hidden activations.  Any misplaced head, token, column or
+chunk row moves y by about |y| and falls far outside it.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from io_aware_exact_flashattention_b200 import fa
+from io_aware_exact_flashattention_b200.inputs import ffn_inputs, prefill_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    fa.lib()
+
+
+def ffn_bound(x, w1, w2, h_ref, y_ref):
+    a1, a2 = np.abs(w1), np.abs(w2)
+    K, F = w1.shape[1], w1.shape[0]
+    hw = np.abs(h_ref) @ a2.T
+    return ((2.0 ** -8 + F * 2.0 ** -24) * hw
+            + 1.13 * K * 2.0 ** -24 * ((np.abs(x) @ a1.T) @ a2.T)
+            + 2.0 ** -8 * np.abs(y_ref) + 1e-6)
+
+
+def check_rows(y_got, x, w1, w2):
+    """y_got [n, D] (torch, any device) against the oracle on token rows x [n, D]."""
+    w1n, w2n = (w.double().numpy() for w in (w1, w2))
+    h_ref = oracle.ffn_hidden(x, w1n)
+    y_ref = oracle.ffn(x, w1n, w2n)
+    tol = ffn_bound(x, w1n, w2n, h_ref, y_ref)
+    got = y_got.float().cpu().numpy().astype(np.float64)
+    assert np.isfinite(got).all(), "non-finite y"
+    ratio = np.abs(got - y_ref) / tol
+    worst = np.unravel_index(int(np.argmax(ratio)), ratio.shape)
+    assert ratio.max() <= 1.0, ("y error over bound", worst, float(ratio.max()),
+                                float(got[worst]), float(y_ref[worst]))
+
+
+@pytest.mark.parametrize("B,Hq,S,d,F,chunk", [
+    (1, 2, 300, 128, 512, 2),     # ragged last tile, two chunks
+    (2, 4, 200, 64, 256, 1),      # two sequences, one tile per chunk
+    (1, 4, 128, 128, 768, 8),     # one full tile, F = 3 column tiles
+    (3, 2, 130, 128, 256, 3),     # tiles of three sequences in one chunk
+])
+def test_ffn_matches_oracle(B, Hq, S, d, F, chunk):
+    o, w1, w2 = ffn_inputs(B, Hq, S, d, F, seed=B * 100 + S)
+    y = fa.bpt_ffn(o.cuda(), w1.cuda(), w2.cuda(), chunk_tiles=chunk)
+    torch.cuda.synchronize()
+    x = oracle.heads_to_tokens(o).reshape(B * S, Hq * d)
+    check_rows(y.reshape(B * S, Hq * d), x, w1, w2)
+
+
+def test_chunking_changes_nothing():
+    """Each tile is computed the same way whatever chunk it falls in."""
+    o, w1, w2 = ffn_inputs(2, 2, 333, 128, 512, seed=7)
+    oc, w1c, w2c = o.cuda(), w1.cuda(), w2.cuda()
+    ys = [fa.bpt_ffn(oc, w1c, w2c, chunk_tiles=c) for c in (1, 2, 3, 100)]
+    torch.cuda.synchronize()
+    for y in ys[1:]:
+        assert torch.equal(y, ys[0])
+
+
+def test_layer_is_attention_then_ffn():
+    """bpt_layer = fa_fwd then the blockwise network, checked against the
+    oracle's layer.  The bound adds the attention's own error (|dO| <= 2e-2,
+    the forward's tolerance) carried through GELU and both maps."""
+    B, Hq, Hkv, S, d, F = 1, 2, 1, 300, 128, 512
+    q, k, v = prefill_inputs(B, Hq, Hkv, S, S, d, seed=9)
+    _, w1, w2 = ffn_inputs(B, Hq, S, d, F, seed=9)
+    scale = 1.0 / math.sqrt(d)
+    y, o, _ = fa.bpt_layer(q.cuda(), k.cuda(), v.cuda(), w1.cuda(), w2.cuda(), causal=True,
+                           scale=scale, chunk_tiles=2)
+    torch.cuda.synchronize()
+    assert torch.equal(y, fa.bpt_ffn(o, w1.cuda(), w2.cuda(), chunk_tiles=2))
+    y_ref, o_ref, _ = oracle.bpt_layer(q, k, v, w1, w2, True, scale)
+    x_ref = oracle.heads_to_tokens(o_ref).reshape(S, Hq * d)
+    w1n, w2n = (w.double().numpy() for w in (w1, w2))
+    tol = ffn_bound(x_ref, w1n, w2n, oracle.ffn_hidden(x_ref, w1n), y_ref.reshape(S, -1))
+    tol = tol + 1.13 * 2e-2 * (np.abs(w2n) @ (np.abs(w1n) @ np.ones(Hq * d)))[None, :]
+    got = y.reshape(S, -1).float().cpu().numpy()
+    assert (np.abs(got - y_ref.reshape(S, -1)) <= tol).all()
+
+
+def test_headline_shape_sampled_tokens():
+    """The bench's configuration: the causal S=2048 workload's attention
+    output shape (B=4, H=16, d=128: D=2048), F = 4 D = 8192, 16 query tiles
+    per chunk; 48 sampled tokens against the oracle."""
+    B, Hq, S, d, F = 4, 16, 2048, 128, 8192
+    o, w1, w2 = ffn_inputs(B, Hq, S, d, F, seed=2)
+    y = fa.bpt_ffn(o.cuda(), w1.cuda(), w2.cuda(), chunk_tiles=16)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(5)
+    toks = sorted(set(rng.integers(0, B * S, 44).tolist()) | {0, S - 1, S, B * S - 1})
+    x_all = oracle.heads_to_tokens(o).reshape(B * S, Hq * d)
+    check_rows(y.reshape(B * S, -1)[toks], x_all[toks], w1, w2)
