@@ -11,12 +11,19 @@ the one-shot, materialising softmax attention of "I/O-Aware Kernels", section
 "The Memory Bottleneck", with scores scaled as in "FlashAttention & IO-aware
 attention", section "Code", and LSE = max + ln(sum of exp).  A paged cache is
 read through its block table by ``paged_gather`` (plain index loops, no
-arithmetic) and then decoded like a contiguous one.
+arithmetic) and then decoded like a contiguous one.  E4M3 inputs are decoded
+from the format's definition and scaled per (batch, key/value head)
+(``e4m3_decode``, ``dequant_heads``, ``attn_fwd_fp8``).  The feed-forward
+network after attention of "I/O-Aware Kernels", section "Blockwise Parallel
+Transformers", is ``ffn`` / ``ffn_hidden`` on the head-concatenated tokens
+(``heads_to_tokens``); ``bpt_layer`` is attention followed by it.
 
 Parity pins (tests/test_oracle_pins.py): closed-form golden cases, an
 independent online-softmax recurrence, invariants, torch fp64 SDPA on small
 shapes, GQA/decode/split reductions, the E4M3 decoding by hand and against
-torch's float8 conversion, and the per-head dequantisation in closed form.
+torch's float8 conversion, the per-head dequantisation in closed form, and
+the feed-forward network against normal-CDF values, torch's fp64 GELU network
+and token independence.
 Every function here is pinned.
 """
 from __future__ import annotations
