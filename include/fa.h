@@ -20,6 +20,11 @@
  *    execution surfaces at the caller's next synchronisation.
  *  - Errors are returned, never printed and never trapped.  Argument checks
  *    run before any CUDA call; a call that fails them launches nothing.
+ *  - A kernel that gives up one of its bounded waits (see
+ *    fa_get_device_status) returns early: the outputs of that call are then
+ *    undefined (partly written, or holding what the buffers held before), and
+ *    only fa_get_device_status() tells.  Check it before trusting outputs of
+ *    a run in which anything went wrong.
  *  - Unsupported head sizes are rejected with FA_ERR_UNSUPPORTED: there is no
  *    slower fallback path ("FlashAttention & IO-aware attention", section
  *    "Interviewer follow-ups", warns that a silent fallback to a materialising
@@ -191,7 +196,10 @@ size_t fa_bpt_workspace_bytes(int F, int chunk_tiles);
  *   lse_partial[b,h,c] = ln sum over the chunk's keys of exp(scale * q.k)
  *
  * An empty chunk writes o_partial = 0 and lse_partial = -inf.  Cache
- * positions >= L_b are never read.
+ * positions >= L_b never contribute to any output, but they may be read:
+ * a chunk's last key tile is fetched in boxes of 32 rows, so up to 31 rows
+ * past the chunk's end (still inside the cache's Lmax rows) can be loaded
+ * and are then zeroed or masked on chip.
  *
  *   q            [B, Hq, d]           bf16
  *   k_cache,
@@ -276,6 +284,39 @@ fa_status fa_combine(const float *o_partial, const float *lse_partial, void *o,
  */
 int fa_decode_default_splits(int B, int Hkv, int Lmax, int num_sms);
 
+/*
+ * Host-only: partition of one fa_fwd / fa_bwd problem over n_shards devices
+ * or processes.  The work units are the B * Hkv (batch, key/value head)
+ * pairs in row-major order; a unit together with its Hq / Hkv query heads is
+ * an attention problem of its own (no query head reads another unit's keys),
+ * so the shards need no exchange of data: each computes its units' rows of
+ * o and lse, and the union of the shards is the whole result.
+ *
+ * Shard `shard` (0 <= shard < n_shards) gets units [*first, *first + *count):
+ * contiguous, in order, sizes differing by at most one (every unit has the
+ * same work).  In the [B * Hkv, Hq / Hkv, S, d] view of q and o and the
+ * [B * Hkv, 1, S, d] view of k and v, a shard is one contiguous slice, i.e.
+ * one fa_fwd call with B' = *count, Hq' = Hq / Hkv, Hkv' = 1.  A shard may be
+ * empty (*count = 0) when n_shards > B * Hkv.
+ * Errors: FA_ERR_INVALID_ARG for B, Hkv, n_shards < 1, shard out of range or
+ * null outputs.  first and count are host pointers.
+ */
+fa_status fa_shard_units(int B, int Hkv, int n_shards, int shard, int *first, int *count);
+
+/*
+ * Host-only: partition of a decode batch over n_shards devices or processes.
+ * Sequences are independent problems; shard s gets sequences
+ * [bounds[s], bounds[s+1]), contiguous and in order, chosen so that the
+ * shards' key counts (sum of max(L_b, 1) over their sequences, the decode's
+ * work) are as even as a contiguous split allows: bounds[s] is the smallest
+ * b' such that sequences [0, b') hold at least s / n_shards of the total.
+ *   seqlens_k  [B] int32, HOST memory (values < 0 count as 0)
+ *   bounds     [n_shards + 1] int32, HOST memory (written; bounds[0] = 0,
+ *              bounds[n_shards] = B, non-decreasing)
+ * Errors: FA_ERR_INVALID_ARG for B < 1, n_shards < 1 or null pointers.
+ */
+fa_status fa_shard_sequences(const int32_t *seqlens_k, int B, int n_shards, int32_t *bounds);
+
 /* Host-only: a static, human-readable name for a status code. */
 const char *fa_status_string(fa_status s);
 
@@ -319,15 +360,21 @@ fa_status fa_debug_exp2_poly(const float *x, float *y, int n, fa_stream_t stream
  * can synchronise the device and stall all of its streams.
  *
  * Limits and behaviour:
- *  - The array is 32 MiB on every device that loads libfa.so, held until the
- *    process exits.  The partials need B*Hq*num_splits*d*4 bytes, rounded up
- *    to 256, plus B*Hq*num_splits*4; a call that needs more returns
- *    FA_ERR_UNSUPPORTED before any CUDA call (use fewer splits, or
- *    fa_decode_splitkv with a caller buffer).
+ *  - The array is FA_DECODE_NOALLOC_BYTES (32 MiB) on every device that loads
+ *    libfa.so, held until the process exits.  The partials need
+ *    B*Hq*num_splits*d*4 bytes, rounded up to 256, plus B*Hq*num_splits*4; a
+ *    call that needs more returns FA_ERR_UNSUPPORTED before any CUDA call
+ *    (use fewer splits, or fa_decode_splitkv with a caller buffer).
  *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current) and keeps it; make that
- *    first call before any stream capture.  No call allocates device or host
+ *    (cudaGetSymbolAddress, with that device current) and keeps it for the
+ *    life of the process; make that first call before any stream capture.
+ *    The kept address belongs to the device's primary context: after
+ *    cudaDeviceReset, or with another context current on that device, it is
+ *    stale and this call must not be used.  No call allocates device or host
  *    memory: no cudaMalloc, no cudaFree, no allocating library routine.
+ *  - If the split kernel gives up a bounded wait, the merge may combine the
+ *    previous call's partials still held in the array, so o and lse are
+ *    undefined unless fa_get_device_status() returns FA_OK.
  *  - All calls on a device share the one array, which keeps the previous
  *    call's partials.  Calls whose kernels overlap on the GPU (other streams,
  *    other host threads) race on it; order them on one stream.  Nothing in it
@@ -335,6 +382,9 @@ fa_status fa_debug_exp2_poly(const float *x, float *y, int n, fa_stream_t stream
  *  - Supported shapes and the other errors are those of fa_decode_splitkv and
  *    fa_combine.
  */
+/* Size in bytes of fa_decode_noalloc's fixed partials array, per device. */
+#define FA_DECODE_NOALLOC_BYTES (32u << 20)
+
 fa_status fa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
                             const int32_t *seqlens_k, void *o, float *lse, int B, int Hq,
                             int Hkv, int Lmax, int d, int num_splits, float scale,

@@ -331,11 +331,11 @@ __global__ void timeout_probe_kernel(unsigned long long limit_ns) {
 // ---------------------------------------------------------------------------
 // Fixed, library-owned scratch for fa_decode_noalloc.
 // ---------------------------------------------------------------------------
-// 32 MiB on every device that loads this library, held until the process
-// exits.  The name is only a host-side stand-in: host code obtains the
+// FA_DECODE_NOALLOC_BYTES (32 MiB) on every device that loads this library,
+// held until the process exits.  The name is only a host-side stand-in: host code obtains the
 // device address with cudaGetSymbolAddress (once per device, that device
 // current) and passes that address to the kernels.
-constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(32) << 20;
+constexpr size_t kNoAllocScratchBytes = FA_DECODE_NOALLOC_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 std::mutex g_noalloc_mu;
@@ -733,6 +733,36 @@ int fa_decode_default_splits(int B, int Hkv, int Lmax, int num_sms) {
   if (n < 1) n = 1;
   if (n > 256) n = 256;
   return static_cast<int>(n);
+}
+
+fa_status fa_shard_units(int B, int Hkv, int n_shards, int shard, int* first, int* count) {
+  if (B < 1 || Hkv < 1 || n_shards < 1 || shard < 0 || shard >= n_shards || first == nullptr ||
+      count == nullptr)
+    return FA_ERR_INVALID_ARG;
+  const long long units = static_cast<long long>(B) * Hkv;
+  const long long a = units * shard / n_shards, b = units * (shard + 1) / n_shards;
+  *first = static_cast<int>(a);
+  *count = static_cast<int>(b - a);
+  return FA_OK;
+}
+
+fa_status fa_shard_sequences(const int32_t* seqlens_k, int B, int n_shards, int32_t* bounds) {
+  if (B < 1 || n_shards < 1 || seqlens_k == nullptr || bounds == nullptr)
+    return FA_ERR_INVALID_ARG;
+  long long total = 0;
+  for (int b = 0; b < B; ++b) total += std::max(seqlens_k[b], 1);
+  // bounds[s] = smallest b' whose prefix [0, b') holds at least s/n of the
+  // total; prefix counts are non-decreasing, so the bounds are too.
+  long long run = 0;
+  int s = 1;
+  bounds[0] = 0;
+  for (int b = 0; b < B && s < n_shards; ++b) {
+    run += std::max(seqlens_k[b], 1);
+    while (s < n_shards && run * n_shards >= total * s) bounds[s++] = b + 1;
+  }
+  while (s < n_shards) bounds[s++] = B;
+  bounds[n_shards] = B;
+  return FA_OK;
 }
 
 const char* fa_status_string(fa_status s) {

@@ -46,6 +46,9 @@ SIGNATURES = {
     "fa_debug_timeout_probe": (_I, [ctypes.c_uint, _VP]),
     "fa_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP]),
     "fa_debug_exp2_poly": (_I, [_VP, _VP, _I, _VP]),
+    "fa_shard_units": (_I, [_I, _I, _I, _I, ctypes.POINTER(ctypes.c_int),
+                            ctypes.POINTER(ctypes.c_int)]),
+    "fa_shard_sequences": (_I, [_VP, _I, _I, _VP]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -481,4 +484,131 @@ def decode_attention_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torc
     o = torch.empty((B, Hq, d), device=q.device, dtype=torch.bfloat16)
     lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32)
     fa_combine(o_part, lse_part, o, lse)
+    return o, lse
+
+
+# ---------------------------------------------------------------------------
+# Sharding one problem over several devices (or processes): no data exchange
+# ---------------------------------------------------------------------------
+
+def shard_units(B: int, Hkv: int, n_shards: int, shard: int) -> Tuple[int, int]:
+    """(first, count): the shard's range of (batch, key/value head) units in
+    row-major order (fa_shard_units)."""
+    first, count = ctypes.c_int(0), ctypes.c_int(0)
+    _check("fa_shard_units", lib().fa_shard_units(int(B), int(Hkv), int(n_shards), int(shard),
+                                                  ctypes.byref(first), ctypes.byref(count)))
+    return first.value, count.value
+
+
+def shard_sequences(seqlens_k, n_shards: int) -> list:
+    """Bounds [n_shards + 1] of a contiguous, work-balanced split of a decode
+    batch (fa_shard_sequences); seqlens_k on any device or a sequence."""
+    import numpy as np
+    sl = np.ascontiguousarray(np.asarray(seqlens_k.cpu().numpy() if hasattr(seqlens_k, "cpu")
+                                         else seqlens_k, dtype=np.int32))
+    bounds = np.zeros(int(n_shards) + 1, dtype=np.int32)
+    _check("fa_shard_sequences", lib().fa_shard_sequences(sl.ctypes.data, int(sl.size),
+                                                          int(n_shards), bounds.ctypes.data))
+    return [int(x) for x in bounds]
+
+
+def unit_views(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor):
+    """q [B,Hq,S,d], k/v [B,Hkv,S,d] as [B*Hkv, Hq/Hkv, S, d] and
+    [B*Hkv, 1, S, d] views: a range of rows of these views is one unit range,
+    an fa_fwd problem of its own."""
+    B, Hq, Sq, d = q.shape
+    _, Hkv, Skv, _ = k.shape
+    if Hkv < 1 or Hq % Hkv != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    G = Hq // Hkv
+    return (q.reshape(B * Hkv, G, Sq, d), k.reshape(B * Hkv, 1, Skv, d),
+            v.reshape(B * Hkv, 1, Skv, d))
+
+
+def flash_attention_sharded(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                            causal: bool = False, scale: Optional[float] = None,
+                            devices: Optional[list] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """One attention problem split over `devices` (default: every visible CUDA
+    device) by (batch, key/value head) units, without any collective: shard s
+    copies its units' q, k, v to device s, runs fa_fwd there on a stream of its
+    own, and copies its rows of o and lse back into outputs that live where q
+    lives (host or device).  Returns (o, lse) after every shard has finished.
+    The result is bit-identical to one fa_fwd call on the whole problem."""
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    if devices is None:
+        devices = [torch.device("cuda", i) for i in range(torch.cuda.device_count())]
+    devices = [torch.device(d) for d in devices]
+    if not devices:
+        raise RuntimeError("no CUDA device to shard over")
+    B, Hq, Sq, d = q.shape
+    _, Hkv, _, _ = k.shape
+    qv, kv, vv = unit_views(q, k, v)
+    pin = not q.is_cuda
+    o = torch.empty(q.shape, dtype=q.dtype, device=q.device, pin_memory=pin)
+    lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device, pin_memory=pin)
+    ov, lv = o.view(qv.shape), lse.view(qv.shape[:3])
+    pending = []
+    for s, dev in enumerate(devices):
+        a, n = shard_units(B, Hkv, len(devices), s)
+        if n == 0:
+            continue
+        with torch.cuda.device(dev):
+            stream = torch.cuda.Stream(dev)
+            stream.wait_stream(torch.cuda.current_stream(dev))
+            if q.is_cuda:
+                stream.wait_stream(torch.cuda.current_stream(q.device))
+            with torch.cuda.stream(stream):
+                qs, ks, vs = (t[a:a + n].to(dev, non_blocking=True) for t in (qv, kv, vv))
+                os_ = torch.empty(qs.shape, dtype=q.dtype, device=dev)
+                ls_ = torch.empty(qs.shape[:3], dtype=torch.float32, device=dev)
+                fa_fwd(qs, ks, vs, os_, ls_, causal, scale, stream=stream)
+                ov[a:a + n].copy_(os_, non_blocking=True)
+                lv[a:a + n].copy_(ls_, non_blocking=True)
+            pending.append((stream, (qs, ks, vs, os_, ls_)))
+    for stream, bufs in pending:
+        stream.synchronize()
+    return o, lse
+
+
+def decode_attention_sharded(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                             seqlens_k: torch.Tensor, scale: Optional[float] = None,
+                             devices: Optional[list] = None,
+                             num_splits: Optional[int] = None
+                             ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Single-query decode with the batch split over `devices` by sequences
+    (fa_shard_sequences, balanced by key count), without any collective: each
+    device decodes its sequences (split-KV + merge) on a stream of its own and
+    its rows of o and lse are copied back to where q lives."""
+    if devices is None:
+        devices = [torch.device("cuda", i) for i in range(torch.cuda.device_count())]
+    devices = [torch.device(d) for d in devices]
+    if not devices:
+        raise RuntimeError("no CUDA device to shard over")
+    B, Hq, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    bounds = shard_sequences(seqlens_k, len(devices))
+    pin = not q.is_cuda
+    o = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device, pin_memory=pin)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device, pin_memory=pin)
+    pending = []
+    for s, dev in enumerate(devices):
+        a, b = bounds[s], bounds[s + 1]
+        if a == b:
+            continue
+        with torch.cuda.device(dev):
+            stream = torch.cuda.Stream(dev)
+            stream.wait_stream(torch.cuda.current_stream(dev))
+            if q.is_cuda:
+                stream.wait_stream(torch.cuda.current_stream(q.device))
+            with torch.cuda.stream(stream):
+                qs, ks, vs, ss = (t[a:b].to(dev, non_blocking=True)
+                                  for t in (q, k_cache, v_cache, seqlens_k))
+                os_, ls_ = decode_attention(qs, ks, vs, ss, scale, num_splits)
+                o[a:b].copy_(os_, non_blocking=True)
+                lse[a:b].copy_(ls_, non_blocking=True)
+            pending.append((stream, (qs, ks, vs, ss, os_, ls_)))
+    for stream, bufs in pending:
+        stream.synchronize()
     return o, lse

@@ -104,15 +104,20 @@ def test_layer_is_attention_then_ffn():
     assert (np.abs(got - y_ref.reshape(S, -1)) <= tol).all()
 
 
-def test_headline_shape_sampled_tokens():
+def test_headline_shape_every_tile():
     """The bench's configuration: the causal S=2048 workload's attention
     output shape (B=4, H=16, d=128: D=2048), F = 4 D = 8192, 16 query tiles
-    per chunk; 48 sampled tokens against the oracle."""
+    per chunk; the first, the last and two random tokens of every 128-token
+    tile (so every tile of every chunk) against the oracle."""
     B, Hq, S, d, F = 4, 16, 2048, 128, 8192
     o, w1, w2 = ffn_inputs(B, Hq, S, d, F, seed=2)
     y = fa.bpt_ffn(o.cuda(), w1.cuda(), w2.cuda(), chunk_tiles=16)
     torch.cuda.synchronize()
     rng = np.random.default_rng(5)
-    toks = sorted(set(rng.integers(0, B * S, 44).tolist()) | {0, S - 1, S, B * S - 1})
+    toks = set()
+    for t0 in range(0, B * S, 128):
+        toks.update({t0, t0 + 127})
+        toks.update(int(x) for x in rng.integers(t0, t0 + 128, 2))
+    toks = sorted(toks)
     x_all = oracle.heads_to_tokens(o).reshape(B * S, Hq * d)
     check_rows(y.reshape(B * S, -1)[toks], x_all[toks], w1, w2)

@@ -116,10 +116,10 @@ def test_decode_equals_prefill_row():
     assert float((lse - l2[:, :, 0]).abs().max()) <= 2 * LSE_TOL
 
 
-def test_full_size_decode_config_sampled():
+def test_full_size_decode_config_every_sequence():
     """The full decode workload (B=64, Hq=32, Hkv=8, L in [4096, 16384], d=128)
-    in the launch the benchmark times; every sequence's output is checked for
-    finiteness and 8 sequences element-wise against the oracle."""
+    in the launch the benchmark times; every sequence and head element-wise
+    against the oracle (one oracle call per sequence, on its L_b keys)."""
     c = CONFIGS["decode_b64_splitkv_d128"]
     q, kc, vc, sl = decode_inputs_for(c, device="cuda")
     sms = torch.cuda.get_device_properties(0).multi_processor_count
@@ -127,8 +127,7 @@ def test_full_size_decode_config_sampled():
     _, _, o, lse = run_decode(q, kc, vc, sl, c.scale, n)
     assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
     lens = sl.cpu().tolist()
-    pick = sorted({0, c.B - 1, int(np.argmin(lens)), int(np.argmax(lens)), 7, 21, 33, 50})
-    for b in pick:
+    for b in range(c.B):
         L = lens[b]
         o_ref, lse_ref = oracle.decode(q[b:b + 1], kc[b:b + 1, :, :L], vc[b:b + 1, :, :L],
                                        np.array([L], np.int32), c.scale)

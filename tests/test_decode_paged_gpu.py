@@ -143,17 +143,18 @@ def test_paged_equals_contiguous_cache():
     assert float((l1 - l2).abs().max()) <= LSE_TOL
 
 
-def test_full_size_workload_sampled():
+def test_full_size_workload_every_sequence():
     """The decode workload (B=64, Hq=32, Hkv=8, d=128, L ~ U{4096..16384}) in
-    16-key pages, launched as the bench launches it; sampled sequences are
-    checked against the oracle."""
+    16-key pages, launched as the bench launches it; every sequence and head
+    against the oracle on the gathered pages."""
     c = CONFIGS["decode_b64_splitkv_d128"]
     q, kp, vp, bt, sl = paged_decode_inputs(c.B, c.Hq, c.Hkv, c.Lmin, c.Lmax, c.d, c.seed,
                                             page_size=16, device="cuda")
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     n = fa.decode_default_splits(c.B, c.Hkv, c.Lmax, sms)
     op, lp, o, lse = run_paged(q, kp, vp, bt, sl, c.scale, n)
-    for b in (0, 17, 40, 63):
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    for b in range(c.B):
         L = int(sl[b])
         pages = bt[b, :(L + 15) // 16].long()
         kg = kp[pages].permute(1, 0, 2, 3).reshape(c.Hkv, -1, c.d)[:, :L].cpu()

@@ -196,38 +196,92 @@ def test_host_buffers_in_chunks_equal_device_call(chunks):
     assert torch.equal(o_h, o_dev.cpu()) and torch.equal(lse_h, lse_dev.cpu())
 
 
-def sample_rows(B, Hq, Sq, n, seed):
-    rng = np.random.default_rng(seed)
-    rows = {(0, 0, 0), (B - 1, Hq - 1, Sq - 1), (0, Hq - 1, 127), (B - 1, 0, 128),
-            (0, 0, Sq // 2), (B - 1, Hq // 2, 255), (0, 1 % Hq, 256)}
-    while len(rows) < n:
-        rows.add((int(rng.integers(B)), int(rng.integers(Hq)), int(rng.integers(Sq))))
+def tile_rows(Sq, per_tile, rng):
+    """`per_tile` query rows drawn from every 128-row tile (the tile's first
+    and last rows always among them), so every tile of a head is checked."""
+    rows = set()
+    for t0 in range(0, Sq, 128):
+        t1 = min(Sq, t0 + 128)
+        rows.update({t0, t1 - 1})
+        rows.update(int(x) for x in rng.integers(t0, t1, max(0, per_tile - 2)))
     return sorted(rows)
 
 
-@pytest.mark.parametrize("name", ["causal_mha_s2048_d128_qx8", "causal_gqa_s8192_d128",
-                                  "causal_gqa_s32768_d128"])
-def test_full_size_config_sampled(name):
-    """The full-size workload in the same launch the benchmark times, checked
-    element-wise at sampled rows and by properties over every row."""
+def full_size_run(name):
+    """The full-size workload in the launch the benchmark times, with the
+    properties that hold at any size checked on every row: finite, and each O
+    row inside the value range of its head."""
     c = CONFIGS[name]
     q, k, v = prefill_inputs_for(c, device="cuda")
     o, lse = run_fa(q, k, v, c.causal, c.scale)
     torch.cuda.synchronize()
-    # properties over all rows: finite, and each O row lies in the value range of its head
     assert torch.isfinite(o).all() and torch.isfinite(lse).all()
     grp = c.Hq // c.Hkv
     vmax = v.float().amax(dim=2).repeat_interleave(grp, dim=1)  # [B,Hq,d]
     vmin = v.float().amin(dim=2).repeat_interleave(grp, dim=1)
     of = o.float()
     assert (of <= vmax[:, :, None, :] + O_TOL).all() and (of >= vmin[:, :, None, :] - O_TOL).all()
-    rows = sample_rows(c.B, c.Hq, c.Sq, 48, seed=c.seed)
-    qr = torch.stack([q[b, h, i] for (b, h, i) in rows]).cpu()
-    o_ref, lse_ref = oracle.attn_rows(qr, k.cpu(), v.cpu(), rows, c.Hq, c.Sq, c.causal, c.scale)
-    o_got = torch.stack([o[b, h, i] for (b, h, i) in rows]).float().cpu().numpy()
-    l_got = torch.stack([lse[b, h, i] for (b, h, i) in rows]).cpu().numpy()
-    assert float(np.abs(o_got - o_ref).max()) <= O_TOL
-    assert float(np.abs(l_got - lse_ref).max()) <= LSE_TOL
+    return c, q, k, v, o, lse
+
+
+def check_whole_head(c, q, k, v, o, lse, b, h):
+    g = h // (c.Hq // c.Hkv)
+    o_ref, lse_ref = oracle.attn_fwd(q[b:b + 1, h:h + 1].cpu(), k[b:b + 1, g:g + 1].cpu(),
+                                     v[b:b + 1, g:g + 1].cpu(), c.causal, c.scale)
+    eo, el = errors(o[b:b + 1, h:h + 1], lse[b:b + 1, h:h + 1], o_ref, lse_ref)
+    assert eo <= O_TOL and el <= LSE_TOL, ("head", b, h, eo, el)
+
+
+def check_tile_rows(c, q, k, v, o, lse, per_tile, seed):
+    """`per_tile` rows of every 128-row tile of every (b, head), one oracle
+    call per key/value head (the oracle reads only that head's keys)."""
+    rng = np.random.default_rng(seed)
+    grp = c.Hq // c.Hkv
+    for b in range(c.B):
+        for g in range(c.Hkv):
+            kb, vb = k[b:b + 1, g:g + 1].cpu(), v[b:b + 1, g:g + 1].cpu()
+            rows = [(0, j, i) for j in range(grp) for i in tile_rows(c.Sq, per_tile, rng)]
+            hs = torch.tensor([g * grp + j for (_, j, _) in rows], device=q.device)
+            ii = torch.tensor([i for (_, _, i) in rows], device=q.device)
+            qr = q[b][hs, ii].cpu()
+            o_ref, lse_ref = oracle.attn_rows(qr, kb, vb, rows, grp, c.Sq, c.causal, c.scale)
+            o_got = o[b][hs, ii].float().cpu()
+            l_got = lse[b][hs, ii].cpu()
+            eo = float(np.abs(o_got.numpy() - o_ref).max())
+            el = float(np.abs(l_got.numpy() - lse_ref).max())
+            assert eo <= O_TOL and el <= LSE_TOL, ("tile rows", b, g, eo, el)
+
+
+def test_full_size_causal_mha_s2048_every_row():
+    """Causal MHA B=4 H=16 S=2048 d=128, Q ~ N(0,1)*8: every row of every head
+    against the oracle (about a second of fp64 work on the host)."""
+    c, q, k, v, o, lse = full_size_run("causal_mha_s2048_d128_qx8")
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, c.causal, c.scale)
+    eo, el = errors(o, lse, o_ref, lse_ref)
+    assert eo <= O_TOL and el <= LSE_TOL, (eo, el)
+
+
+def test_full_size_causal_gqa_s8192():
+    """Causal GQA B=2 Hq=32 Hkv=8 S=8192 d=128: one whole query head of every
+    (batch, key/value head) pair, and 4 rows of every 128-row tile of every
+    query head."""
+    c, q, k, v, o, lse = full_size_run("causal_gqa_s8192_d128")
+    grp = c.Hq // c.Hkv
+    for b in range(c.B):
+        for g in range(c.Hkv):
+            check_whole_head(c, q, k, v, o, lse, b, g * grp + (g + b) % grp)
+    check_tile_rows(c, q, k, v, o, lse, 4, seed=c.seed)
+
+
+def test_full_size_causal_gqa_s32768():
+    """Causal GQA B=1 Hq=32 Hkv=8 S=32768 d=128 (the persistent scheduler's
+    last round of items holds the first query tiles of the last heads): the
+    first query head of key/value head 0 and the last query head of key/value
+    head 7 whole, and 4 rows of every 128-row tile of every query head."""
+    c, q, k, v, o, lse = full_size_run("causal_gqa_s32768_d128")
+    check_whole_head(c, q, k, v, o, lse, 0, 0)
+    check_whole_head(c, q, k, v, o, lse, 0, c.Hq - 1)
+    check_tile_rows(c, q, k, v, o, lse, 4, seed=c.seed)
 
 
 def test_timeout_probe_reports_and_context_survives():
