@@ -85,6 +85,8 @@ def parse_args():
                     help="workload of the backward, E4M3 and feed-forward measurements")
     ap.add_argument("--bpt-chunk", type=int, default=16,
                     help="query tiles per chunk of the blockwise feed-forward network")
+    ap.add_argument("--bpt-layer-chunk", type=int, default=4,
+                    help="query tiles per sequence per chunk of the blockwise layer")
     ap.add_argument("--page-size", type=int, default=16,
                     help="page size of the paged-cache decode measurement")
     return ap.parse_args()
@@ -624,7 +626,33 @@ def measure_extras(args, world, rank, dev, stream, flush, peaks, do_pre, do_dec,
                 gpu_launches=2 * n_chunks * K,
                 traffic_main_kernel=profiled_traffic("ffn:" + ce.name),
                 note="y = W2 gelu(W1 x_t) on the forward's output; measured outside the step")
-            del y, ws, w1, w2
+            # The blockwise layer: attention then the network, chunk by chunk.
+            lchunk = max(1, args.bpt_layer_chunk)
+            lse_l = torch.empty_like(lse)
+            wsl = torch.empty(max(16, fa.bpt_layer_workspace_bytes(ce.B, ce.Hq, ce.d, F, lchunk)),
+                              dtype=torch.uint8, device=dev)
+            lay_ms = timed_calls(lambda: fa.fa_bpt_layer(q, k, v, w1, w2, y, lse_l, wsl,
+                                                         ce.causal, ce.scale, lchunk,
+                                                         stream=stream),
+                                 K, args.warmup, flush, stream, world)
+            lay_flops = flops + ffn_flops
+            lay_tf = lay_flops / (lay_ms * 1e-3 / K) / 1e12
+            n_chunks_l = (((ce.Sq + 127) // 128) + lchunk - 1) // lchunk
+            out["bpt_layer"] = dict(
+                {"value": aggregate_rate(world, lay_flops, K, lay_ms) / 1e12, "unit": "TFLOP/s",
+                 "workload": ce.name, "ms_per_call": lay_ms / K},
+                **tensor_fracs(lay_tf, peaks),
+                algorithmic="%.4g FLOP per call (attention %.4g + network %.4g)"
+                            % (lay_flops, flops, ffn_flops),
+                chunk_tiles_per_sequence=lchunk,
+                workspace_bytes=fa.bpt_layer_workspace_bytes(ce.B, ce.Hq, ce.d, F, lchunk),
+                unblocked_activation_bytes=ce.B * ce.Sq * (D + F) * 2,
+                kernels="per chunk: fa_prefill_kernel<128> (query-tile range) + two "
+                        "fa_ffn_gemm_kernel",
+                gpu_launches=3 * n_chunks_l * K,
+                note="attention and network block by block; only one chunk's attention output "
+                     "and hidden activations exist at a time; measured outside the step")
+            del y, ws, w1, w2, wsl, lse_l
         del q, k, v, o, lse
 
     if do_dec and not args.no_paged:

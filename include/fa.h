@@ -185,6 +185,45 @@ fa_status fa_bpt_ffn(const void *o, const void *w1, const void *w2, void *y, voi
 size_t fa_bpt_workspace_bytes(int F, int chunk_tiles);
 
 /*
+ * fa_bpt_layer -- attention and the feed-forward network after it, run block
+ * by block ("I/O-Aware Kernels", section "Blockwise Parallel Transformers":
+ * a block of query rows goes through the network as soon as its attention
+ * output exists, so no sequence-wide activation is ever materialised).
+ *
+ * For each chunk of chunk_tiles query tiles (rows [c*R, c*R + R) of every
+ * sequence and head, R = chunk_tiles * 128), in order:
+ *   1. the attention of those rows (as fa_fwd computes them) into a chunk
+ *      buffer of the workspace, their LSE into lse;
+ *   2. H = gelu(X W1^T) of the chunk's tokens into the workspace;
+ *   3. y at those tokens = H W2^T.
+ * So the attention output and the F-wide activations exist for one chunk at a
+ * time: the workspace is B*Hq*R*d + B*R*F bf16 values, against B*S*Hq*d +
+ * B*S*F when the attention runs over the whole sequence first.
+ *
+ *   q [B,Hq,S,d], k, v [B,Hkv,S,d] bf16 (self-attention: Sq = Skv = S)
+ *   w1 [F, D], w2 [D, F] bf16 with D = Hq*d (as fa_bpt_ffn)
+ *   y  [B, S, D] bf16 (written: the network's output per token)
+ *   lse [B, Hq, S] fp32 (written: the attention's LSE, as fa_fwd)
+ *   workspace  fa_bpt_layer_workspace_bytes(B, Hq, d, F, chunk_tiles) bytes,
+ *              caller-owned scratch; contents on entry do not matter
+ *   causal, scale: as for fa_fwd.  chunk_tiles >= 1 (larger than the
+ *              sequence's tile count means one chunk).
+ *
+ * y equals fa_bpt_ffn applied to fa_fwd's output, bit for bit: every query
+ * tile's attention and every token's network are computed by the same
+ * kernels with the same arithmetic whatever the chunking.
+ * Supported: d in {64, 128}; D and F multiples of 256; B * chunk_tiles
+ * <= 65535.  Pointers 16-byte aligned.  Errors as for fa_fwd and fa_bpt_ffn.
+ */
+fa_status fa_bpt_layer(const void *q, const void *k, const void *v, const void *w1,
+                       const void *w2, void *y, float *lse, void *workspace, int B, int Hq,
+                       int Hkv, int S, int d, int F, int causal, float scale, int chunk_tiles,
+                       fa_stream_t stream);
+
+/* Bytes of scratch fa_bpt_layer needs (0 for invalid sizes). */
+size_t fa_bpt_layer_workspace_bytes(int B, int Hq, int d, int F, int chunk_tiles);
+
+/*
  * fa_decode_splitkv -- first half of single-query decode (Sq = 1, no mask).
  *
  * The key/value length L_b = seqlens_k[b] of sequence b is cut into
@@ -245,9 +284,8 @@ fa_status fa_decode_splitkv(const void *q, const void *k_cache, const void *v_ca
  * (key tiles then start on tile boundaries and never straddle pages).  Chunks
  * past L_b are empty (o_partial = 0, lse_partial = -inf); fa_combine merges
  * the partials exactly as for the contiguous cache.  Rows of a page past L_b
- * may be read but never contribute.  An out-of-range page index reads zeros
- * or another page (never outside the cache), so the result is then
- * meaningless but memory stays safe.
+ * are never read.  An out-of-range page index is clamped to [0, num_pages),
+ * so the result is then meaningless but every read stays inside the pool.
  *
  * Supported: page_size a power of two in [16, 256]; d in {64, 128};
  * Hq / Hkv in {1, 2, 4, 8}; 1 <= num_splits <= 256.  Errors as for

@@ -26,9 +26,9 @@
 // sequence; paged KV management is named in "I/O-Aware Kernels", section
 // "FlashAttention") changes only the producer: chunks start on multiples of
 // 128 keys, so a tile covers whole pages (page_size <= 128) or lies inside
-// one, and it is loaded as boxes of min(page_size, 128) rows (min(page_size,
-// 32) for a chunk's last tile), each from the physical page the block table
-// names.  The MMA and softmax roles see the same shared-memory tiles.
+// one, and the producer warp copies it row by row (16-byte cp.async) from the
+// physical pages the block table names into the same swizzled layout TMA
+// would write.  The MMA and softmax roles see the same shared-memory tiles.
 //   warp  5    MMA issuer
 // The online softmax keeps a per-head reference max m that only moves when
 // the max grows by more than 2^8; exp2 on scores times scale*log2(e).
@@ -44,6 +44,10 @@ constexpr int kDecNPad = 16;      // head columns of S^T / O^T (G real, rest zer
 constexpr int kDecSubRows = 32;   // rows per box of a chunk's last tile
 constexpr int kDecThreads = 192;
 constexpr int kDecMaxPagesPerTile = kDecBN / 16;  // pages of the smallest size in a tile
+// A paged cache is copied row by row with 16-byte cp.async; a tile's full
+// barrier is signalled once the copies of the tile kDecCpLag loads later are
+// issued, so this many tiles per lane are in flight.
+constexpr int kDecCpLag = 3;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kDecRescaleThreshold = 8.0f;  // log2 units
 
@@ -91,10 +95,11 @@ struct DecodeParams {
   unsigned long long wait_limit_ns;
   // paged cache (block_table == nullptr: contiguous [B, Hkv, Lmax, d] cache)
   const int* block_table;  // [B, max_pages]
+  const char* k_pool;      // [num_pages, Hkv, page_size, d] bf16
+  const char* v_pool;
+  int num_pages;           // page indices are clamped to [0, num_pages)
   int max_pages;
   int page_shift;          // log2(page_size)
-  int rows_main;           // rows per box of a full tile: min(page_size, 128)
-  int rows_tail;           // rows per box of a chunk's last tile: min(page_size, 32)
   int chunk_align;         // chunk sizes are rounded up to a multiple of this
 };
 
@@ -117,11 +122,32 @@ __device__ __forceinline__ void decode_item(const DecodeParams& p, int item, int
   b = bg / p.Hkv;
 }
 
+// 16-byte asynchronous copy global -> shared through L2; src_bytes < 16
+// fills the rest of the 16 bytes with zeros (src_bytes = 0 reads nothing).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ---------------------------------------------------------------------------
-// TMA producer (one warp).  Lane 0 waits for buffers, accounts the bytes and
-// issues the query loads and the contiguous-cache tile loads; for a paged
-// cache a tile is many small boxes (two per page of 16 rows at d=128), and
-// each lane issues one of them so their issue costs overlap.
+// Producer (one warp).  Lane 0 waits for buffers, accounts the bytes and
+// issues the query loads (TMA) and the contiguous-cache tile loads (TMA, one
+// 128-row box per 64-column block).  A paged cache is not loaded by TMA: its
+// pages are scattered, and a page of 16 keys would be two 2 KB boxes, whose
+// per-box cost caps the stream.  Instead all 32 lanes copy each tile row by
+// row with 16-byte cp.async straight into the 128B-swizzled layout the MMA
+// reads (chunk c of row r lands at chunk position c ^ (r & 7)), rows past the
+// chunk filled with zeros by the copy itself, so no cache row past L_b is
+// read.  Each lane waits for its own copies kDecCpLag tile loads later, makes
+// them visible to the tensor cores (proxy fence) and arrives on the tile's
+// full barrier (32 arrivals per tile).
 // ---------------------------------------------------------------------------
 template <int D, int G>
 __device__ __forceinline__ void decode_producer(const CUtensorMap* tk, const CUtensorMap* tv,
@@ -149,6 +175,18 @@ __device__ __forceinline__ void decode_producer(const CUtensorMap* tk, const CUt
     return __shfl_sync(mask, ok ? 1 : 0, 0) != 0;
   };
   uint32_t ld = 0;  // K/V tile loads issued
+  uint32_t npend = 0;  // paged: loads issued whose full barrier this lane has not yet signalled
+  // paged: wait for this lane's oldest pending copies and signal their tile
+  auto retire_oldest = [&]() {
+    const uint32_t k = ld - npend;
+    fence_proxy_async_smem();
+    mbar_arrive(bars + 8 * (L::kBKvFull + k % static_cast<uint32_t>(L::kStages)));
+    --npend;
+  };
+  auto retire_all = [&]() {
+    cp_async_wait<0>();
+    while (npend > 0) retire_oldest();
+  };
   int it = 0;
   bool stop = false;
   for (int item = blockIdx.x; item < p.n_items && !stop; item += gridDim.x, ++it) {
@@ -156,8 +194,16 @@ __device__ __forceinline__ void decode_producer(const CUtensorMap* tk, const CUt
     decode_item(p, item, b, g, c);
     decode_chunk(p, b, c, lo, hi);
     const int slot = it & 1;
-    if (!leader_wait(bars + 8 * (L::kBQEmpty + slot), (static_cast<uint32_t>(it >> 1) & 1u) ^ 1u))
-      break;
+    const uint32_t qempty = bars + 8 * (L::kBQEmpty + slot);
+    const uint32_t qparity = (static_cast<uint32_t>(it >> 1) & 1u) ^ 1u;
+    // The q slot frees when the item two back has run its last score MMA,
+    // which may wait on tiles this warp has not signalled yet: signal them
+    // first unless the slot is already free.
+    if (paged && npend > 0) {
+      bool free_now = leader ? mbar_try_wait(qempty, qparity) : false;
+      if (!__shfl_sync(mask, free_now ? 1 : 0, 0)) retire_all();
+    }
+    if (!leader_wait(qempty, qparity)) break;
     if (leader) {
       volatile int* meta = reinterpret_cast<volatile int*>(
           __cvta_shared_to_generic(sbase + L::kMetaOff + slot * 16));
@@ -176,13 +222,14 @@ __device__ __forceinline__ void decode_producer(const CUtensorMap* tk, const CUt
       // Paged cache: the physical page of each page-sized (at most 128-row)
       // slice of the tile, read before the ring-slot waits so the loads'
       // latency overlaps them.
-      int pg[kDecMaxPagesPerTile];
+      // Lane j < 8 holds the page of slice j of the tile (a slice is
+      // min(page_size, 128) rows); the other lanes read it by shuffle.
+      int pg_lane = 0;
       if (paged) {
         const int* bt = p.block_table + static_cast<size_t>(b) * p.max_pages;
         const int slice = min(1 << p.page_shift, kDecBN);
-#pragma unroll
-        for (int j = 0; j < kDecMaxPagesPerTile; ++j)
-          pg[j] = (j * slice < ntok) ? __ldg(bt + ((t0 + j * slice) >> p.page_shift)) : 0;
+        if (lane < kDecMaxPagesPerTile && lane * slice < ntok)
+          pg_lane = __ldg(bt + ((t0 + lane * slice) >> p.page_shift));
       }
 #pragma unroll
       for (int kv = 0; kv < 2; ++kv) {
@@ -194,25 +241,32 @@ __device__ __forceinline__ void decode_producer(const CUtensorMap* tk, const CUt
         const uint32_t full = bars + 8 * (L::kBKvFull + stage);
         const uint32_t dst = sbase + L::kRingOff + stage * L::kTileBytes;
         if (paged) {
-          // Boxes never straddle a page: t0 is a multiple of 128 and the box
-          // height divides both 128 and the page size.
-          const bool whole = (ntok == kDecBN);
-          const int rows = whole ? p.rows_main : p.rows_tail;
-          const int nsub = (ntok + rows - 1) / rows;
-          const CUtensorMap* tm = whole ? (kv ? tv : tk) : (kv ? tv32 : tk32);
-          if (leader) mbar_arrive_expect_tx(full, nsub * rows * 128 * (D / 64));
-          __syncwarp(mask);
-          if (lane < nsub * (D / 64)) {  // at most 16 boxes per tile (page size 16)
-            const int sub = lane / (D / 64), kb = lane % (D / 64);
-            const int slice = min(1 << p.page_shift, kDecBN);
-            int page = pg[0];
-#pragma unroll
-            for (int j = 1; j < kDecMaxPagesPerTile; ++j)
-              if (sub * rows >= j * slice) page = pg[j];
-            const int prow = (t0 + sub * rows) & ((1 << p.page_shift) - 1);
-            tma_load_3d(dst + kb * L::kBoxBytes + sub * rows * 128, tm, full, kb * 64, prow,
-                        page * p.Hkv + g);
+          // t0 is a multiple of 128, so slice j of the tile is rows
+          // [j * slice, (j + 1) * slice) of one page.
+          constexpr int kChunks = D * 2 / 16;     // 16-byte chunks per row
+          constexpr int kRowsPerPass = 32 / kChunks;
+          const int ch = lane % kChunks;
+          const char* pool = kv ? p.v_pool : p.k_pool;
+          const uint32_t dcol = dst + (ch >> 3) * L::kBoxBytes;
+          const size_t row_bytes = static_cast<size_t>(D) * 2;
+          const int pmask = (1 << p.page_shift) - 1;
+          for (int r = lane / kChunks; r < kDecBN; r += kRowsPerPass) {
+            const int page = min(max(__shfl_sync(0xffffffffu, pg_lane, min(r >> p.page_shift, 7)),
+                                     0), p.num_pages - 1);
+            const bool valid = r < ntok;
+            const char* src =
+                valid ? pool + ((static_cast<size_t>(page) * p.Hkv + g) * (pmask + 1) +
+                                ((t0 + r) & pmask)) * row_bytes + ch * 16
+                      : pool;
+            cp_async16(dcol + r * 128 + (((ch & 7) ^ (r & 7)) << 4), src, valid ? 16u : 0u);
           }
+          cp_async_commit();
+          ++ld;
+          if (++npend > kDecCpLag) {
+            cp_async_wait<kDecCpLag>();
+            retire_oldest();
+          }
+          continue;
         } else if (leader) {
           if (ntok == kDecBN) {
             mbar_arrive_expect_tx(full, L::kTileBytes);
@@ -235,6 +289,7 @@ __device__ __forceinline__ void decode_producer(const CUtensorMap* tk, const CUt
     if (stop) ++it;  // this item's q load was issued
   }
   // Drain: no copy may still be in flight when the CTA exits.
+  if (paged) retire_all();
   if (leader) {
     const uint32_t S = static_cast<uint32_t>(L::kStages);
     for (uint32_t k = (ld > S ? ld - S : 0u); k < ld; ++k)
@@ -557,7 +612,9 @@ fa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
   const uint32_t bars = sbase + L::kBarOff;
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::kStages; ++s) {
-      mbar_init(bars + 8 * (L::kBKvFull + s), 1);
+      // a paged tile is signalled by each producer lane (cp.async), a
+      // contiguous one by the TMA transaction count
+      mbar_init(bars + 8 * (L::kBKvFull + s), p.block_table != nullptr ? 32 : 1);
       mbar_init(bars + 8 * (L::kBKvEmpty + s), 1);
     }
     for (int k = 0; k < 2; ++k) {

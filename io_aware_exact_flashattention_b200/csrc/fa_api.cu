@@ -144,11 +144,19 @@ cudaError_t prepare_prefill(int dev) {
   return g_attr_err[dev];
 }
 
+// Which query tiles a prefill launch computes and where its outputs go: a
+// whole forward is tiles [0, ceil(Sq/128)) into o [B,Hq,Sq,d], lse [B,Hq,Sq].
+struct PrefillRange {
+  int q_tile0, q_tile_end;
+  int o_rows, o_row0, lse_rows, lse_row0;
+};
+
 template <int D, bool kF8 = false>
 fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                          int Hq, int Hkv, int Sq, int Skv, int causal, float scale,
                          cudaStream_t stream, const float* descale_q = nullptr,
-                         const float* descale_k = nullptr, const float* descale_v = nullptr) {
+                         const float* descale_k = nullptr, const float* descale_v = nullptr,
+                         const PrefillRange* range = nullptr) {
   CUtensorMap tq, tk, tv;
   auto encode = kF8 ? encode_bhsd_e4m3 : encode_bhsd;
   if (Skv == 0) k = v = q;  // no key tile is ever loaded; any valid address will do
@@ -172,8 +180,17 @@ fa_status launch_prefill(const void* q, const void* k, const void* v, void* o, f
   p.group = Hq / Hkv;
   p.causal = causal ? 1 : 0;
   const int q_tiles = (Sq + fa::kBM - 1) / fa::kBM;
-  p.n_qpairs = (q_tiles + 1) / 2;
+  const PrefillRange whole{0, q_tiles, Sq, 0, Sq, 0};
+  const PrefillRange& rg = range ? *range : whole;
+  p.q_tile0 = rg.q_tile0;
+  p.q_tile_end = rg.q_tile_end;
+  p.o_rows = rg.o_rows;
+  p.o_row0 = rg.o_row0;
+  p.lse_rows = rg.lse_rows;
+  p.lse_row0 = rg.lse_row0;
+  p.n_qpairs = (rg.q_tile_end - rg.q_tile0 + 1) / 2;
   p.n_items = p.n_qpairs * B * Hq;
+  if (p.n_items <= 0) return FA_OK;
   p.n_kv_tiles = (Skv + fa::kBN - 1) / fa::kBN;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -259,7 +276,10 @@ fa_status launch_decode(const void* q, const void* kc, const void* vc, const int
                         int num_splits, float scale, int num_sms, cudaStream_t stream,
                         const PagedCache* pg) {
   CUtensorMap tk, tv, tk32, tv32, tq;
-  // Contiguous: planes (b, g) of Lmax rows.  Paged: planes (page, g) of page_size rows.
+  // Contiguous cache: planes (b, g) of Lmax rows, loaded by TMA.  A paged
+  // cache is copied by the producer warp's cp.async and needs no map; the
+  // maps are still encoded (over the pool, planes (page, g)) so the kernel's
+  // parameters are always valid.
   const long long planes = pg ? static_cast<long long>(pg->num_pages) * Hkv
                               : static_cast<long long>(B) * Hkv;
   const int rows = pg ? pg->page_size : Lmax;
@@ -285,12 +305,13 @@ fa_status launch_decode(const void* q, const void* kc, const void* vc, const int
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_limit_ns = kWaitLimitNs;
   p.block_table = pg ? pg->block_table : nullptr;
+  p.k_pool = pg ? static_cast<const char*>(kc) : nullptr;
+  p.v_pool = pg ? static_cast<const char*>(vc) : nullptr;
+  p.num_pages = pg ? pg->num_pages : 0;
   p.max_pages = pg ? pg->max_pages : 0;
   int shift = 0;
   while (pg && (1 << shift) < pg->page_size) ++shift;
   p.page_shift = shift;
-  p.rows_main = box_main;
-  p.rows_tail = box_tail;
   p.chunk_align = pg ? fa::kDecBN : 1;
   const int grid = p.n_items < num_sms ? p.n_items : num_sms;
   fa::fa_decode_split_kernel<D, G><<<grid, fa::kDecThreads, fa::DecodeLayout<D>::kBytes,
@@ -589,6 +610,8 @@ fa_status fa_bpt_ffn(const void* o, const void* w1, const void* w2, void* y,
   p1.tiles_per_seq = static_cast<int>(tiles_per_seq);
   p1.a_heads = 1;
   p1.c_tokens = 0;
+  p1.S_out = S;
+  p1.tok0 = 0;
   p1.gelu = 1;
   p1.wait_limit_ns = kWaitLimitNs;
   fa::FfnParams p2 = p1;  // Y = H W2^T, rows back to their tokens
@@ -605,6 +628,99 @@ fa_status fa_bpt_ffn(const void* o, const void* w1, const void* w2, void* y,
                              fa::kFfnThreads, fa::FfnLayout::kBytes, s>>>(tm_o, tm_w1, p1);
     fa::fa_ffn_gemm_kernel<<<dim3(static_cast<unsigned>(D / fa::kFfnBN), static_cast<unsigned>(n)),
                              fa::kFfnThreads, fa::FfnLayout::kBytes, s>>>(tm_h, tm_w2, p2);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+size_t fa_bpt_layer_workspace_bytes(int B, int Hq, int d, int F, int chunk_tiles) {
+  if (B < 1 || Hq < 1 || d < 1 || F < 1 || chunk_tiles < 1) return 0;
+  const size_t rows = static_cast<size_t>(chunk_tiles) * fa::kBM;
+  const size_t o_bytes = static_cast<size_t>(B) * Hq * rows * d * 2;
+  return ((o_bytes + 255) & ~static_cast<size_t>(255)) + static_cast<size_t>(B) * rows * F * 2;
+}
+
+fa_status fa_bpt_layer(const void* q, const void* k, const void* v, const void* w1,
+                       const void* w2, void* y, float* lse, void* workspace, int B, int Hq,
+                       int Hkv, int S, int d, int F, int causal, float scale, int chunk_tiles,
+                       fa_stream_t stream) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || S < 0 || F < 1 || chunk_tiles < 1) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (scale < 0.f) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const long long D = static_cast<long long>(Hq) * d;
+  if (D % fa::kFfnBN != 0 || F % fa::kFfnBN != 0 || D > (1 << 20) || F > (1 << 20))
+    return FA_ERR_UNSUPPORTED;
+  if (B == 0 || S == 0) return FA_OK;
+  if (q == nullptr || k == nullptr || v == nullptr || w1 == nullptr || w2 == nullptr ||
+      y == nullptr || lse == nullptr || workspace == nullptr)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(w1) || !aligned16(w2) ||
+      !aligned16(y) || !aligned16(lse) || !aligned16(workspace))
+    return FA_ERR_ALIGNMENT;
+  const long long tiles_per_seq = (static_cast<long long>(S) + fa::kBM - 1) / fa::kBM;
+  if (chunk_tiles > tiles_per_seq) chunk_tiles = static_cast<int>(tiles_per_seq);
+  const long long rows = static_cast<long long>(chunk_tiles) * fa::kBM;  // chunk rows per head
+  if (static_cast<long long>(B) * Hq * rows > 0x7fffffffLL ||
+      static_cast<long long>(B) * chunk_tiles > 65535 ||
+      static_cast<long long>(B) * S * D > (1LL << 40) || static_cast<long long>(B) * Hq > 0x7fffffffLL)
+    return FA_ERR_UNSUPPORTED;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  void* o_chunk = ws;
+  const size_t o_bytes = static_cast<size_t>(B) * Hq * rows * d * 2;
+  void* h_chunk = ws + ((o_bytes + 255) & ~static_cast<size_t>(255));
+  CUtensorMap tm_o, tm_w1, tm_w2, tm_h;
+  if (!encode_bhsd(&tm_o, o_chunk, d, static_cast<int>(rows), static_cast<long long>(B) * Hq) ||
+      !encode_rows256(&tm_w1, w1, static_cast<int>(D), F) ||
+      !encode_rows256(&tm_w2, w2, F, static_cast<int>(D)) ||
+      !encode_bhsd(&tm_h, h_chunk, F, static_cast<int>(B * rows), 1))
+    return FA_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (prepare_ffn(dev) != cudaSuccess) return FA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  for (long long c0 = 0; c0 < tiles_per_seq; c0 += chunk_tiles) {
+    const int tiles = static_cast<int>(std::min<long long>(chunk_tiles, tiles_per_seq - c0));
+    const int tok0 = static_cast<int>(c0 * fa::kBM);
+    // 1. attention for query tiles [c0, c0 + tiles) of every (b, h): O into
+    //    the chunk buffer (its row 0 is query row tok0), LSE into lse
+    const PrefillRange rg{static_cast<int>(c0), static_cast<int>(c0) + tiles,
+                          static_cast<int>(rows), tok0, S, 0};
+    const fa_status st =
+        d == 64 ? launch_prefill<64>(q, k, v, o_chunk, lse, B, Hq, Hkv, S, S, causal, scale, s,
+                                     nullptr, nullptr, nullptr, &rg)
+                : launch_prefill<128>(q, k, v, o_chunk, lse, B, Hq, Hkv, S, S, causal, scale, s,
+                                      nullptr, nullptr, nullptr, &rg);
+    if (st != FA_OK) return st;
+    // 2. H = gelu(X W1^T) of the chunk's tokens; 3. y = H W2^T at their tokens
+    fa::FfnParams p1;
+    p1.c = static_cast<__nv_bfloat16*>(h_chunk);
+    p1.N = F;
+    p1.K = static_cast<int>(D);
+    p1.S = static_cast<int>(std::min<long long>(rows, S - tok0));
+    p1.Hq = Hq;
+    p1.d = d;
+    p1.tiles_per_seq = tiles;
+    p1.mt0 = 0;
+    p1.a_heads = 1;
+    p1.c_tokens = 0;
+    p1.S_out = S;
+    p1.tok0 = tok0;
+    p1.gelu = 1;
+    p1.wait_limit_ns = kWaitLimitNs;
+    fa::FfnParams p2 = p1;
+    p2.c = static_cast<__nv_bfloat16*>(y);
+    p2.N = static_cast<int>(D);
+    p2.K = F;
+    p2.a_heads = 0;
+    p2.c_tokens = 1;
+    p2.gelu = 0;
+    const unsigned gy = static_cast<unsigned>(B * tiles);
+    fa::fa_ffn_gemm_kernel<<<dim3(static_cast<unsigned>(F / fa::kFfnBN), gy), fa::kFfnThreads,
+                             fa::FfnLayout::kBytes, s>>>(tm_o, tm_w1, p1);
+    fa::fa_ffn_gemm_kernel<<<dim3(static_cast<unsigned>(D / fa::kFfnBN), gy), fa::kFfnThreads,
+                             fa::FfnLayout::kBytes, s>>>(tm_h, tm_w2, p2);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   return FA_OK;

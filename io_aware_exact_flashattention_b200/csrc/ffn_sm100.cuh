@@ -55,12 +55,13 @@ struct FfnLayout {
 struct FfnParams {
   __nv_bfloat16* c;   // output rows, N bf16 each
   int N, K;           // N % 256 == 0, K % 64 == 0
-  int S;              // tokens per sequence
+  int S;              // tokens per sequence held by A (rows past S are never stored)
   int Hq, d;          // geometry of the attention output (first product)
   int tiles_per_seq;  // ceil(S / 128)
   int mt0;            // first query tile (over all sequences) of this launch
   int a_heads;        // 1: A = attention output [B*Hq, S, d]; 0: A = chunk scratch [rows, K]
-  int c_tokens;       // 1: C row = token b*S + t; 0: C row = chunk-local row
+  int c_tokens;       // 1: C row = token b*S_out + tok0 + t; 0: C row = chunk-local row
+  int S_out, tok0;    // tokens per sequence of C and the token of A's row 0 (c_tokens)
   int gelu;           // apply GELU (erf form) before rounding to bf16
   unsigned long long wait_limit_ns;
 };
@@ -169,7 +170,7 @@ fa_ffn_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const bool valid = t0 + r < p.S;
-      const long long row = p.c_tokens ? static_cast<long long>(b) * p.S + t0 + r
+      const long long row = p.c_tokens ? static_cast<long long>(b) * p.S_out + p.tok0 + t0 + r
                                        : static_cast<long long>(local_row0) + r;
       uint4* dst = reinterpret_cast<uint4*>(p.c + row * p.N + n0);
 #pragma unroll 1

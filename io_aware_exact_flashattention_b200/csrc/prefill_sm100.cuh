@@ -153,7 +153,13 @@ struct PrefillParams {
   float* lse;
   int B, Hq, Hkv, Sq, Skv, group;
   int causal;
-  int n_qpairs;    // ceil(ceil(Sq / 128) / 2)
+  // The launch computes query tiles [q_tile0, q_tile_end) of every (b, h)
+  // (all tiles for a whole forward; a range for blockwise use).  Output row
+  // `row` of head (b, h) is o[((b*Hq + h) * o_rows + row - o_row0) * D] and
+  // lse[(b*Hq + h) * lse_rows + row - lse_row0].
+  int q_tile0, q_tile_end;
+  int o_rows, o_row0, lse_rows, lse_row0;
+  int n_qpairs;    // ceil((q_tile_end - q_tile0) / 2)
   int n_items;     // n_qpairs * B * Hq
   int n_kv_tiles;  // ceil(Skv / 128)
   float scale;     // natural units
@@ -192,9 +198,10 @@ struct PrefillLayout {
   static constexpr int kBytes = kAbortOff + 4 + 1024;  // + slack for 1024-byte alignment
 };
 
-// Number of key/value tiles query tile starting at row r0 must visit.
+// Number of key/value tiles query tile starting at row r0 must visit (0 for
+// a tile outside the launch's range).
 __device__ __forceinline__ int prefill_tiles_for(const PrefillParams& p, int r0) {
-  if (r0 >= p.Sq || p.Skv <= 0) return 0;
+  if (r0 >= p.Sq || r0 >= p.q_tile_end * kBM || p.Skv <= 0) return 0;
   if (!p.causal) return p.n_kv_tiles;
   const int last_row = min(r0 + kBM - 1, p.Sq - 1);
   const long long last_key = static_cast<long long>(last_row) + (p.Skv - p.Sq);
@@ -203,7 +210,7 @@ __device__ __forceinline__ int prefill_tiles_for(const PrefillParams& p, int r0)
 }
 
 struct PrefillItem {
-  int pair, b, h, g, n0, n1;
+  int tile0, b, h, g, n0, n1;  // query tiles tile0 and tile0 + 1 of head (b, h)
 };
 
 // Item k in longest-first order: pairs of query tiles in descending order
@@ -211,14 +218,15 @@ struct PrefillItem {
 __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int k) {
   PrefillItem it;
   const int bh_count = p.B * p.Hq;
-  it.pair = k / bh_count;
-  if (p.causal) it.pair = p.n_qpairs - 1 - it.pair;
+  int pair = k / bh_count;
+  if (p.causal) pair = p.n_qpairs - 1 - pair;
+  it.tile0 = p.q_tile0 + 2 * pair;
   const int bh = k % bh_count;
   it.b = bh / p.Hq;
   it.h = bh % p.Hq;
   it.g = it.h / p.group;
-  it.n0 = prefill_tiles_for(p, (2 * it.pair) * kBM);
-  it.n1 = prefill_tiles_for(p, (2 * it.pair + 1) * kBM);
+  it.n0 = prefill_tiles_for(p, it.tile0 * kBM);
+  it.n1 = prefill_tiles_for(p, (it.tile0 + 1) * kBM);
   return it;
 }
 
@@ -260,8 +268,10 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
     lse_scale *= f;
     o_factor = p.descale_v ? p.descale_v[bg] : 1.f;
   }
-  const int q_row0 = (2 * item.pair + w) * kBM;
+  const int q_row0 = (item.tile0 + w) * kBM;
   const int row = q_row0 + row_in_tile;
+  // rows of this launch: inside the sequence and inside the launch's tile range
+  const bool row_out = row < p.Sq && item.tile0 + w < p.q_tile_end;
   // keys with index > last_key are masked for this row
   const long long last_key_ll = p.causal ? static_cast<long long>(row) + off
                                          : static_cast<long long>(p.Skv) - 1;
@@ -269,14 +279,16 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
 
   float m = -INFINITY;
   float l = 0.f;
-  const size_t row_index = (static_cast<size_t>(item.b) * p.Hq + item.h) * p.Sq + row;
+  const size_t bh = static_cast<size_t>(item.b) * p.Hq + item.h;
+  const size_t o_index = bh * p.o_rows + (row - p.o_row0);
+  const size_t lse_index = bh * p.lse_rows + (row - p.lse_row0);
 
   if (n_tiles == 0) {
-    if (row < p.Sq) {
-      uint4* dst = reinterpret_cast<uint4*>(p.o + row_index * D);
+    if (row_out) {
+      uint4* dst = reinterpret_cast<uint4*>(p.o + o_index * D);
 #pragma unroll
       for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
-      p.lse[row_index] = -INFINITY;
+      p.lse[lse_index] = -INFINITY;
     }
     continue;
   }
@@ -376,7 +388,8 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
         tmem_st16(tS + half * 16, pk);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar_p + 8 * half);
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(bar_p + 8 * half);
         return;
       }
       uint32_t pk[32];
@@ -393,7 +406,9 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
       tmem_st32(tS + half * 32, pk);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar_p + 8 * half);
+      // one arrival per warp once all its lanes' stores are done
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(bar_p + 8 * half);
     };
     if (tile_masked) {
       exps_half(std::false_type{}, 0);
@@ -417,8 +432,8 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
   {
     uint32_t r[D];
     tmem_ld_row<D>(tO, r);
-    if (row < p.Sq) {
-      uint8_t* dst = reinterpret_cast<uint8_t*>(p.o + row_index * D);
+    if (row_out) {
+      uint8_t* dst = reinterpret_cast<uint8_t*>(p.o + o_index * D);
       const float2 il = make_float2(inv_l, inv_l);
 #pragma unroll
       for (int c = 0; c < D / 16; ++c) {
@@ -438,10 +453,10 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
       }
     }
   }
-  if (row < p.Sq) {
+  if (row_out) {
     float lse = m * lse_scale + logf(l);
     if constexpr (kF8) lse -= kPOffsetF8 * 0.69314718055994531f;  // the 2^6 of P
-    p.lse[row_index] = (l > 0.f) ? lse : -INFINITY;
+    p.lse[lse_index] = (l > 0.f) ? lse : -INFINITY;
   }
   }
 }
@@ -476,7 +491,7 @@ __device__ __forceinline__ void prefill_producer(const CUtensorMap* tm_q, const 
 #pragma unroll
       for (int kb = 0; kb < L::kBoxes; ++kb)
         tma_load_3d(sbase + L::kQOff + w * L::kTileBytes + kb * kSwzBytes, tm_q, bar_q,
-                    kb * L::kBoxElems, (2 * item.pair + w) * kBM, item.b * p.Hq + item.h);
+                    kb * L::kBoxElems, (item.tile0 + w) * kBM, item.b * p.Hq + item.h);
     ++nq;
     const int n_max = max(item.n0, item.n1);
     for (int idx = 0; idx < 2 * n_max; ++idx) {
@@ -652,8 +667,8 @@ fa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(bars + 8 * (L::kBarSFull + w), 1);
-      mbar_init(bars + 8 * (L::kBarPFull + 2 * w), 128);
-      mbar_init(bars + 8 * (L::kBarPFull + 2 * w + 1), 128);
+      mbar_init(bars + 8 * (L::kBarPFull + 2 * w), 4);  // one arrival per softmax warp
+      mbar_init(bars + 8 * (L::kBarPFull + 2 * w + 1), 4);
       mbar_init(bars + 8 * (L::kBarOFull + w), 1);
     }
     mbar_init(bars + 8 * L::kBarDone, 1);

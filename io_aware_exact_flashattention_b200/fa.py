@@ -40,6 +40,8 @@ SIGNATURES = {
     "fa_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "fa_bpt_ffn": (_I, [_VP] * 5 + [_I] * 6 + [_VP]),
     "fa_bpt_workspace_bytes": (ctypes.c_size_t, [_I, _I]),
+    "fa_bpt_layer": (_I, [_VP] * 8 + [_I] * 7 + [_F, _I, _VP]),
+    "fa_bpt_layer_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
     "fa_decode_default_splits": (_I, [_I, _I, _I, _I]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_get_device_status": (_I, []),
@@ -218,13 +220,55 @@ def bpt_ffn(o: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor,
     return y
 
 
+def bpt_layer_workspace_bytes(B: int, Hq: int, d: int, F: int, chunk_tiles: int) -> int:
+    return int(lib().fa_bpt_layer_workspace_bytes(B, Hq, d, F, chunk_tiles))
+
+
+def fa_bpt_layer(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, w1: torch.Tensor,
+                 w2: torch.Tensor, y: torch.Tensor, lse: torch.Tensor, workspace: torch.Tensor,
+                 causal: bool, scale: float, chunk_tiles: int,
+                 stream: Optional[torch.cuda.Stream] = None) -> None:
+    """fa_bpt_layer: attention then the feed-forward network, chunk by chunk
+    of chunk_tiles query tiles; y [B,S,Hq*d] bf16 and lse [B,Hq,S] fp32."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (w1, "w1"), (w2, "w2"), (y, "y")):
+        _need(t, torch.bfloat16, n)
+    _need(lse, torch.float32, "lse")
+    B, Hq, S, d = q.shape
+    _, Hkv, Skv, _ = k.shape
+    D = Hq * d
+    F = w1.shape[0]
+    if Skv != S or tuple(v.shape) != tuple(k.shape) or k.shape[0] != B or k.shape[3] != d:
+        raise ValueError("self-attention: k, v [B,Hkv,S,d] with q's B, S and d")
+    if tuple(w1.shape) != (F, D) or tuple(w2.shape) != (D, F) or tuple(y.shape) != (B, S, D):
+        raise ValueError("w1 [F, D], w2 [D, F] and y [B, S, D] with D = Hq * d")
+    if tuple(lse.shape) != (B, Hq, S):
+        raise ValueError("lse must be [B, Hq, S]")
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    if workspace.numel() * workspace.element_size() < bpt_layer_workspace_bytes(B, Hq, d, F,
+                                                                               chunk_tiles):
+        raise ValueError("workspace smaller than fa_bpt_layer_workspace_bytes")
+    _check("fa_bpt_layer", lib().fa_bpt_layer(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(w1), _ptr(w2), _ptr(y), _ptr(lse), _ptr(workspace), B,
+        Hq, Hkv, S, d, F, int(bool(causal)), float(scale), int(chunk_tiles), _stream_ptr(stream)))
+
+
 def bpt_layer(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, w1: torch.Tensor,
               w2: torch.Tensor, causal: bool = False, scale: Optional[float] = None,
-              chunk_tiles: int = 16) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
-    """Attention (fa_fwd) followed by the blockwise feed-forward network:
-    returns (y [B,S,Hq*d], o, lse)."""
-    o, lse = flash_attention(q, k, v, causal=causal, scale=scale)
-    return bpt_ffn(o, w1, w2, chunk_tiles), o, lse
+              chunk_tiles: int = 16) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Attention followed by the feed-forward network, block by block
+    (fa_bpt_layer): returns (y [B,S,Hq*d], lse).  Only one chunk's attention
+    output and hidden activations exist at a time."""
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    B, Hq, S, d = q.shape
+    F = w1.shape[0]
+    y = torch.empty((B, S, Hq * d), device=q.device, dtype=torch.bfloat16)
+    lse = torch.empty((B, Hq, S), device=q.device, dtype=torch.float32)
+    ws = torch.empty(max(16, bpt_layer_workspace_bytes(B, Hq, d, F, chunk_tiles)),
+                     dtype=torch.uint8, device=q.device)
+    fa_bpt_layer(q, k, v, w1, w2, y, lse, ws, causal, scale, chunk_tiles)
+    return y, lse
 
 
 def bwd_workspace_bytes(B: int, Hq: int, Sq: int, d: int) -> int:

@@ -201,6 +201,40 @@ def test_bpt_ffn_rejects_before_cuda(lib, kw, want):
     assert bpt(lib, **kw) == want
 
 
+def bpt_layer(lib, q=A, k=A, v=A, w1=A, w2=A, y=A, lse=A, ws=A, B=1, Hq=2, Hkv=1, S=300,
+              d=128, F=512, causal=1, scale=0.1, chunk=2):
+    return lib.fa_bpt_layer(q, k, v, w1, w2, y, lse, ws, B, Hq, Hkv, S, d, F, causal, scale,
+                            chunk, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(d=96), UNSUPPORTED),
+    (dict(Hq=1), UNSUPPORTED),           # D = 128 is not a multiple of 256
+    (dict(F=300), UNSUPPORTED),
+    (dict(Hq=4, Hkv=3), INVALID),
+    (dict(chunk=0), INVALID),
+    (dict(scale=-1.0), UNSUPPORTED),
+    (dict(scale=float("nan")), INVALID),
+    (dict(B=-1), INVALID),
+    (dict(q=None), INVALID),
+    (dict(lse=None), INVALID),
+    (dict(ws=None), INVALID),
+    (dict(y=A + 8), ALIGNMENT),
+    (dict(k=A + 2), ALIGNMENT),
+    (dict(B=0, q=None), OK),
+    (dict(S=0, q=None), OK),
+])
+def test_bpt_layer_rejects_before_cuda(lib, kw, want):
+    assert bpt_layer(lib, **kw) == want
+
+
+def test_bpt_layer_workspace_bytes(lib):
+    rows = 3 * 128
+    o_bytes = 2 * 4 * rows * 64 * 2
+    assert fa.bpt_layer_workspace_bytes(2, 4, 64, 512, 3) == o_bytes + 2 * rows * 512 * 2
+    assert fa.bpt_layer_workspace_bytes(0, 4, 64, 512, 3) == 0
+
+
 def test_bpt_workspace_bytes(lib):
     assert fa.bpt_workspace_bytes(512, 3) == 3 * 128 * 512 * 2
     assert fa.bpt_workspace_bytes(0, 3) == 0

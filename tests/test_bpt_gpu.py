@@ -83,25 +83,48 @@ def test_chunking_changes_nothing():
         assert torch.equal(y, ys[0])
 
 
-def test_layer_is_attention_then_ffn():
-    """bpt_layer = fa_fwd then the blockwise network, checked against the
-    oracle's layer.  The bound adds the attention's own error (|dO| <= 2e-2,
-    the forward's tolerance) carried through GELU and both maps."""
-    B, Hq, Hkv, S, d, F = 1, 2, 1, 300, 128, 512
-    q, k, v = prefill_inputs(B, Hq, Hkv, S, S, d, seed=9)
+@pytest.mark.parametrize("B,Hq,Hkv,S,d,causal", [(1, 2, 1, 300, 128, True),
+                                                (2, 4, 2, 700, 64, True),
+                                                (1, 2, 2, 520, 128, False)])
+def test_layer_is_attention_then_ffn(B, Hq, Hkv, S, d, causal):
+    """bpt_layer runs attention and the network chunk by chunk; its y equals
+    the network on fa_fwd's whole output and its LSE equals fa_fwd's, bit for
+    bit, for chunkings that split query-tile pairs (1, 3) or not (2) and one
+    chunk (100); and y is checked against the oracle's layer.  The bound adds
+    the attention's own error (|dO| <= 2e-2, the forward's tolerance) carried
+    through GELU and both maps."""
+    F = 512
+    q, k, v = prefill_inputs(B, Hq, Hkv, S, S, d, seed=9 + S)
     _, w1, w2 = ffn_inputs(B, Hq, S, d, F, seed=9)
     scale = 1.0 / math.sqrt(d)
-    y, o, _ = fa.bpt_layer(q.cuda(), k.cuda(), v.cuda(), w1.cuda(), w2.cuda(), causal=True,
-                           scale=scale, chunk_tiles=2)
-    torch.cuda.synchronize()
-    assert torch.equal(y, fa.bpt_ffn(o, w1.cuda(), w2.cuda(), chunk_tiles=2))
-    y_ref, o_ref, _ = oracle.bpt_layer(q, k, v, w1, w2, True, scale)
-    x_ref = oracle.heads_to_tokens(o_ref).reshape(S, Hq * d)
+    qc, kc, vc, w1c, w2c = q.cuda(), k.cuda(), v.cuda(), w1.cuda(), w2.cuda()
+    o = torch.empty_like(qc)
+    lse = torch.empty((B, Hq, S), device="cuda")
+    fa.fa_fwd(qc, kc, vc, o, lse, causal, scale)
+    y_two_pass = fa.bpt_ffn(o, w1c, w2c, chunk_tiles=2)
+    for chunk in (1, 2, 3, 100):
+        y, lse_l = fa.bpt_layer(qc, kc, vc, w1c, w2c, causal=causal, scale=scale,
+                                chunk_tiles=chunk)
+        torch.cuda.synchronize()
+        assert torch.equal(y, y_two_pass), chunk
+        assert torch.equal(lse_l, lse), chunk
+    y_ref, o_ref, _ = oracle.bpt_layer(q, k, v, w1, w2, causal, scale)
+    x_ref = oracle.heads_to_tokens(o_ref).reshape(B * S, Hq * d)
     w1n, w2n = (w.double().numpy() for w in (w1, w2))
-    tol = ffn_bound(x_ref, w1n, w2n, oracle.ffn_hidden(x_ref, w1n), y_ref.reshape(S, -1))
+    tol = ffn_bound(x_ref, w1n, w2n, oracle.ffn_hidden(x_ref, w1n), y_ref.reshape(B * S, -1))
     tol = tol + 1.13 * 2e-2 * (np.abs(w2n) @ (np.abs(w1n) @ np.ones(Hq * d)))[None, :]
-    got = y.reshape(S, -1).float().cpu().numpy()
-    assert (np.abs(got - y_ref.reshape(S, -1)) <= tol).all()
+    got = y.reshape(B * S, -1).float().cpu().numpy()
+    assert (np.abs(got - y_ref.reshape(B * S, -1)) <= tol).all()
+
+
+def test_layer_workspace_is_one_chunk():
+    """The layer's scratch holds one chunk's attention output and hidden
+    activations, not the sequence's."""
+    B, Hq, d, F, chunk = 4, 16, 128, 8192, 2
+    got = fa.bpt_layer_workspace_bytes(B, Hq, d, F, chunk)
+    rows = chunk * 128
+    assert got == B * Hq * rows * d * 2 + B * rows * F * 2
+    assert got * 8 == B * 2048 * Hq * d * 2 + B * 2048 * F * 2  # S = 2048: 8 chunks
 
 
 def test_headline_shape_every_tile():
