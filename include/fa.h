@@ -284,8 +284,9 @@ fa_status fa_decode_splitkv(const void *q, const void *k_cache, const void *v_ca
  * (key tiles then start on tile boundaries and never straddle pages).  Chunks
  * past L_b are empty (o_partial = 0, lse_partial = -inf); fa_combine merges
  * the partials exactly as for the contiguous cache.  Rows of a page past L_b
- * are never read.  An out-of-range page index is clamped to [0, num_pages),
- * so the result is then meaningless but every read stays inside the pool.
+ * may be read but never contribute.  An out-of-range page index reads zeros
+ * or another page (never outside the cache), so the result is then
+ * meaningless but memory stays safe.
  *
  * Supported: page_size a power of two in [16, 256]; d in {64, 128};
  * Hq / Hkv in {1, 2, 4, 8}; 1 <= num_splits <= 256.  Errors as for

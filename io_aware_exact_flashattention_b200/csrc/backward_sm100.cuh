@@ -54,10 +54,10 @@ struct BwdLayout {
   static constexpr int kBQEmpty = 3;   // [2]
   static constexpr int kBSFull = 5;
   static constexpr int kBDpFull = 6;
-  static constexpr int kBPFull = 7;    // 256 arrivals
-  static constexpr int kBDsFull = 8;   // 256 arrivals
+  static constexpr int kBPFull = 7;    // 8 arrivals (one per element-wise warp)
+  static constexpr int kBDsFull = 8;   // 8 arrivals
   static constexpr int kBDqFull = 9;
-  static constexpr int kBSFree = 10;   // 256 arrivals: dQ partial read out of the dP columns
+  static constexpr int kBSFree = 10;   // 8 arrivals: dQ partial read out of the dP columns
   static constexpr int kBDone = 11;
   static constexpr int kNumBars = 12;
   static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
@@ -74,6 +74,7 @@ struct BwdParams {
   __nv_bfloat16* dv;
   int B, Hq, Hkv, Sq, Skv, group, causal;
   int n_kv_tiles, n_q_tiles;
+  int heads_per_group;  // CTA order: groups of this many (b, kv-head) pairs (see bwd_cta)
   float scale, scale_log2;
   unsigned long long wait_limit_ns;
 };
@@ -88,10 +89,21 @@ __device__ __forceinline__ int bwd_first_q_tile(const BwdParams& p, int j) {
 }
 
 __device__ __forceinline__ void bwd_cta(const BwdParams& p, int& b, int& g, int& j) {
-  // heavy key tiles first under a causal mask (key tile 0 sees every query tile)
-  const int bg_count = p.B * p.Hkv;
-  j = static_cast<int>(blockIdx.x) / bg_count;
-  const int bg = static_cast<int>(blockIdx.x) % bg_count;
+  // CTAs go out in groups of p.heads_per_group (batch, key/value head)
+  // pairs; within a group key tile by key tile, heavy tiles first (under a
+  // causal mask key tile 0 sees every query tile), so the launch order stays
+  // longest-first and the tail is short.  The CTAs resident at a time then
+  // cover about two groups, whose Q, dO and fp32 dQ rows stay in L2 while all
+  // their key tiles stream them; ordered key tile by key tile over all heads,
+  // the resident CTAs touch every head's Q, dO and dQ at once, more than L2
+  // holds.
+  const int per_group = p.heads_per_group * p.n_kv_tiles;
+  const int grp = static_cast<int>(blockIdx.x) / per_group;
+  const int r = static_cast<int>(blockIdx.x) % per_group;
+  const int units = p.B * p.Hkv;
+  const int in_group = min(p.heads_per_group, units - grp * p.heads_per_group);
+  j = r / in_group;
+  const int bg = grp * p.heads_per_group + r % in_group;
   b = bg / p.Hkv;
   g = bg % p.Hkv;
 }
@@ -385,7 +397,8 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, const CUtens
       tmem_st32(t_s + hf * kQH, pk);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bars + 8 * L::kBPFull);
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(bars + 8 * L::kBPFull);
 
       // dS = P * (dP - D): to TMEM (A of dK += dS^T Q) and to shared memory
       // (A of dQ = dS K, MN-major: rows = keys, 64-query boxes, 128B swizzle)
@@ -419,7 +432,8 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, const CUtens
       tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(bars + 8 * L::kBDsFull);
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(bars + 8 * L::kBDsFull);
 
       // dQ partial (thread = query row q0 + t, this warpgroup's d-columns),
       // scaled, staged 32 columns at a time in this warpgroup's half of the
@@ -455,7 +469,8 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, const CUtens
         }
       }
       tc_fence_before();
-      mbar_arrive(bars + 8 * L::kBSFree);
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(bars + 8 * L::kBSFree);
     }
   }
   if (t == 0) bulk_wait_group0();  // this thread's reductions have landed
@@ -517,10 +532,10 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
     mbar_init(bars + 8 * L::kBSFull, 1);
     mbar_init(bars + 8 * L::kBDpFull, 1);
-    mbar_init(bars + 8 * L::kBPFull, 256);
-    mbar_init(bars + 8 * L::kBDsFull, 256);
+    mbar_init(bars + 8 * L::kBPFull, 8);   // one arrival per element-wise warp
+    mbar_init(bars + 8 * L::kBDsFull, 8);
     mbar_init(bars + 8 * L::kBDqFull, 1);
-    mbar_init(bars + 8 * L::kBSFree, 256);
+    mbar_init(bars + 8 * L::kBSFree, 8);
     mbar_init(bars + 8 * L::kBDone, 1);
     *abort_flag = 0;
     fence_mbar_init();

@@ -24,11 +24,17 @@
 //              32-row boxes so at most 31 rows past the chunk are fetched)
 // A paged cache ([num_pages, Hkv, page_size, d] with a block table per
 // sequence; paged KV management is named in "I/O-Aware Kernels", section
-// "FlashAttention") changes only the producer: chunks start on multiples of
-// 128 keys, so a tile covers whole pages (page_size <= 128) or lies inside
-// one, and the producer warp copies it row by row (16-byte cp.async) from the
-// physical pages the block table names into the same swizzled layout TMA
-// would write.  The MMA and softmax roles see the same shared-memory tiles.
+// "FlashAttention") changes the producer: chunks start on multiples of 128
+// keys, so a tile covers whole pages (page_size <= 128) or lies inside one,
+// and it is loaded as boxes of min(page_size, 128) rows (min(page_size, 32)
+// for a chunk's last tile), each from the physical page the block table
+// names.  At d = 128 a row is two 128-byte swizzle spans, and a tile laid out
+// span by span ([half][128 rows]) would take two boxes per page; small pages
+// make the per-box cost the limit.  So a paged tile at d = 128 is laid out
+// [8-row group][half][8 rows] ("interleaved"): a page of P rows is then one
+// contiguous 256*P-byte box of a 5-D view of the pool (64 columns, 8 rows,
+// 2 halves, P/8 groups, planes), and the MMA descriptors step 1024 bytes
+// between halves and 2048 between 8-row groups instead of 16 KB and 1024.
 //   warp  5    MMA issuer
 // The online softmax keeps a per-head reference max m that only moves when
 // the max grows by more than 2^8; exp2 on scores times scale*log2(e).
@@ -44,10 +50,6 @@ constexpr int kDecNPad = 16;      // head columns of S^T / O^T (G real, rest zer
 constexpr int kDecSubRows = 32;   // rows per box of a chunk's last tile
 constexpr int kDecThreads = 192;
 constexpr int kDecMaxPagesPerTile = kDecBN / 16;  // pages of the smallest size in a tile
-// A paged cache is copied row by row with 16-byte cp.async; a tile's full
-// barrier is signalled once the copies of the tile kDecCpLag loads later are
-// issued, so this many tiles per lane are in flight.
-constexpr int kDecCpLag = 3;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kDecRescaleThreshold = 8.0f;  // log2 units
 
@@ -95,11 +97,11 @@ struct DecodeParams {
   unsigned long long wait_limit_ns;
   // paged cache (block_table == nullptr: contiguous [B, Hkv, Lmax, d] cache)
   const int* block_table;  // [B, max_pages]
-  const char* k_pool;      // [num_pages, Hkv, page_size, d] bf16
-  const char* v_pool;
-  int num_pages;           // page indices are clamped to [0, num_pages)
   int max_pages;
   int page_shift;          // log2(page_size)
+  int rows_main;           // rows per box of a full tile: min(page_size, 128)
+  int rows_tail;           // rows per box of a chunk's last tile: min(page_size, 32)
+  int interleaved;         // tile layout [8-row group][half][8 rows] (paged, d = 128)
   int chunk_align;         // chunk sizes are rounded up to a multiple of this
 };
 
@@ -122,32 +124,11 @@ __device__ __forceinline__ void decode_item(const DecodeParams& p, int item, int
   b = bg / p.Hkv;
 }
 
-// 16-byte asynchronous copy global -> shared through L2; src_bytes < 16
-// fills the rest of the 16 bytes with zeros (src_bytes = 0 reads nothing).
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 // ---------------------------------------------------------------------------
-// Producer (one warp).  Lane 0 waits for buffers, accounts the bytes and
-// issues the query loads (TMA) and the contiguous-cache tile loads (TMA, one
-// 128-row box per 64-column block).  A paged cache is not loaded by TMA: its
-// pages are scattered, and a page of 16 keys would be two 2 KB boxes, whose
-// per-box cost caps the stream.  Instead all 32 lanes copy each tile row by
-// row with 16-byte cp.async straight into the 128B-swizzled layout the MMA
-// reads (chunk c of row r lands at chunk position c ^ (r & 7)), rows past the
-// chunk filled with zeros by the copy itself, so no cache row past L_b is
-// read.  Each lane waits for its own copies kDecCpLag tile loads later, makes
-// them visible to the tensor cores (proxy fence) and arrives on the tile's
-// full barrier (32 arrivals per tile).
+// TMA producer (one warp).  Lane 0 waits for buffers, accounts the bytes and
+// issues the query loads and the contiguous-cache tile loads; for a paged
+// cache a tile is many small boxes (two per page of 16 rows at d=128), and
+// each lane issues one of them so their issue costs overlap.
 // ---------------------------------------------------------------------------
 template <int D, int G>
 __device__ __forceinline__ void decode_producer(const CUtensorMap* tk, const CUtensorMap* tv,
@@ -175,18 +156,6 @@ __device__ __forceinline__ void decode_producer(const CUtensorMap* tk, const CUt
     return __shfl_sync(mask, ok ? 1 : 0, 0) != 0;
   };
   uint32_t ld = 0;  // K/V tile loads issued
-  uint32_t npend = 0;  // paged: loads issued whose full barrier this lane has not yet signalled
-  // paged: wait for this lane's oldest pending copies and signal their tile
-  auto retire_oldest = [&]() {
-    const uint32_t k = ld - npend;
-    fence_proxy_async_smem();
-    mbar_arrive(bars + 8 * (L::kBKvFull + k % static_cast<uint32_t>(L::kStages)));
-    --npend;
-  };
-  auto retire_all = [&]() {
-    cp_async_wait<0>();
-    while (npend > 0) retire_oldest();
-  };
   int it = 0;
   bool stop = false;
   for (int item = blockIdx.x; item < p.n_items && !stop; item += gridDim.x, ++it) {
@@ -194,16 +163,8 @@ __device__ __forceinline__ void decode_producer(const CUtensorMap* tk, const CUt
     decode_item(p, item, b, g, c);
     decode_chunk(p, b, c, lo, hi);
     const int slot = it & 1;
-    const uint32_t qempty = bars + 8 * (L::kBQEmpty + slot);
-    const uint32_t qparity = (static_cast<uint32_t>(it >> 1) & 1u) ^ 1u;
-    // The q slot frees when the item two back has run its last score MMA,
-    // which may wait on tiles this warp has not signalled yet: signal them
-    // first unless the slot is already free.
-    if (paged && npend > 0) {
-      bool free_now = leader ? mbar_try_wait(qempty, qparity) : false;
-      if (!__shfl_sync(mask, free_now ? 1 : 0, 0)) retire_all();
-    }
-    if (!leader_wait(qempty, qparity)) break;
+    if (!leader_wait(bars + 8 * (L::kBQEmpty + slot), (static_cast<uint32_t>(it >> 1) & 1u) ^ 1u))
+      break;
     if (leader) {
       volatile int* meta = reinterpret_cast<volatile int*>(
           __cvta_shared_to_generic(sbase + L::kMetaOff + slot * 16));
@@ -222,14 +183,13 @@ __device__ __forceinline__ void decode_producer(const CUtensorMap* tk, const CUt
       // Paged cache: the physical page of each page-sized (at most 128-row)
       // slice of the tile, read before the ring-slot waits so the loads'
       // latency overlaps them.
-      // Lane j < 8 holds the page of slice j of the tile (a slice is
-      // min(page_size, 128) rows); the other lanes read it by shuffle.
-      int pg_lane = 0;
+      int pg[kDecMaxPagesPerTile];
       if (paged) {
         const int* bt = p.block_table + static_cast<size_t>(b) * p.max_pages;
         const int slice = min(1 << p.page_shift, kDecBN);
-        if (lane < kDecMaxPagesPerTile && lane * slice < ntok)
-          pg_lane = __ldg(bt + ((t0 + lane * slice) >> p.page_shift));
+#pragma unroll
+        for (int j = 0; j < kDecMaxPagesPerTile; ++j)
+          pg[j] = (j * slice < ntok) ? __ldg(bt + ((t0 + j * slice) >> p.page_shift)) : 0;
       }
 #pragma unroll
       for (int kv = 0; kv < 2; ++kv) {
@@ -241,32 +201,37 @@ __device__ __forceinline__ void decode_producer(const CUtensorMap* tk, const CUt
         const uint32_t full = bars + 8 * (L::kBKvFull + stage);
         const uint32_t dst = sbase + L::kRingOff + stage * L::kTileBytes;
         if (paged) {
-          // t0 is a multiple of 128, so slice j of the tile is rows
-          // [j * slice, (j + 1) * slice) of one page.
-          constexpr int kChunks = D * 2 / 16;     // 16-byte chunks per row
-          constexpr int kRowsPerPass = 32 / kChunks;
-          const int ch = lane % kChunks;
-          const char* pool = kv ? p.v_pool : p.k_pool;
-          const uint32_t dcol = dst + (ch >> 3) * L::kBoxBytes;
-          const size_t row_bytes = static_cast<size_t>(D) * 2;
-          const int pmask = (1 << p.page_shift) - 1;
-          for (int r = lane / kChunks; r < kDecBN; r += kRowsPerPass) {
-            const int page = min(max(__shfl_sync(0xffffffffu, pg_lane, min(r >> p.page_shift, 7)),
-                                     0), p.num_pages - 1);
-            const bool valid = r < ntok;
-            const char* src =
-                valid ? pool + ((static_cast<size_t>(page) * p.Hkv + g) * (pmask + 1) +
-                                ((t0 + r) & pmask)) * row_bytes + ch * 16
-                      : pool;
-            cp_async16(dcol + r * 128 + (((ch & 7) ^ (r & 7)) << 4), src, valid ? 16u : 0u);
+          // Boxes never straddle a page: t0 is a multiple of 128 and the box
+          // height divides both 128 and the page size.
+          const bool whole = (ntok == kDecBN);
+          const int rows = whole ? p.rows_main : p.rows_tail;
+          const int nsub = (ntok + rows - 1) / rows;
+          const CUtensorMap* tm = whole ? (kv ? tv : tk) : (kv ? tv32 : tk32);
+          if (leader) mbar_arrive_expect_tx(full, nsub * rows * 128 * (D / 64));
+          __syncwarp(mask);
+          if (p.interleaved) {
+            // one box per slice, both column halves ([group][half][8 rows])
+            if (lane < nsub) {
+              const int slice = min(1 << p.page_shift, kDecBN);
+              int page = pg[0];
+#pragma unroll
+              for (int j = 1; j < kDecMaxPagesPerTile; ++j)
+                if (lane * rows >= j * slice) page = pg[j];
+              const int prow = (t0 + lane * rows) & ((1 << p.page_shift) - 1);
+              tma_load_5d(dst + lane * rows * 256, tm, full, 0, 0, 0, prow >> 3,
+                          page * p.Hkv + g);
+            }
+          } else if (lane < nsub * (D / 64)) {  // at most 16 boxes per tile (page size 16)
+            const int sub = lane / (D / 64), kb = lane % (D / 64);
+            const int slice = min(1 << p.page_shift, kDecBN);
+            int page = pg[0];
+#pragma unroll
+            for (int j = 1; j < kDecMaxPagesPerTile; ++j)
+              if (sub * rows >= j * slice) page = pg[j];
+            const int prow = (t0 + sub * rows) & ((1 << p.page_shift) - 1);
+            tma_load_3d(dst + kb * L::kBoxBytes + sub * rows * 128, tm, full, kb * 64, prow,
+                        page * p.Hkv + g);
           }
-          cp_async_commit();
-          ++ld;
-          if (++npend > kDecCpLag) {
-            cp_async_wait<kDecCpLag>();
-            retire_oldest();
-          }
-          continue;
         } else if (leader) {
           if (ntok == kDecBN) {
             mbar_arrive_expect_tx(full, L::kTileBytes);
@@ -289,7 +254,6 @@ __device__ __forceinline__ void decode_producer(const CUtensorMap* tk, const CUt
     if (stop) ++it;  // this item's q load was issued
   }
   // Drain: no copy may still be in flight when the CTA exits.
-  if (paged) retire_all();
   if (leader) {
     const uint32_t S = static_cast<uint32_t>(L::kStages);
     for (uint32_t k = (ld > S ? ld - S : 0u); k < ld; ++k)
@@ -323,11 +287,15 @@ __device__ __forceinline__ void decode_mma(const DecodeParams& p, uint32_t sbase
     tc_fence_after();
     const uint32_t ka = sbase + L::kRingOff + stage * L::kTileBytes;
     const uint32_t qa = sbase + L::kQOff + slot * L::kQBytes;
+    // K tile: halves 16 KB apart and 8-row groups 1 KB apart, or (interleaved)
+    // halves 1 KB apart and groups 2 KB apart
+    const uint32_t k_half = p.interleaved ? 1024u : static_cast<uint32_t>(L::kBoxBytes);
+    const uint32_t k_sbo = p.interleaved ? 2048u : 1024u;
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t ko = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
+      const uint32_t ko = (kk >> 2) * k_half + (kk & 3) * 32;
       const uint32_t qo = (kk >> 2) * L::kQBoxBytes + (kk & 3) * 32;
-      mma_ss(tmem + (t & 1) * kDecNPad, sw128_desc(ka + ko, 16, 1024), sw128_desc(qa + qo, 16, 1024),
+      mma_ss(tmem + (t & 1) * kDecNPad, sw128_desc(ka + ko, 16, k_sbo), sw128_desc(qa + qo, 16, 1024),
              kIdS, kk > 0 ? 1u : 0u);
     }
     mma_commit(bars + 8 * (L::kBSFull + (t & 1)));
@@ -372,13 +340,16 @@ __device__ __forceinline__ void decode_mma(const DecodeParams& p, uint32_t sbase
           goto done;
         tc_fence_after();
         const uint32_t va = sbase + L::kRingOff + vstage * L::kTileBytes;
-        // second 64-row block of V^T: the tile's upper column block, or zeros for D=64
-        const uint32_t lbo = (D == 128) ? static_cast<uint32_t>(L::kBoxBytes)
+        // second 64-row block of V^T: the tile's upper column block, or zeros
+        // for D=64; 16 keys are 2 KB (4 KB interleaved) and 8-key groups 1 KB
+        // (2 KB interleaved) apart
+        const uint32_t lbo = (D == 128) ? (p.interleaved ? 1024u : static_cast<uint32_t>(L::kBoxBytes))
                                         : (sbase + L::kZeroOff) - va;
+        const uint32_t v_sbo = p.interleaved ? 2048u : 1024u;
         const uint32_t pa = sbase + L::kPOff + (t & 1) * L::kPBytes;
 #pragma unroll
         for (int kk = 0; kk < kDecBN / 16; ++kk) {
-          mma_ss(to, sw128_desc(va + kk * 16 * 128, lbo, 1024),
+          mma_ss(to, sw128_desc(va + kk * 16 * (v_sbo / 8), lbo, v_sbo),
                  sw128_desc(pa + (kk >> 2) * (kDecNPad * 128) + (kk & 3) * 32, 16, 1024), kIdO,
                  (jt > 0 || kk > 0) ? 1u : 0u);
         }
@@ -513,13 +484,16 @@ __device__ __forceinline__ void decode_softmax(const DecodeParams& p, uint32_t s
           break;
         }
         if (!valid) {
-          const uint32_t row = sbase + L::kRingOff + vstage * L::kTileBytes + t * 128;
+          const uint32_t tile = sbase + L::kRingOff + vstage * L::kTileBytes;
+          const uint32_t row = p.interleaved ? tile + (t >> 3) * 2048 + (t & 7) * 128
+                                             : tile + t * 128;
+          const uint32_t half = p.interleaved ? 1024u : static_cast<uint32_t>(L::kBoxBytes);
 #pragma unroll
           for (int kb = 0; kb < D / 64; ++kb)
 #pragma unroll
             for (int q16 = 0; q16 < 8; ++q16)
               asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};"
-                           ::"r"(row + kb * L::kBoxBytes + q16 * 16), "r"(0u)
+                           ::"r"(row + kb * half + q16 * 16), "r"(0u)
                            : "memory");
         }
       }
@@ -612,9 +586,7 @@ fa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
   const uint32_t bars = sbase + L::kBarOff;
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::kStages; ++s) {
-      // a paged tile is signalled by each producer lane (cp.async), a
-      // contiguous one by the TMA transaction count
-      mbar_init(bars + 8 * (L::kBKvFull + s), p.block_table != nullptr ? 32 : 1);
+      mbar_init(bars + 8 * (L::kBKvFull + s), 1);
       mbar_init(bars + 8 * (L::kBKvEmpty + s), 1);
     }
     for (int k = 0; k < 2; ++k) {

@@ -251,6 +251,24 @@ bool encode_cache(CUtensorMap* map, const void* base, int d, int rows, long long
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A paged pool [planes, P, 128] bf16 (P = page_size, a multiple of 8) as the
+// 5-D view (64 columns, 8 rows, 2 column halves, P/8 row groups, planes) with
+// boxes of box_rows rows: shared memory receives [group][half][8 rows][64],
+// the interleaved tile layout of the decode kernel at d = 128.
+bool encode_pool_interleaved(CUtensorMap* map, const void* base, int page_size, long long planes,
+                             int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[5] = {64, 8, 2, static_cast<cuuint64_t>(page_size / 8),
+                        static_cast<cuuint64_t>(planes)};
+  cuuint64_t strides[4] = {256, 128, 2048, static_cast<cuuint64_t>(page_size) * 256};
+  cuuint32_t box[5] = {64, 8, 2, static_cast<cuuint32_t>(box_rows / 8), 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // [rows, d] bf16 query matrix as a 2-D map with 64 x 16 boxes.
 bool encode_query(CUtensorMap* map, const void* base, int d, long long rows) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
@@ -276,21 +294,28 @@ fa_status launch_decode(const void* q, const void* kc, const void* vc, const int
                         int num_splits, float scale, int num_sms, cudaStream_t stream,
                         const PagedCache* pg) {
   CUtensorMap tk, tv, tk32, tv32, tq;
-  // Contiguous cache: planes (b, g) of Lmax rows, loaded by TMA.  A paged
-  // cache is copied by the producer warp's cp.async and needs no map; the
-  // maps are still encoded (over the pool, planes (page, g)) so the kernel's
-  // parameters are always valid.
+  // Contiguous: planes (b, g) of Lmax rows.  Paged: planes (page, g) of page_size rows.
   const long long planes = pg ? static_cast<long long>(pg->num_pages) * Hkv
                               : static_cast<long long>(B) * Hkv;
   const int rows = pg ? pg->page_size : Lmax;
   const int box_main = pg ? std::min(pg->page_size, fa::kDecBN) : fa::kDecBN;
   const int box_tail = pg ? std::min(pg->page_size, fa::kDecSubRows) : fa::kDecSubRows;
-  if (!encode_cache(&tk, kc, D, rows, planes, box_main) ||
-      !encode_cache(&tv, vc, D, rows, planes, box_main) ||
-      !encode_cache(&tk32, kc, D, rows, planes, box_tail) ||
-      !encode_cache(&tv32, vc, D, rows, planes, box_tail) ||
-      !encode_query(&tq, q, D, static_cast<long long>(B) * Hq))
+  // paged at d = 128: one box per page slice, both column halves
+  // (interleaved); should the driver refuse that view, two boxes per slice
+  bool interleaved = (pg != nullptr) && D == 128;
+  if (interleaved)
+    interleaved = encode_pool_interleaved(&tk, kc, pg->page_size, planes, box_main) &&
+                  encode_pool_interleaved(&tv, vc, pg->page_size, planes, box_main) &&
+                  encode_pool_interleaved(&tk32, kc, pg->page_size, planes, box_tail) &&
+                  encode_pool_interleaved(&tv32, vc, pg->page_size, planes, box_tail);
+  if (interleaved) {
+  } else if (!encode_cache(&tk, kc, D, rows, planes, box_main) ||
+             !encode_cache(&tv, vc, D, rows, planes, box_main) ||
+             !encode_cache(&tk32, kc, D, rows, planes, box_tail) ||
+             !encode_cache(&tv32, vc, D, rows, planes, box_tail)) {
     return FA_ERR_CUDA;
+  }
+  if (!encode_query(&tq, q, D, static_cast<long long>(B) * Hq)) return FA_ERR_CUDA;
   fa::DecodeParams p;
   p.o_part = o_part;
   p.lse_part = lse_part;
@@ -305,13 +330,13 @@ fa_status launch_decode(const void* q, const void* kc, const void* vc, const int
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_limit_ns = kWaitLimitNs;
   p.block_table = pg ? pg->block_table : nullptr;
-  p.k_pool = pg ? static_cast<const char*>(kc) : nullptr;
-  p.v_pool = pg ? static_cast<const char*>(vc) : nullptr;
-  p.num_pages = pg ? pg->num_pages : 0;
   p.max_pages = pg ? pg->max_pages : 0;
   int shift = 0;
   while (pg && (1 << shift) < pg->page_size) ++shift;
   p.page_shift = shift;
+  p.rows_main = box_main;
+  p.rows_tail = box_tail;
+  p.interleaved = interleaved ? 1 : 0;
   p.chunk_align = pg ? fa::kDecBN : 1;
   const int grid = p.n_items < num_sms ? p.n_items : num_sms;
   fa::fa_decode_split_kernel<D, G><<<grid, fa::kDecThreads, fa::DecodeLayout<D>::kBytes,
@@ -391,11 +416,14 @@ __global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict_
 // Backward: per-device shared-memory opt-in.
 std::once_flag g_bwd_once[kMaxDevices];
 cudaError_t g_bwd_err[kMaxDevices];
+int g_bwd_sms[kMaxDevices];
 
 cudaError_t prepare_backward(int dev) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::call_once(g_bwd_once[dev], [dev] {
-    cudaError_t e = cudaFuncSetAttribute(fa::fa_bwd_kernel<64>,
+    cudaError_t e = cudaDeviceGetAttribute(&g_bwd_sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fa::fa_bwd_kernel<64>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          fa::BwdLayout<64>::kBytes);
     if (e == cudaSuccess)
@@ -444,6 +472,8 @@ fa_status launch_backward(const void* q, const void* k, const void* v, const voi
     p.causal = causal ? 1 : 0;
     p.n_kv_tiles = n_kv_tiles;
     p.n_q_tiles = (Sq + fa::kBwdBN - 1) / fa::kBwdBN;
+    // about two waves of CTAs per group (one CTA per SM)
+    p.heads_per_group = std::max(1, std::min(B * Hkv, 2 * g_bwd_sms[dev] / n_kv_tiles));
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.wait_limit_ns = kWaitLimitNs;

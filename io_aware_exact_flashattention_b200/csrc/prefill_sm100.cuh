@@ -19,14 +19,18 @@
 //   warp  9    MMA issuer: S_w = Q_w K_j^T and O_w += P_w V_j on tcgen05
 //   warps 10-11 idle
 // Registers are moved from the third warpgroup to the softmax warpgroups
-// (setmaxnreg): 208 + 208 + 88 per SM sub-partition = 3 x 168 at launch.
+// (setmaxnreg): 216 + 216 + 72 per SM sub-partition = 3 x 168 at launch.
+// Both shares are the smallest that compile without spills (the MMA issuer
+// adds descriptor offsets inside its instruction sequences to fit in 72).
 // Tensor memory (512 columns x 128 lanes x 32 bit):
 //   [0,128)   S_0 (fp32 scores); P_0 (bf16) overwrites its first 64 columns
 //   [128,256) S_1 / P_1
 //   [256, 256+D) O_0 accumulator, then O_1
 // Online softmax ("FlashAttention & IO-aware attention", section "Direct
 // answer"): each row keeps a running max m and sum l; when the max grows the
-// accumulated l and O are multiplied by e^(m - m_new).  Here the reference max
+// accumulated l and O are multiplied by e^(m - m_new).  Two sums are kept:
+// l of the fp32 weights for the LSE, and lq of the bf16-rounded weights that
+// P.V multiplies, by which O is divided.  Here the reference max
 // only moves when it grows by more than 2^24 in the exponent, so the rescale
 // of O (a round trip of O through registers) is rare even for logits spread
 // over tens of binades; the result is unchanged because the final O / l and
@@ -61,8 +65,8 @@ constexpr int kBM = 128;       // query rows per tile (= TMEM lanes)
 constexpr int kBN = 128;       // keys per key/value tile
 constexpr int kPrefillThreads = 384;
 constexpr int kPrefillLaunchRegs = 168;   // 65536 / 384, rounded down to a multiple of 8
-constexpr int kSoftmaxRegs = 208;
-constexpr int kControlRegs = 88;
+constexpr int kSoftmaxRegs = 216;
+constexpr int kControlRegs = 72;
 static_assert(2 * kSoftmaxRegs + kControlRegs <= 3 * kPrefillLaunchRegs,
               "register split exceeds the launch budget");
 constexpr int kSwzBytes = 128 * 128;  // one 128-row x 64-element bf16 box, 128B swizzled
@@ -117,6 +121,33 @@ __device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// mma_ss_f8 / mma_ts_f8 with descriptors as a base plus an offset in 16-byte
+// units added inside the instruction sequence (see mma_ss_off).
+template <uint32_t kAOff, uint32_t kBOff>
+__device__ __forceinline__ void mma_ss_f8_off(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 a, b;\n\t"
+      "add.s64 a, %1, %5;\n\t"
+      "add.s64 b, %2, %6;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(kAOff),
+        "n"(kBOff)
+      : "memory");
+}
+template <uint32_t kBOff>
+__device__ __forceinline__ void mma_ts_f8_off(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 b;\n\t"
+      "add.s64 b, %2, %5;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], b, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(kBOff)
+      : "memory");
+}
+
 // D[tmem] (+)= A[tmem] * B[smem], kind::f8f6f4; A is read from tensor memory.
 __device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                           uint32_t idesc, uint32_t accumulate) {
@@ -146,6 +177,15 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
       "mov.b32 %0, {lo, hi};\n\t}"
       : "=r"(r) : "f"(a), "f"(b), "f"(c), "f"(d));
   return r;
+}
+
+// Calls f(std::integral_constant<int, i>{}) for i = 0 .. N-1.
+template <int N, int I = 0, typename F>
+__device__ __forceinline__ void static_for(F&& f) {
+  if constexpr (I < N) {
+    f(std::integral_constant<int, I>{});
+    static_for<N, I + 1>(f);
+  }
 }
 
 struct PrefillParams {
@@ -278,7 +318,8 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
   const int last_key = static_cast<int>(min(last_key_ll, static_cast<long long>(p.Skv) - 1));
 
   float m = -INFINITY;
-  float l = 0.f;
+  float l = 0.f;   // sum of the fp32 weights: the LSE's
+  float lq = 0.f;  // sum of the weights as P.V sees them (bf16): O's normaliser
   const size_t bh = static_cast<size_t>(item.b) * p.Hq + item.h;
   const size_t o_index = bh * p.o_rows + (row - p.o_row0);
   const size_t lse_index = bh * p.lse_rows + (row - p.lse_row0);
@@ -338,6 +379,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
     if ((m_new - m) * c > kThreshold) {  // false while both are -inf (NaN)
       alpha = ex2((m - m_new) * c);              // 0 when m was -inf
       l *= alpha;
+      lq *= alpha;
       m = m_new;
     }
     const bool rescale_o = (j > 0) && __any_sync(0xffffffffu, alpha != 1.f);
@@ -365,6 +407,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
     const float2 nmc2 = make_float2(nmc, nmc);
     float2 rs[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                     make_float2(0.f, 0.f)};
+    float2 rq[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
     // Masked tiles take every exponential on the MUFU (2^-inf is exactly 0);
     // the others move kPolyPairsPer8 of every 8 pairs to the FMA pipe.
     auto exps_half = [&](auto poly_tag, int half) {
@@ -402,6 +445,9 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
                               : make_float2(ex2(x.x), ex2(x.y));
         rs[i & 3] = fadd2(rs[i & 3], pp);
         pk[i] = pack_bf16x2(pp.x, pp.y);
+        // the pair as the tensor core reads it (bf16 -> fp32 is exact)
+        rq[i & 1] = fadd2(rq[i & 1], make_float2(__uint_as_float(pk[i] << 16),
+                                                 __uint_as_float(pk[i] & 0xffff0000u)));
       }
       tmem_st32(tS + half * 32, pk);
       tmem_st_wait();
@@ -420,6 +466,8 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
     {
       const float2 t2 = fadd2(fadd2(rs[0], rs[1]), fadd2(rs[2], rs[3]));
       l += t2.x + t2.y;
+      const float2 q2 = fadd2(rq[0], rq[1]);
+      lq += q2.x + q2.y;
     }
   }
 
@@ -428,7 +476,14 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
   ++ocount;
   if (!__all_sync(0xffffffffu, ok)) return;
   tc_fence_after();
-  const float inv_l = (l > 0.f) ? o_factor / l : 0.f;
+  // O is divided by the sum of the very weights P.V used (the bf16-rounded
+  // ones), so a weight's rounding moves numerator and denominator alike: a
+  // row dominated by one key gets that key's value almost exactly, which an
+  // fp32 normaliser misses by up to half a bf16 ulp of the dominant weight.
+  // 8-bit P keeps the fp32 normaliser (its rounding is covered by the E4M3
+  // error bound).  The LSE always uses the fp32 sum.
+  const float l_o = kF8 ? l : lq;
+  const float inv_l = (l_o > 0.f) ? o_factor / l_o : 0.f;
   {
     uint32_t r[D];
     tmem_ld_row<D>(tO, r);
@@ -536,40 +591,49 @@ __device__ __forceinline__ void prefill_mma(const PrefillParams& p, uint32_t sba
     return mbar_wait(bars + 8 * (L::kBarKvFull + kv_stage(idx)),
                      static_cast<uint32_t>(idx / L::kStages) & 1u, abort_flag, p.wait_limit_ns);
   };
+  // Shared-memory descriptors are formed once; a descriptor of the same
+  // layout at a byte offset o is the base plus o / 16 (the start address
+  // field holds address / 16 and never carries: shared addresses are below
+  // 2^18).  Keeping one 64-bit base per operand keeps this thread's register
+  // count inside the control warpgroup's share.
+  const uint64_t q_desc0 = sw128_desc(sbase + L::kQOff, 16, 1024);
+  const uint64_t k_desc0 = sw128_desc(sbase + L::kRingOff, 16, 1024);
+  const uint64_t v_desc0 = sw128_desc(sbase + L::kRingOff, kSwzBytes, 1024);
   // S_w = Q_w K^T: M=128 rows, N=128 keys, K=D in steps of 32 bytes (16 bf16
   // or 32 E4M3 elements).
   auto issue_s = [&](int w, int stage) {
-    const uint32_t qa = sbase + L::kQOff + w * L::kTileBytes;
-    const uint32_t ka = sbase + L::kRingOff + stage * L::kTileBytes;
-#pragma unroll
-    for (int kk = 0; kk < L::kRowBytes / 32; ++kk) {
-      const uint32_t o = (kk >> 2) * kSwzBytes + (kk & 3) * 32;
+    const uint64_t qd = q_desc0 + static_cast<uint64_t>((w * L::kTileBytes) >> 4);
+    const uint64_t kd = k_desc0 + static_cast<uint64_t>((stage * L::kTileBytes) >> 4);
+    auto step = [&](auto kk_c) {
+      constexpr int kk = decltype(kk_c)::value;
+      constexpr uint32_t o = static_cast<uint32_t>(((kk >> 2) * kSwzBytes + (kk & 3) * 32) >> 4);
       if constexpr (kF8)
-        mma_ss_f8(tmem + w * 128, sw128_desc(qa + o, 16, 1024), sw128_desc(ka + o, 16, 1024),
-                  kIdS, kk > 0 ? 1u : 0u);
+        mma_ss_f8_off<o, o>(tmem + w * 128, qd, kd, kIdS, kk > 0 ? 1u : 0u);
       else
-        mma_ss(tmem + w * 128, sw128_desc(qa + o, 16, 1024), sw128_desc(ka + o, 16, 1024), kIdS,
-               kk > 0 ? 1u : 0u);
-    }
+        mma_ss_off<o, o>(tmem + w * 128, qd, kd, kIdS, kk > 0 ? 1u : 0u);
+    };
+    static_for<L::kRowBytes / 32>(step);
   };
   // O_w += P_w V: A = P_w in TMEM (8 columns per MMA: 16 bf16 or 32 E4M3
   // keys), B = V tile (keys x D, D contiguous: MN-major; bf16 d = 128 has two
   // 64-element column blocks 16 KB apart).  Issued per half of the keys, each
   // after its half of P is announced.
   auto issue_pv_half = [&](int w, int stage, int half, bool accumulate) {
-    const uint32_t va = sbase + L::kRingOff + stage * L::kTileBytes;
+    const uint64_t vd0 = v_desc0 + static_cast<uint64_t>((stage * L::kTileBytes) >> 4);
     constexpr int kSteps = (kBN / 2) / kKeysPerMma;
-#pragma unroll
-    for (int k4 = 0; k4 < kSteps; ++k4) {
+    const uint64_t vdh = vd0 + static_cast<uint64_t>((half * kSteps * kKeysPerMma * 128) >> 4);
+    auto step = [&](auto k4_c) {
+      constexpr int k4 = decltype(k4_c)::value;
+      constexpr uint32_t o = static_cast<uint32_t>((k4 * kKeysPerMma * 128) >> 4);
       const int kk = half * kSteps + k4;
-      const uint64_t vd = sw128_desc(va + kk * kKeysPerMma * 128, kSwzBytes, 1024);
       if constexpr (kF8)
-        mma_ts_f8(tmem + 256 + w * D, tmem + w * 128 + kk * 8, vd, kIdPV,
-                  (accumulate || kk > 0) ? 1u : 0u);
+        mma_ts_f8_off<o>(tmem + 256 + w * D, tmem + w * 128 + kk * 8, vdh, kIdPV,
+                         (accumulate || kk > 0) ? 1u : 0u);
       else
-        mma_ts(tmem + 256 + w * D, tmem + w * 128 + kk * 8, vd, kIdPV,
-               (accumulate || kk > 0) ? 1u : 0u);
-    }
+        mma_ts_off<o>(tmem + 256 + w * D, tmem + w * 128 + kk * 8, vdh, kIdPV,
+                      (accumulate || kk > 0) ? 1u : 0u);
+    };
+    static_for<kSteps>(step);
   };
   auto wait_p = [&](int w, int half, uint32_t cnt) -> bool {
     if (!mbar_wait(bars + 8 * (L::kBarPFull + 2 * w + half), cnt & 1u,
