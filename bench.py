@@ -227,10 +227,14 @@ def barrier(world):
         dist.barrier()
 
 
-def timed_calls(fn, steps, warmup, flush, stream, world):
+def timed_calls(fn, steps, warmup, flush, stream, world, settle_s=1.0):
     """Run `fn` `warmup` times, then `steps` times with L2 flushed before each
     call (outside the timed region); return the total CUDA-event milliseconds
-    of the timed calls, max over ranks."""
+    of the timed calls, max over ranks.  Each side measurement starts after
+    `settle_s` seconds idle, so it does not inherit the power-capped clocks
+    of the long step before it."""
+    torch.cuda.synchronize()
+    time.sleep(settle_s)
     for _ in range(max(warmup, 1)):
         fn()
     torch.cuda.synchronize()
@@ -437,13 +441,18 @@ def run_ours(args, world, rank, local):
             qs, ks, vs = prefill_inputs(cs.B, cs.Hq, cs.Hkv, cs.Sq, cs.Skv, cs.d,
                                         rank_seed(cs.seed, rank), cs.q_mult, device=dev)
             os_, ls_ = torch.empty_like(qs), torch.empty((cs.B, cs.Hq, cs.Sq), device=dev)
-            ms = timed_calls(lambda: fa.fa_fwd(qs, ks, vs, os_, ls_, cs.causal, cs.scale,
-                                               stream=stream), K, args.warmup, flush, stream, world)
+            torch.cuda.synchronize()
+            time.sleep(1.0)  # idle first: the step before ran power-capped
+            with ClockSampler(local) as sclk:
+                ms = timed_calls(lambda: fa.fa_fwd(qs, ks, vs, os_, ls_, cs.causal, cs.scale,
+                                                   stream=stream), K, args.warmup, flush, stream,
+                                 world, settle_s=0.0)
             tf = cs.flops() / (ms * 1e-3 / K) / 1e12
             side[name] = dict({"tflops": aggregate_rate(world, cs.flops(), K, ms) / 1e12,
                                "ms_per_launch": ms / K, "flops_per_launch": cs.flops(),
                                "B": cs.B, "Hq": cs.Hq, "Hkv": cs.Hkv, "S": cs.Sq, "d": cs.d,
-                               "causal": cs.causal, "q_mult": cs.q_mult},
+                               "causal": cs.causal, "q_mult": cs.q_mult,
+                               "clocks": sclk.summary()},
                               **tensor_fracs(tf, peaks))
             del qs, ks, vs, os_, ls_
 

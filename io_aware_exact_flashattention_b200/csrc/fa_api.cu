@@ -21,6 +21,9 @@
 namespace {
 
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s per mbarrier wait
+// Backward CTA order: groups of (batch, kv-head) pairs worth this many waves
+// of CTAs (see bwd_cta).
+constexpr int kBwdGroupWaves = 4;
 constexpr int kMaxDevices = 64;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -472,8 +475,9 @@ fa_status launch_backward(const void* q, const void* k, const void* v, const voi
     p.causal = causal ? 1 : 0;
     p.n_kv_tiles = n_kv_tiles;
     p.n_q_tiles = (Sq + fa::kBwdBN - 1) / fa::kBwdBN;
-    // about two waves of CTAs per group (one CTA per SM)
-    p.heads_per_group = std::max(1, std::min(B * Hkv, 2 * g_bwd_sms[dev] / n_kv_tiles));
+    // about kBwdGroupWaves waves of CTAs per group (one CTA per SM)
+    p.heads_per_group =
+        std::max(1, std::min(B * Hkv, kBwdGroupWaves * g_bwd_sms[dev] / n_kv_tiles));
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.wait_limit_ns = kWaitLimitNs;
@@ -490,15 +494,29 @@ fa_status launch_backward(const void* q, const void* k, const void* v, const voi
 // Feed-forward network after attention: per-device shared-memory opt-in.
 std::once_flag g_ffn_once[kMaxDevices];
 cudaError_t g_ffn_err[kMaxDevices];
+int g_ffn_sms[kMaxDevices];
 
 cudaError_t prepare_ffn(int dev) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::call_once(g_ffn_once[dev], [dev] {
-    g_ffn_err[dev] = cudaFuncSetAttribute(fa::fa_ffn_gemm_kernel,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          fa::FfnLayout::kBytes);
+    cudaError_t e = cudaDeviceGetAttribute(&g_ffn_sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fa::fa_ffn_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::FfnLayout::kBytes);
+    g_ffn_err[dev] = e;
   });
   return g_ffn_err[dev];
+}
+
+// One persistent launch of the feed-forward GEMM over row_tiles query tiles
+// (one CTA per SM, at most one per output tile).
+void launch_ffn(const CUtensorMap& tm_a, const CUtensorMap& tm_b, fa::FfnParams p, int row_tiles,
+                int dev, cudaStream_t s) {
+  p.n_row_tiles = row_tiles;
+  const int tiles = row_tiles * (p.N / fa::kFfnBN);
+  const int grid = std::max(1, std::min(tiles, g_ffn_sms[dev]));
+  fa::fa_ffn_gemm_kernel<<<static_cast<unsigned>(grid), fa::kFfnThreads, fa::FfnLayout::kBytes,
+                           s>>>(tm_a, tm_b, p);
 }
 
 extern "C" {
@@ -654,10 +672,8 @@ fa_status fa_bpt_ffn(const void* o, const void* w1, const void* w2, void* y,
   for (long long mt0 = 0; mt0 < total_tiles; mt0 += chunk_tiles) {
     const int n = static_cast<int>(std::min<long long>(chunk_tiles, total_tiles - mt0));
     p1.mt0 = p2.mt0 = static_cast<int>(mt0);
-    fa::fa_ffn_gemm_kernel<<<dim3(static_cast<unsigned>(F / fa::kFfnBN), static_cast<unsigned>(n)),
-                             fa::kFfnThreads, fa::FfnLayout::kBytes, s>>>(tm_o, tm_w1, p1);
-    fa::fa_ffn_gemm_kernel<<<dim3(static_cast<unsigned>(D / fa::kFfnBN), static_cast<unsigned>(n)),
-                             fa::kFfnThreads, fa::FfnLayout::kBytes, s>>>(tm_h, tm_w2, p2);
+    launch_ffn(tm_o, tm_w1, p1, n, dev, s);
+    launch_ffn(tm_h, tm_w2, p2, n, dev, s);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   return FA_OK;
@@ -746,11 +762,8 @@ fa_status fa_bpt_layer(const void* q, const void* k, const void* v, const void* 
     p2.a_heads = 0;
     p2.c_tokens = 1;
     p2.gelu = 0;
-    const unsigned gy = static_cast<unsigned>(B * tiles);
-    fa::fa_ffn_gemm_kernel<<<dim3(static_cast<unsigned>(F / fa::kFfnBN), gy), fa::kFfnThreads,
-                             fa::FfnLayout::kBytes, s>>>(tm_o, tm_w1, p1);
-    fa::fa_ffn_gemm_kernel<<<dim3(static_cast<unsigned>(D / fa::kFfnBN), gy), fa::kFfnThreads,
-                             fa::FfnLayout::kBytes, s>>>(tm_h, tm_w2, p2);
+    launch_ffn(tm_o, tm_w1, p1, B * tiles, dev, s);
+    launch_ffn(tm_h, tm_w2, p2, B * tiles, dev, s);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   return FA_OK;

@@ -22,7 +22,10 @@
 //
 // Roles (192 threads): warps 0-3 epilogue (thread = row = TMEM lane), warp 4
 // TMA producer (4-stage ring of A and B boxes), warp 5 MMA issuer and TMEM
-// owner.  Every mbarrier wait is bounded (see mbar_wait).
+// owner.  The kernel is persistent (one CTA per SM over the launch's output
+// tiles) with two accumulators in tensor memory, so a tile's epilogue
+// overlaps the next tile's products.  Every mbarrier wait is bounded (see
+// mbar_wait).
 #pragma once
 
 #include <cuda.h>
@@ -41,11 +44,12 @@ struct FfnLayout {
   static constexpr int kBBytes = kFfnBN * kFfnBK * 2;     // 32 KB
   static constexpr int kStageBytes = kABytes + kBBytes;   // 48 KB
   static constexpr int kBarOff = kFfnStages * kStageBytes;
-  // full[S], empty[S], acc_full, done
+  // full[S], empty[S], acc_full[2], acc_empty[2], done
   static constexpr int kBarFull = 0;
   static constexpr int kBarEmpty = kFfnStages;
-  static constexpr int kBarAcc = 2 * kFfnStages;
-  static constexpr int kBarDone = kBarAcc + 1;
+  static constexpr int kBarAccFull = 2 * kFfnStages;
+  static constexpr int kBarAccEmpty = kBarAccFull + 2;
+  static constexpr int kBarDone = kBarAccEmpty + 2;
   static constexpr int kNumBars = kBarDone + 1;
   static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kAbortOff = kTmemSlotOff + 4;
@@ -59,6 +63,7 @@ struct FfnParams {
   int Hq, d;          // geometry of the attention output (first product)
   int tiles_per_seq;  // ceil(S / 128)
   int mt0;            // first query tile (over all sequences) of this launch
+  int n_row_tiles;    // query tiles of this launch
   int a_heads;        // 1: A = attention output [B*Hq, S, d]; 0: A = chunk scratch [rows, K]
   int c_tokens;       // 1: C row = token b*S_out + tok0 + t; 0: C row = chunk-local row
   int S_out, tok0;    // tokens per sequence of C and the token of A's row 0 (c_tokens)
@@ -70,6 +75,28 @@ __device__ __forceinline__ float gelu_erf(float x) {
   return 0.5f * x * (1.f + erff(x * 0.70710678118654752f));
 }
 
+// Output tile t of a launch: row tile t / (N/256) (a query tile), column
+// tile t % (N/256); the column tiles of one row tile are adjacent, so CTAs
+// running together share their A rows in L2.
+struct FfnTile {
+  int n0, local_row0, b, t0;
+};
+__device__ __forceinline__ FfnTile ffn_tile(const FfnParams& p, int t) {
+  FfnTile f;
+  const int n_col = p.N / kFfnBN;
+  const int rt = t / n_col;
+  f.n0 = (t % n_col) * kFfnBN;
+  f.local_row0 = rt * kFfnBM;
+  const int g = p.mt0 + rt;
+  f.b = g / p.tiles_per_seq;
+  f.t0 = (g % p.tiles_per_seq) * kFfnBM;
+  return f;
+}
+
+// Persistent: one CTA per SM walks the launch's output tiles round-robin.
+// Two tensor-memory accumulators (256 columns each) alternate between tiles,
+// so the epilogue of one tile (TMEM read-out, GELU, stores) runs while the
+// next tile's products accumulate.
 __global__ void __launch_bounds__(kFfnThreads, 1)
 fa_ffn_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
                    const __grid_constant__ CUtensorMap tm_b, const FfnParams p) {
@@ -83,13 +110,7 @@ fa_ffn_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbortOff);
-
-  // this CTA's tile: output columns [n0, n0 + 256) of query tile g
-  const int n0 = static_cast<int>(blockIdx.x) * kFfnBN;
-  const int local_row0 = static_cast<int>(blockIdx.y) * kFfnBM;
-  const int g = p.mt0 + static_cast<int>(blockIdx.y);
-  const int b = g / p.tiles_per_seq;
-  const int t0 = (g % p.tiles_per_seq) * kFfnBM;
+  const int n_tiles = p.n_row_tiles * (p.N / kFfnBN);
   const int nk = p.K / kFfnBK;
 
   if (threadIdx.x == 0) {
@@ -97,13 +118,16 @@ fa_ffn_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
       mbar_init(bars + 8 * (L::kBarFull + s), 1);
       mbar_init(bars + 8 * (L::kBarEmpty + s), 1);
     }
-    mbar_init(bars + 8 * L::kBarAcc, 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bars + 8 * (L::kBarAccFull + a), 1);
+      mbar_init(bars + 8 * (L::kBarAccEmpty + a), 4);  // one arrival per epilogue warp
+    }
     mbar_init(bars + 8 * L::kBarDone, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 5) {
-    tmem_alloc(sbase + L::kTmemSlotOff, kFfnBN);
+    tmem_alloc(sbase + L::kTmemSlotOff, 2 * kFfnBN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -113,51 +137,70 @@ fa_ffn_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
 
   if (warp == 4) {
     if (lane == 0) {
-      // producer: A and B boxes of each K step into the ring
+      // producer: A and B boxes of every K step of every tile into the ring
       tma_prefetch_desc(&tm_a);
       tma_prefetch_desc(&tm_b);
-      int issued = 0;
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % kFfnStages;
-        if (!mbar_wait(bars + 8 * (L::kBarEmpty + s), ((kb / kFfnStages) & 1) ^ 1, abort_flag,
-                       p.wait_limit_ns))
-          break;
-        const uint32_t full = bars + 8 * (L::kBarFull + s);
-        const uint32_t sa = sbase + s * L::kStageBytes;
-        mbar_arrive_expect_tx(full, L::kStageBytes);
-        const int k0 = kb * kFfnBK;
-        if (p.a_heads)
-          tma_load_3d(sa, &tm_a, full, k0 % p.d, t0, b * p.Hq + k0 / p.d);
-        else
-          tma_load_3d(sa, &tm_a, full, k0, local_row0, 0);
-        tma_load_3d(sa + L::kABytes, &tm_b, full, k0, n0, 0);
-        ++issued;
+      uint32_t issued = 0;
+      bool stop = false;
+      for (int t = blockIdx.x; t < n_tiles && !stop; t += gridDim.x) {
+        const FfnTile f = ffn_tile(p, t);
+        for (int kb = 0; kb < nk; ++kb, ++issued) {
+          const uint32_t s = issued % kFfnStages;
+          if (!mbar_wait(bars + 8 * (L::kBarEmpty + s), ((issued / kFfnStages) & 1u) ^ 1u,
+                         abort_flag, p.wait_limit_ns)) {
+            stop = true;
+            break;
+          }
+          const uint32_t full = bars + 8 * (L::kBarFull + s);
+          const uint32_t sa = sbase + s * L::kStageBytes;
+          mbar_arrive_expect_tx(full, L::kStageBytes);
+          const int k0 = kb * kFfnBK;
+          if (p.a_heads)
+            tma_load_3d(sa, &tm_a, full, k0 % p.d, f.t0, f.b * p.Hq + k0 / p.d);
+          else
+            tma_load_3d(sa, &tm_a, full, k0, f.local_row0, 0);
+          tma_load_3d(sa + L::kABytes, &tm_b, full, k0, f.n0, 0);
+        }
       }
       // drain: no copy may still be in flight when the CTA exits
-      for (int kb = (issued > kFfnStages ? issued - kFfnStages : 0); kb < issued; ++kb)
-        mbar_wait(bars + 8 * (L::kBarFull + kb % kFfnStages), (kb / kFfnStages) & 1, nullptr,
-                  p.wait_limit_ns);
+      const uint32_t S = kFfnStages;
+      for (uint32_t k = (issued > S ? issued - S : 0u); k < issued; ++k)
+        mbar_wait(bars + 8 * (L::kBarFull + k % S), (k / S) & 1u, nullptr, p.wait_limit_ns);
     }
   } else if (warp == 5) {
     if (lane == 0) {
-      // MMA issuer: acc[128 x 256] (+)= A_k B_k^T, four K = 16 steps per stage
+      // MMA issuer: acc[i & 1] [128 x 256] (+)= A_k B_k^T, four K = 16 steps per stage
       constexpr uint32_t kId = idesc_bf16_f32(kFfnBM, kFfnBN, false);
-      bool ok = true;
-      for (int kb = 0; kb < nk && ok; ++kb) {
-        const int s = kb % kFfnStages;
-        ok = mbar_wait(bars + 8 * (L::kBarFull + s), (kb / kFfnStages) & 1, abort_flag,
-                       p.wait_limit_ns);
-        if (!ok) break;
+      const uint64_t a_desc0 = sw128_desc(sbase, 16, 1024);
+      const uint64_t b_desc0 = sw128_desc(sbase + L::kABytes, 16, 1024);
+      uint32_t used = 0;  // ring stages consumed
+      int i = 0;          // tiles of this CTA
+      for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
+        const uint32_t acc = static_cast<uint32_t>(i & 1);
+        // the accumulator is free once the epilogue has read the tile two back
+        if (!mbar_wait(bars + 8 * (L::kBarAccEmpty + acc), ((i >> 1) & 1) ^ 1, abort_flag,
+                       p.wait_limit_ns))
+          break;
         tc_fence_after();
-        const uint32_t sa = sbase + s * L::kStageBytes;
-        const uint32_t sb = sa + L::kABytes;
-#pragma unroll
-        for (int kk = 0; kk < kFfnBK / 16; ++kk)
-          mma_ss(tmem, sw128_desc(sa + kk * 32, 16, 1024), sw128_desc(sb + kk * 32, 16, 1024), kId,
-                 (kb > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bars + 8 * (L::kBarEmpty + s));
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb, ++used) {
+          const uint32_t s = used % kFfnStages;
+          ok = mbar_wait(bars + 8 * (L::kBarFull + s), (used / kFfnStages) & 1u, abort_flag,
+                         p.wait_limit_ns);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t so = static_cast<uint64_t>((s * L::kStageBytes) >> 4);
+          const uint64_t ad = a_desc0 + so, bd = b_desc0 + so;
+          const uint32_t d = tmem + acc * kFfnBN;
+          mma_ss_off<0, 0>(d, ad, bd, kId, kb > 0 ? 1u : 0u);
+          mma_ss_off<2, 2>(d, ad, bd, kId, 1u);
+          mma_ss_off<4, 4>(d, ad, bd, kId, 1u);
+          mma_ss_off<6, 6>(d, ad, bd, kId, 1u);
+          mma_commit(bars + 8 * (L::kBarEmpty + s));
+        }
+        if (!ok) break;
+        mma_commit(bars + 8 * (L::kBarAccFull + acc));
       }
-      if (ok) mma_commit(bars + 8 * L::kBarAcc);
       // every MMA this thread issued completes before tensor memory is freed
       mma_commit(bars + 8 * L::kBarDone);
       mbar_wait(bars + 8 * L::kBarDone, 0u, nullptr, p.wait_limit_ns);
@@ -166,17 +209,23 @@ fa_ffn_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
     // epilogue: row r of the tile, 32 columns per TMEM load
     const int r = threadIdx.x;  // warps 0-3: TMEM lanes 0-127
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const bool ok = mbar_wait(bars + 8 * L::kBarAcc, 0u, abort_flag, p.wait_limit_ns);
-    if (__all_sync(0xffffffffu, ok)) {
+    int i = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
+      const FfnTile f = ffn_tile(p, t);
+      const uint32_t acc = static_cast<uint32_t>(i & 1);
+      const bool ok = mbar_wait(bars + 8 * (L::kBarAccFull + acc), (i >> 1) & 1, abort_flag,
+                                p.wait_limit_ns);
+      if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const bool valid = t0 + r < p.S;
-      const long long row = p.c_tokens ? static_cast<long long>(b) * p.S_out + p.tok0 + t0 + r
-                                       : static_cast<long long>(local_row0) + r;
-      uint4* dst = reinterpret_cast<uint4*>(p.c + row * p.N + n0);
+      const bool valid = f.t0 + r < p.S;
+      const long long row = p.c_tokens
+                                ? static_cast<long long>(f.b) * p.S_out + p.tok0 + f.t0 + r
+                                : static_cast<long long>(f.local_row0) + r;
+      uint4* dst = reinterpret_cast<uint4*>(p.c + row * p.N + f.n0);
 #pragma unroll 1
       for (int c = 0; c < kFfnBN / 32; ++c) {
         uint32_t v[32];
-        tmem_ld32(tmem + lane_off + static_cast<uint32_t>(c * 32), v);
+        tmem_ld32(tmem + lane_off + acc * kFfnBN + static_cast<uint32_t>(c * 32), v);
         uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -193,6 +242,10 @@ fa_ffn_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
             dst[4 * c + q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
         }
       }
+      // this warp's reads of the accumulator are done: hand it back
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + 8 * (L::kBarAccEmpty + acc));
     }
   }
 
@@ -201,7 +254,7 @@ fa_ffn_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
   if (warp == 5) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, kFfnBN);
+    tmem_dealloc(tmem, 2 * kFfnBN);
   }
 }
 

@@ -445,9 +445,8 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
                               : make_float2(ex2(x.x), ex2(x.y));
         rs[i & 3] = fadd2(rs[i & 3], pp);
         pk[i] = pack_bf16x2(pp.x, pp.y);
-        // the pair as the tensor core reads it (bf16 -> fp32 is exact)
-        rq[i & 1] = fadd2(rq[i & 1], make_float2(__uint_as_float(pk[i] << 16),
-                                                 __uint_as_float(pk[i] & 0xffff0000u)));
+        // the pair as the tensor core reads it, added straight from bf16
+        add_bf16x2_to(rq[i & 1], pk[i]);
       }
       tmem_st32(tS + half * 32, pk);
       tmem_st_wait();
@@ -456,7 +455,8 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams& p, uint32_t
       __syncwarp();
       if ((threadIdx.x & 31) == 0) mbar_arrive(bar_p + 8 * half);
     };
-    if (tile_masked) {
+    // (with no polynomial share the two variants would be the same code twice)
+    if (tile_masked || (kF8 ? kPolyPairsPer8F8 : kPolyPairsPer8) == 0) {
       exps_half(std::false_type{}, 0);
       exps_half(std::false_type{}, 1);
     } else {

@@ -366,6 +366,8 @@ __device__ __forceinline__ void tmem_ld_row(uint32_t taddr, uint32_t (&r)[D]);
 template <>
 __device__ __forceinline__ void tmem_ld_row<128>(uint32_t taddr, uint32_t (&r)[128]) { tmem_ld128(taddr, r); }
 template <>
+__device__ __forceinline__ void tmem_ld_row<32>(uint32_t taddr, uint32_t (&r)[32]) { tmem_ld32(taddr, r); }
+template <>
 __device__ __forceinline__ void tmem_ld_row<64>(uint32_t taddr, uint32_t (&r)[64]) {
   tmem_ld64_nowait(taddr, r);
   tmem_ld_wait_hold(r);
@@ -410,6 +412,14 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
+}
+
+// acc.x += lo half of pk, acc.y += hi half, the bf16 halves taken exactly
+// (mixed-precision add: bf16 operand, fp32 accumulate and result).
+__device__ __forceinline__ void add_bf16x2_to(float2& acc, uint32_t pk) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+      : "+f"(acc.x), "+f"(acc.y) : "r"(pk));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
