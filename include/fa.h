@@ -134,21 +134,25 @@ fa_status fa_fwd_fp8(const void *q, const void *k, const void *v, const float *d
  *   q, o, d_o, dq [B, Hq, Sq, d] bf16     k, v, dk, dv [B, Hkv, Skv, d] bf16
  *   lse           [B, Hq, Sq] fp32 (natural log, as fa_fwd writes it)
  *   workspace     fa_bwd_workspace_bytes(B, Hq, Sq, d) bytes, 16-byte aligned,
- *                 caller-owned scratch (fp32 dq accumulator, then D); its
- *                 contents on entry do not matter
+ *                 caller-owned scratch (D per query row, fp32); its contents
+ *                 on entry do not matter
  *   causal, scale: as passed to fa_fwd.
  *
- * dq, dk, dv are written (dk = dv = 0 for keys no query sees).  P and dS
- * enter the tensor-core products as bf16; accumulation is fp32.
- * Supported: d in {64, 128}; Hq % Hkv == 0.  All pointers 16-byte aligned.
- * Errors as for fa_fwd.
+ * dq, dk, dv are written once each (dk = dv = 0 for keys no query sees, dq = 0
+ * for queries that see no key): dk, dv by a kernel with one CTA per key tile,
+ * dq by one with one CTA per query tile, each accumulating in tensor memory,
+ * so the result does not depend on scheduling.  P and dS enter the
+ * tensor-core products as bf16; accumulation is fp32.
+ * Supported: d in {64, 128}; Hq % Hkv == 0.  All pointers 16-byte aligned;
+ * k, v, dk, dv may be null when Skv = 0, and q, o, lse, d_o, dq, workspace
+ * when Sq = 0.  Errors as for fa_fwd.
  */
 fa_status fa_bwd(const void *q, const void *k, const void *v, const void *o,
                  const float *lse, const void *d_o, void *dq, void *dk, void *dv,
                  float *workspace, int B, int Hq, int Hkv, int Sq, int Skv, int d,
                  int causal, float scale, fa_stream_t stream);
 
-/* Bytes of scratch fa_bwd needs: B * Hq * Sq * (d + 1) floats (0 for empty). */
+/* Bytes of scratch fa_bwd needs: B * Hq * Sq floats (0 for empty); d is unused. */
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Sq, int d);
 
 /*

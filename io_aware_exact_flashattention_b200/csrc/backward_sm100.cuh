@@ -6,27 +6,38 @@
 // the forward's LSE, D_i = dO_i . O_i and dS = P * (dO.v - D):
 //   dV_j = sum_i P_ij dO_i,  dK_j = scale * sum_i dS_ij q_i,  dQ_i = scale * sum_j dS_ij k_j.
 //
-// One CTA per (batch, key/value head, 128-key tile j): K_j and V_j stay in
-// shared memory and dK_j, dV_j accumulate in tensor memory while the query
-// tiles of every query head of the group stream past (key-stationary loop, so
-// dK and dV are written once; dQ rows collect contributions from every key
-// tile and are added into an fp32 workspace by bulk tensor reductions).  Per
-// query tile, all on tcgen05 with fp32 accumulators in TMEM:
-//   S^T  = K_j Q_i^T      (M=128 keys, N=128 queries; SS)
-//   dP^T = V_j dO_i^T     (M=128 keys, N=128 queries; SS)
-//   dV  += P^T dO_i       (A = P^T in TMEM, B = dO_i MN-major; TS)
-//   dK  += dS^T Q_i       (A = dS^T in TMEM, B = Q_i MN-major; TS)
-//   dQ_i = dS K_j         (A = dS from shared memory MN-major, B = K_j MN-major; SS)
-// Roles (320 threads):
-//   warps 0-7  two warpgroups, each half of every tile's queries: thread =
-//              key row for P and dS (from S^T, dP^T, LSE and D); thread =
-//              query row for the dQ partial (half the d-columns each) into
-//              the workspace; dK, dV out
-//   warp  8    TMA producer: K_j, V_j once, then Q_i and dO_i (two stages)
+// Two kernels, each with its accumulators resident in tensor memory for the
+// whole loop, so that every gradient is written once, in bf16, with no
+// reductions in global memory (and the result does not depend on the order
+// in which CTAs run):
+//
+// fa_bwd_dkdv_kernel -- one CTA per (batch, key/value head, 128-key tile j).
+//   K_j and V_j stay in shared memory and dK_j, dV_j accumulate in TMEM while
+//   the query tiles of every query head of the group stream past.  Per query
+//   tile, on tcgen05 with fp32 accumulators:
+//     S^T  = K_j Q_i^T      (M=128 keys, N=128 queries; SS)
+//     dP^T = V_j dO_i^T     (M=128 keys, N=128 queries; SS)
+//     dV  += P^T dO_i       (A = P^T in TMEM, B = dO_i MN-major; TS)
+//     dK  += dS^T Q_i       (A = dS^T K-major in shared memory, B = Q_i MN-major; SS)
+//   Tensor memory columns: dV [0,128), dK [128,256), S^T / P [256,384),
+//   dP^T [384,512).
+//
+// fa_bwd_dq_kernel -- one CTA per (batch, query head, 128-query tile i).
+//   Q_i and dO_i stay in shared memory, dQ_i accumulates in TMEM while the
+//   key tiles the queries see stream past (two-stage ring):
+//     S   = Q_i K_j^T       (M=128 queries, N=128 keys; SS), two buffers
+//     dP  = dO_i V_j^T      (M=128 queries, N=128 keys; SS)
+//     dQ += dS K_j          (A = dS packed in the S buffer; B = K_j MN-major; TS)
+//   Tensor memory columns: S [0,128) and [128,256), dP [256,384), dQ [384,384+d).
+//   Against a single kernel that adds partial dQ tiles into an fp32 buffer,
+//   this recomputes S and dP once more (7 products per tile pair instead of
+//   5) but removes 64 KB of fp32 additions per tile pair, whose memory-side
+//   throughput bounded that design.
+//
+// Roles of both (320 threads):
+//   warps 0-7  two element-wise warpgroups (P, dS; the gradients out)
+//   warp  8    TMA producer
 //   warp  9    MMA issuer; allocates tensor memory
-// Tensor memory columns: dV [0,128), dK [128,256), S^T / P [256,384),
-// dP^T / dS / dQ partial [384,512).  The next tile's S^T is issued as soon as
-// dQ_i is, so it runs while dQ_i is read out; its dP^T waits for the read-out.
 #pragma once
 
 #include <cuda.h>
@@ -36,117 +47,33 @@
 namespace fa {
 
 constexpr int kBwdThreads = 320;
-constexpr int kBwdBM = 128;  // keys per CTA (TMEM lanes)
-constexpr int kBwdBN = 128;  // queries per tile
-
-template <int D>
-struct BwdLayout {
-  static constexpr int kTileBytes = 128 * D * 2;
-  static constexpr int kBoxBytes = 128 * 128;  // 128 rows x 64 bf16, 128B swizzled
-  static constexpr int kKOff = 0;
-  static constexpr int kVOff = kTileBytes;
-  static constexpr int kQOff = 2 * kTileBytes;  // stage s: Q at kQOff + 2*s*tile, dO after it
-  static constexpr int kDsOff = 6 * kTileBytes;  // dS^T: 128 keys x 128 queries bf16 (2 boxes)
-  static constexpr int kLseOff = kDsOff + 128 * 128 * 2;  // [128] LSE*log2(e), [128] D
-  static constexpr int kBarOff = kLseOff + 2 * 128 * 4;
-  static constexpr int kBKv = 0;
-  static constexpr int kBQFull = 1;    // [2]
-  static constexpr int kBQEmpty = 3;   // [2]
-  static constexpr int kBSFull = 5;
-  static constexpr int kBDpFull = 6;
-  static constexpr int kBPFull = 7;    // 8 arrivals (one per element-wise warp)
-  static constexpr int kBDsFull = 8;   // 8 arrivals
-  static constexpr int kBDqFull = 9;
-  static constexpr int kBSFree = 10;   // 8 arrivals: dQ partial read out of the dP columns
-  static constexpr int kBDone = 11;
-  static constexpr int kNumBars = 12;
-  static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
-  static constexpr int kAbortOff = kTmemSlotOff + 4;
-  static constexpr int kBytes = kAbortOff + 4 + 1024;  // + slack for 1024-byte alignment
-};
-static_assert(BwdLayout<128>::kBytes <= 232448, "backward shared memory over the limit");
+constexpr int kBwdBM = 128;  // keys per key tile
+constexpr int kBwdBN = 128;  // queries per query tile
 
 struct BwdParams {
-  float* dq_acc;       // [B, Hq, Sq, d] fp32, zeroed; receives scale * dS K
   const float* lse;    // [B, Hq, Sq] natural log
   const float* dsum;   // [B, Hq, Sq]: D = dO . O
+  __nv_bfloat16* dq;   // [B, Hq, Sq, d]
   __nv_bfloat16* dk;   // [B, Hkv, Skv, d]
   __nv_bfloat16* dv;
   int B, Hq, Hkv, Sq, Skv, group, causal;
   int n_kv_tiles, n_q_tiles;
-  int heads_per_group;  // CTA order: groups of this many (b, kv-head) pairs (see bwd_cta)
+  int heads_per_group;  // dK/dV CTA order: groups of this many (b, kv-head) pairs
   float scale, scale_log2;
   unsigned long long wait_limit_ns;
 };
 
-// First query tile that sees any key of key tile j (causal: key k is visible
-// to query q iff k <= q + Skv - Sq).
-__device__ __forceinline__ int bwd_first_q_tile(const BwdParams& p, int j) {
-  if (!p.causal) return 0;
-  const long long need = static_cast<long long>(j) * kBwdBM - (p.Skv - p.Sq);  // q >= need
-  if (need <= 0) return 0;
-  return static_cast<int>(need / kBwdBN);
-}
-
-__device__ __forceinline__ void bwd_cta(const BwdParams& p, int& b, int& g, int& j) {
-  // CTAs go out in groups of p.heads_per_group (batch, key/value head)
-  // pairs; within a group key tile by key tile, heavy tiles first (under a
-  // causal mask key tile 0 sees every query tile), so the launch order stays
-  // longest-first and the tail is short.  The CTAs resident at a time then
-  // cover about two groups, whose Q, dO and fp32 dQ rows stay in L2 while all
-  // their key tiles stream them; ordered key tile by key tile over all heads,
-  // the resident CTAs touch every head's Q, dO and dQ at once, more than L2
-  // holds.
-  const int per_group = p.heads_per_group * p.n_kv_tiles;
-  const int grp = static_cast<int>(blockIdx.x) / per_group;
-  const int r = static_cast<int>(blockIdx.x) % per_group;
-  const int units = p.B * p.Hkv;
-  const int in_group = min(p.heads_per_group, units - grp * p.heads_per_group);
-  j = r / in_group;
-  const int bg = grp * p.heads_per_group + r % in_group;
-  b = bg / p.Hkv;
-  g = bg % p.Hkv;
-}
-
-// Element-wise add of a shared-memory box into global memory (bulk reduction
-// in L2), tracked by the issuing thread's bulk-async group.
-__device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, uint32_t src, int c0, int c1,
-                                                  int c2) {
-  asm volatile(
-      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
-      " [%0, {%2, %3, %4}], [%1];"
-      ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(src), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_commit_group() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-// Wait until every committed bulk operation of this thread has completed.
-__device__ __forceinline__ void bulk_wait_group0() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-// Wait until every committed bulk operation of this thread has finished
-// reading its shared-memory source.
-__device__ __forceinline__ void bulk_wait_group_read0() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-
 // ---------------------------------------------------------------------------
-// D = rowsum(dO * O) for every query row (one warp per row); the row's fp32
-// dq accumulator is zeroed on the way.
+// D = rowsum(dO * O) for every query row (one warp per row).
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_dsum_kernel(const __nv_bfloat16* __restrict__ o,
                                                           const __nv_bfloat16* __restrict__ d_o,
                                                           float* __restrict__ dsum,
-                                                          float* __restrict__ dq_acc,
                                                           long long rows) {
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
-#pragma unroll
-  for (int c = lane * 4; c < D; c += 128)
-    *reinterpret_cast<float4*>(dq_acc + row * D + c) = make_float4(0.f, 0.f, 0.f, 0.f);
   float acc = 0.f;
 #pragma unroll
   for (int c = lane * 2; c < D; c += 64) {
@@ -160,33 +87,96 @@ __global__ void __launch_bounds__(256) fa_bwd_dsum_kernel(const __nv_bfloat16* _
   if (lane == 0) dsum[row] = acc;
 }
 
-// dq (bf16) from the fp32 workspace.
-__global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float* __restrict__ acc,
-                                                        __nv_bfloat16* __restrict__ dq,
-                                                        long long n) {
-  const long long i = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) * 4;
-  if (i >= n) return;
-  const float4 v = *reinterpret_cast<const float4*>(acc + i);
-  __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
-  __nv_bfloat162 c = __floats2bfloat162_rn(v.z, v.w);
-  uint2 w;
-  w.x = *reinterpret_cast<uint32_t*>(&a);
-  w.y = *reinterpret_cast<uint32_t*>(&c);
-  *reinterpret_cast<uint2*>(dq + i) = w;
+// Offsets (16-byte descriptor units) of K step kk in a 128B-swizzled tile.
+// K-major: rows of 64 elements, step kk at byte (kk / 4) * box + (kk % 4) * 32.
+// MN-major: 64-element column blocks one box apart (LBO), step kk at byte
+// kk * 16 rows * 128.
+__host__ __device__ constexpr uint32_t bwd_km_off(int kk) {
+  return static_cast<uint32_t>(((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4);
+}
+__host__ __device__ constexpr uint32_t bwd_mn_off(int kk) { return static_cast<uint32_t>(kk * 128); }
+
+// TMEM column of the packed bf16 pairs for elements 16*kk .. 16*kk+15 of a
+// 128-wide row whose two 64-wide halves are packed by two warpgroups, each at
+// the start of its own 64 columns.
+__host__ __device__ constexpr uint32_t bwd_packed_col(int kk) {
+  return static_cast<uint32_t>(kk * 8 + (kk >= 4 ? 32 : 0));
 }
 
-// ---------------------------------------------------------------------------
-// Producer (one thread)
-// ---------------------------------------------------------------------------
+// d_tmem = A B^T over K = D, A and B K-major 128-row tiles (descriptor bases).
 template <int D>
-__device__ __forceinline__ void bwd_producer(const CUtensorMap* tq, const CUtensorMap* tk,
-                                             const CUtensorMap* tv, const CUtensorMap* tdo,
-                                             const BwdParams& p, uint32_t sbase,
-                                             volatile int* abort_flag) {
-  using L = BwdLayout<D>;
+__device__ __forceinline__ void bwd_gemm_kmajor(uint32_t d_tmem, uint64_t a, uint64_t b) {
+  constexpr uint32_t kId = idesc_bf16_f32(128, 128, false);
+  static_for<D / 16>([&](auto kk_c) {
+    constexpr int kk = decltype(kk_c)::value;
+    mma_ss_off<bwd_km_off(kk), bwd_km_off(kk)>(d_tmem, a, b, kId, kk > 0 ? 1u : 0u);
+  });
+}
+
+// ===========================================================================
+// dK, dV: key-stationary kernel
+// ===========================================================================
+template <int D>
+struct BwdKvLayout {
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kBoxBytes = 128 * 128;  // 128 rows x 64 bf16, 128B swizzled
+  static constexpr int kKOff = 0;
+  static constexpr int kVOff = kTileBytes;
+  static constexpr int kQOff = 2 * kTileBytes;  // stage s: Q at kQOff + 2*s*tile, dO after it
+  static constexpr int kDsOff = 6 * kTileBytes;  // dS^T: 128 keys x 128 queries bf16 (2 boxes)
+  static constexpr int kLseOff = kDsOff + 128 * 128 * 2;  // [128] -LSE*log2(e), [128] D
+  static constexpr int kBarOff = kLseOff + 2 * 128 * 4;
+  static constexpr int kBKv = 0;
+  static constexpr int kBQFull = 1;    // [2]
+  static constexpr int kBQEmpty = 3;   // [2]
+  static constexpr int kBSFull = 5;
+  static constexpr int kBDpFull = 6;
+  static constexpr int kBPFull = 7;    // 8 arrivals (one per element-wise warp)
+  static constexpr int kBDsFull = 8;   // 8 arrivals
+  static constexpr int kBDone = 9;
+  static constexpr int kNumBars = 10;
+  static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
+  static constexpr int kAbortOff = kTmemSlotOff + 4;
+  static constexpr int kBytes = kAbortOff + 4 + 1024;  // + slack for 1024-byte alignment
+};
+static_assert(BwdKvLayout<128>::kBytes <= 232448, "dK/dV shared memory over the limit");
+
+// First query tile that sees any key of key tile j (causal: key k is visible
+// to query q iff k <= q + Skv - Sq).
+__device__ __forceinline__ int bwd_first_q_tile(const BwdParams& p, int j) {
+  if (!p.causal) return 0;
+  const long long need = static_cast<long long>(j) * kBwdBM - (p.Skv - p.Sq);  // q >= need
+  if (need <= 0) return 0;
+  return static_cast<int>(need / kBwdBN);
+}
+
+__device__ __forceinline__ void bwd_kv_cta(const BwdParams& p, int& b, int& g, int& j) {
+  // CTAs go out in groups of p.heads_per_group (batch, key/value head)
+  // pairs; within a group key tile by key tile, heavy tiles first (under a
+  // causal mask key tile 0 sees every query tile), so the launch order stays
+  // longest-first and the tail is short.  The CTAs resident at a time then
+  // cover about two groups, whose Q and dO rows stay in L2 while all their
+  // key tiles stream them.
+  const int per_group = p.heads_per_group * p.n_kv_tiles;
+  const int grp = static_cast<int>(blockIdx.x) / per_group;
+  const int r = static_cast<int>(blockIdx.x) % per_group;
+  const int units = p.B * p.Hkv;
+  const int in_group = min(p.heads_per_group, units - grp * p.heads_per_group);
+  j = r / in_group;
+  const int bg = grp * p.heads_per_group + r % in_group;
+  b = bg / p.Hkv;
+  g = bg % p.Hkv;
+}
+
+template <int D>
+__device__ __forceinline__ void bwd_kv_producer(const CUtensorMap* tq, const CUtensorMap* tk,
+                                                const CUtensorMap* tv, const CUtensorMap* tdo,
+                                                const BwdParams& p, uint32_t sbase,
+                                                volatile int* abort_flag) {
+  using L = BwdKvLayout<D>;
   const uint32_t bars = sbase + L::kBarOff;
   int b, g, j;
-  bwd_cta(p, b, g, j);
+  bwd_kv_cta(p, b, g, j);
   tma_prefetch_desc(tq);
   tma_prefetch_desc(tk);
   tma_prefetch_desc(tv);
@@ -223,82 +213,71 @@ drain:
     mbar_wait(bars + 8 * (L::kBQFull + (k & 1u)), (k >> 1) & 1u, nullptr, p.wait_limit_ns);
 }
 
-// ---------------------------------------------------------------------------
-// MMA issuer (one thread)
-// ---------------------------------------------------------------------------
+// Per query tile n the MMA thread issues dV_n once P_n is announced, the next
+// tile's S^T (its columns hold P_n, which dV_n reads first), then dK_n once
+// dS_n is in shared memory, and the next tile's dP^T (the element-wise warps
+// have read dP_n before announcing dS_n).  dK_n precedes dP^T_{n+1}, so the
+// commit that announces dP^T_{n+1} also covers dK_n's reads of dS_n, which
+// the next dS overwrites.
 template <int D>
-__device__ __forceinline__ void bwd_mma(const BwdParams& p, uint32_t sbase, uint32_t tmem,
-                                        volatile int* abort_flag) {
-  using L = BwdLayout<D>;
+__device__ __forceinline__ void bwd_kv_mma(const BwdParams& p, uint32_t sbase, uint32_t tmem,
+                                           volatile int* abort_flag) {
+  using L = BwdKvLayout<D>;
   const uint32_t bars = sbase + L::kBarOff;
-  constexpr uint32_t kIdS = idesc_bf16_f32(kBwdBM, kBwdBN, false);         // K-major A and B
-  constexpr uint32_t kIdAcc = idesc_bf16_f32(kBwdBM, D, true);             // A TMEM, B MN-major
-  constexpr uint32_t kIdDq = idesc_bf16_f32(kBwdBN, D, true, true);        // A, B MN-major
+  constexpr uint32_t kIdAcc = idesc_bf16_f32(kBwdBM, D, true);  // A K-major, B MN-major
   const uint32_t t_dv = tmem, t_dk = tmem + 128, t_s = tmem + 256, t_dp = tmem + 384;
-  const uint32_t ka = sbase + L::kKOff, va = sbase + L::kVOff, dsa = sbase + L::kDsOff;
   int b, g, j;
-  bwd_cta(p, b, g, j);
+  bwd_kv_cta(p, b, g, j);
   const int i0 = bwd_first_q_tile(p, j);
   const int per_head = p.n_q_tiles - i0;
   const uint32_t total = per_head > 0 ? static_cast<uint32_t>(per_head * p.group) : 0u;
-  // TMEM column of the packed bf16 pairs for queries 16*kk .. 16*kk+15: each
-  // warpgroup packs its 64 queries at the start of its own 64 columns
-  auto packed_col = [](int kk) -> uint32_t {
-    constexpr int kSteps = kBwdBN / 16;
-    return static_cast<uint32_t>(kk * 8 + (kk >= kSteps / 2 ? 32 : 0));
-  };
   auto wait = [&](int bar, uint32_t parity) -> bool {
     if (!mbar_wait(bars + 8 * bar, parity, abort_flag, p.wait_limit_ns)) return false;
     tc_fence_after();
     return true;
   };
-  // A, B both K-major (rows of 64 elements, 128B swizzle), K = D in steps of 16
-  auto gemm_kmajor = [&](uint32_t d_tmem, uint32_t a, uint32_t bb) {
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t o = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-      mma_ss(d_tmem, sw128_desc(a + o, 16, 1024), sw128_desc(bb + o, 16, 1024), kIdS,
-             kk > 0 ? 1u : 0u);
-    }
-  };
+  // Descriptors are built once; a K step adds a compile-time offset inside
+  // the MMA's own asm, a Q/dO stage a multiple of the stage size.
+  const uint64_t k_km = sw128_desc(sbase + L::kKOff, 16, 1024);
+  const uint64_t v_km = sw128_desc(sbase + L::kVOff, 16, 1024);
+  const uint64_t ds_km = sw128_desc(sbase + L::kDsOff, 16, 1024);
+  const uint64_t q_km0 = sw128_desc(sbase + L::kQOff, 16, 1024);
+  const uint64_t q_mn0 = sw128_desc(sbase + L::kQOff, L::kBoxBytes, 1024);
+  constexpr uint64_t kStageStep = (2 * L::kTileBytes) >> 4;
+  constexpr uint64_t kDoStep = L::kTileBytes >> 4;  // dO after Q
   if (total > 0) {
     if (!wait(L::kBKv, 0u) || !wait(L::kBQFull + 0, 0u)) goto done;
-    gemm_kmajor(t_s, ka, sbase + L::kQOff);                        // S^T = K Q^T
+    bwd_gemm_kmajor<D>(t_s, k_km, q_km0);             // S^T = K Q^T
     mma_commit(bars + 8 * L::kBSFull);
-    gemm_kmajor(t_dp, va, sbase + L::kQOff + L::kTileBytes);       // dP^T = V dO^T
+    bwd_gemm_kmajor<D>(t_dp, v_km, q_km0 + kDoStep);  // dP^T = V dO^T
     mma_commit(bars + 8 * L::kBDpFull);
   }
   for (uint32_t n = 0; n < total; ++n) {
     const uint32_t s = n & 1u, ph = n & 1u;
-    const uint32_t qa = sbase + L::kQOff + 2 * s * L::kTileBytes;
-    const uint32_t doa = qa + L::kTileBytes;
+    const uint64_t q_mn = q_mn0 + s * kStageStep, do_mn = q_mn + kDoStep;
+    const bool more = n + 1 < total;
+    const uint32_t s1 = (n + 1) & 1u;
+    const uint64_t q_km1 = q_km0 + s1 * kStageStep;
     if (!wait(L::kBPFull, ph)) goto done;
-#pragma unroll
-    for (int kk = 0; kk < kBwdBN / 16; ++kk)       // dV += P^T dO
-      mma_ts(t_dv, t_s + packed_col(kk), sw128_desc(doa + kk * 16 * 128, L::kBoxBytes, 1024),
-             kIdAcc, (n > 0 || kk > 0) ? 1u : 0u);
-    if (!wait(L::kBDsFull, ph)) goto done;
-#pragma unroll
-    for (int kk = 0; kk < kBwdBN / 16; ++kk)       // dK += dS^T Q
-      mma_ts(t_dk, t_dp + packed_col(kk), sw128_desc(qa + kk * 16 * 128, L::kBoxBytes, 1024),
-             kIdAcc, (n > 0 || kk > 0) ? 1u : 0u);
-    mma_commit(bars + 8 * (L::kBQEmpty + s));     // Q_i, dO_i read by everything issued so far
-    // dQ_i = dS K (K = keys) into the dP^T / dS columns (dS already read by dK)
-#pragma unroll
-    for (int kk = 0; kk < kBwdBM / 16; ++kk)
-      mma_ss(t_dp, sw128_desc(dsa + kk * 16 * 128, L::kBoxBytes, 1024),
-             sw128_desc(ka + kk * 16 * 128, L::kBoxBytes, 1024), kIdDq, kk > 0 ? 1u : 0u);
-    mma_commit(bars + 8 * L::kBDqFull);
-    if (n + 1 < total) {
-      // next tile's scores while dQ_i is read out (P_i was read by dV already)
-      const uint32_t s1 = (n + 1) & 1u;
-      const uint32_t qa1 = sbase + L::kQOff + 2 * s1 * L::kTileBytes;
+    static_for<kBwdBN / 16>([&](auto kk_c) {      // dV += P^T dO
+      constexpr int kk = decltype(kk_c)::value;
+      mma_ts_off<bwd_mn_off(kk)>(t_dv, t_s + bwd_packed_col(kk), do_mn, kIdAcc,
+                                 (n > 0 || kk > 0) ? 1u : 0u);
+    });
+    if (more) {                                   // next tile's scores
       if (!wait(L::kBQFull + s1, ((n + 1) >> 1) & 1u)) goto done;
-      gemm_kmajor(t_s, ka, qa1);
+      bwd_gemm_kmajor<D>(t_s, k_km, q_km1);
       mma_commit(bars + 8 * L::kBSFull);
-      // dP^T of the next tile once dQ_i has left the dP^T columns
-      if (!wait(L::kBSFree, ph)) goto done;
-      gemm_kmajor(t_dp, va, qa1 + L::kTileBytes);
+    }
+    if (!wait(L::kBDsFull, ph)) goto done;
+    static_for<kBwdBN / 16>([&](auto kk_c) {      // dK += dS^T Q (K-dim = queries)
+      constexpr int kk = decltype(kk_c)::value;
+      mma_ss_off<bwd_km_off(kk), bwd_mn_off(kk)>(t_dk, ds_km, q_mn, kIdAcc,
+                                                 (n > 0 || kk > 0) ? 1u : 0u);
+    });
+    mma_commit(bars + 8 * (L::kBQEmpty + s));     // Q_n, dO_n read by everything issued so far
+    if (more) {                                   // next tile's dP^T
+      bwd_gemm_kmajor<D>(t_dp, v_km, q_km1 + kDoStep);
       mma_commit(bars + 8 * L::kBDpFull);
     }
   }
@@ -307,17 +286,14 @@ done:
   mbar_wait(bars + 8 * L::kBDone, 0u, nullptr, p.wait_limit_ns);
 }
 
-// ---------------------------------------------------------------------------
 // Element-wise warpgroups (warps 0-7).  Warpgroup hf takes queries
 // [64*hf, 64*hf + 64) of each tile for P and dS (thread t = key row t, the
-// TMEM lane) and d-columns [hf*D/2, (hf+1)*D/2) for the dQ partial (thread t
-// = query row t) and for dK, dV; the two halves run side by side.
-// ---------------------------------------------------------------------------
+// TMEM lane) and d-columns [hf*D/2, (hf+1)*D/2) of dK, dV at the end.
 template <int D>
-__device__ __forceinline__ void bwd_elementwise(const BwdParams& p, const CUtensorMap* tm_dq,
-                                                uint32_t sbase, uint8_t* smem, uint32_t tmem,
-                                                volatile int* abort_flag) {
-  using L = BwdLayout<D>;
+__device__ __forceinline__ void bwd_kv_elementwise(const BwdParams& p, uint32_t sbase,
+                                                   uint8_t* smem, uint32_t tmem,
+                                                   volatile int* abort_flag) {
+  using L = BwdKvLayout<D>;
   const uint32_t bars = sbase + L::kBarOff;
   const int t = threadIdx.x & 127;
   const int hf = threadIdx.x >> 7;  // warpgroup: query half / column half
@@ -331,31 +307,31 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, const CUtens
   float* d_s = lse_s + 128;
   uint8_t* ds_smem = smem + L::kDsOff;
   int b, g, j;
-  bwd_cta(p, b, g, j);
+  bwd_kv_cta(p, b, g, j);
   const int key = j * kBwdBM + t;
   const int off = p.Skv - p.Sq;
   const int i0 = bwd_first_q_tile(p, j);
   uint32_t n = 0;
-  // LSE (in log2 units) and D of this thread's query for a tile: loaded one
+  // -LSE (in log2 units) and D of this thread's query for a tile: loaded one
   // tile ahead, so the load latency hides behind the previous tile's work.
+  // Query rows past Sq take -LSE = -inf, so their weights are exactly 0.
   auto load_ld = [&](int hh_, int i_, float& lse_v, float& d_v) {
     const int c = hf * kQH + t;
     const int q = i_ * kBwdBN + c;
     const size_t rb = (static_cast<size_t>(b) * p.Hq + g * p.group + hh_) * p.Sq;
-    lse_v = (t < kQH && q < p.Sq) ? p.lse[rb + q] * 1.4426950408889634f : INFINITY;
+    lse_v = (t < kQH && q < p.Sq) ? p.lse[rb + q] * -1.4426950408889634f : -INFINITY;
     d_v = (t < kQH && q < p.Sq) ? p.dsum[rb + q] : 0.f;
   };
-  float lse_next = INFINITY, d_next = 0.f;
+  float lse_next = -INFINITY, d_next = 0.f;
   if (i0 < p.n_q_tiles) load_ld(0, i0, lse_next, d_next);
   // After a failed wait a warp skips the remaining work but still takes every
   // named barrier, so the other warps of its warpgroup can never block there.
   bool ok = true;
   for (int hh = 0; hh < p.group; ++hh) {
-    const int h = g * p.group + hh;
     for (int i = i0; i < p.n_q_tiles; ++i, ++n) {
       const uint32_t ph = n & 1u;
       const int q0 = i * kBwdBN;
-      // this warpgroup's 64 queries: LSE and D into shared memory
+      // this warpgroup's 64 queries: -LSE and D into shared memory
       named_barrier(1 + hf, 128);
       if (t < kQH) {
         lse_s[hf * kQH + t] = lse_next;
@@ -370,6 +346,7 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, const CUtens
 
       if (!ok) continue;
       // P^T for this key and the warpgroup's queries: p = 2^(s*scale*log2e - LSE*log2e)
+      // (a key that every query of the half sees takes the branch without masks)
       ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * L::kBSFull, ph, abort_flag, p.wait_limit_ns));
       if (!ok) continue;
       tc_fence_after();
@@ -379,17 +356,29 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, const CUtens
         tmem_ld64_nowait(t_s + hf * kQH, ra);
         tmem_ld_wait_hold(ra);
         const int lim = key - off;  // first query that sees this key
+        const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+        const bool all_vis = (key < p.Skv) && (!p.causal || q0 + hf * kQH >= lim);
+        if (__all_sync(0xffffffffu, all_vis)) {
 #pragma unroll
-        for (int c2 = 0; c2 < kQH / 2; ++c2) {
-          float pr[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = hf * kQH + 2 * c2 + e;
-            const bool vis = (key < p.Skv) && (!p.causal || q0 + c >= lim);
-            const float x = fmaf(__uint_as_float(ra[2 * c2 + e]), p.scale_log2, -lse_s[c]);
-            pr[e] = vis ? ex2(x) : 0.f;
+          for (int c2 = 0; c2 < kQH / 2; ++c2) {
+            const float2 nl = *reinterpret_cast<const float2*>(lse_s + hf * kQH + 2 * c2);
+            const float2 x = ffma2(make_float2(__uint_as_float(ra[2 * c2]),
+                                               __uint_as_float(ra[2 * c2 + 1])), sl2, nl);
+            pk[c2] = pack_bf16x2(ex2(x.x), ex2(x.y));
           }
-          pk[c2] = pack_bf16x2(pr[0], pr[1]);
+        } else {
+#pragma unroll
+          for (int c2 = 0; c2 < kQH / 2; ++c2) {
+            float pr[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int c = hf * kQH + 2 * c2 + e;
+              const bool vis = (key < p.Skv) && (!p.causal || q0 + c >= lim);
+              const float x = fmaf(__uint_as_float(ra[2 * c2 + e]), p.scale_log2, lse_s[c]);
+              pr[e] = vis ? ex2(x) : 0.f;
+            }
+            pk[c2] = pack_bf16x2(pr[0], pr[1]);
+          }
         }
       }
       // packed pairs of queries, inside this warpgroup's own (already read)
@@ -400,8 +389,8 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, const CUtens
       __syncwarp();
       if ((threadIdx.x & 31) == 0) mbar_arrive(bars + 8 * L::kBPFull);
 
-      // dS = P * (dP - D): to TMEM (A of dK += dS^T Q) and to shared memory
-      // (A of dQ = dS K, MN-major: rows = keys, 64-query boxes, 128B swizzle)
+      // dS = P * (dP - D) to shared memory: rows = keys, 64-query boxes, 128B
+      // swizzle (the K-major A operand of dK += dS^T Q)
       ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * L::kBDpFull, ph, abort_flag, p.wait_limit_ns));
       if (!ok) continue;
       tc_fence_after();
@@ -419,7 +408,6 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, const CUtens
           const float d1 = __bfloat162float(pb.y) * (__uint_as_float(dp[2 * e2 + 1]) - d_s[c + 1]);
           dsk[e2] = pack_bf16x2(d0, d1);
         }
-        tmem_st16(t_dp + hf * kQH + hq * 16, dsk);  // own columns, already read
         // queries hf*64 + hq*32 .. +31: box hf, 16-byte chunks hq*4 .. +3 of row t
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
@@ -429,51 +417,12 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, const CUtens
           *dst = make_uint4(dsk[4 * k4], dsk[4 * k4 + 1], dsk[4 * k4 + 2], dsk[4 * k4 + 3]);
         }
       }
-      tmem_st_wait();
       fence_proxy_async_smem();
-      tc_fence_before();
+      tc_fence_before();  // the dP^T loads are complete before the next dP^T overwrites them
       __syncwarp();
       if ((threadIdx.x & 31) == 0) mbar_arrive(bars + 8 * L::kBDsFull);
-
-      // dQ partial (thread = query row q0 + t, this warpgroup's d-columns),
-      // scaled, staged 32 columns at a time in this warpgroup's half of the
-      // dS buffer (free: the dQ MMA that read dS is complete) and added into
-      // the fp32 workspace by one bulk tensor reduction per 128 x 32 box.
-      ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * L::kBDqFull, ph, abort_flag, p.wait_limit_ns));
-      if (!ok) continue;
-      tc_fence_after();
-      {
-        uint8_t* stage = ds_smem + hf * L::kBoxBytes;  // 128 rows x 128 B, 128B swizzle
-        const uint32_t stage_s = sbase + L::kDsOff + hf * L::kBoxBytes;
-#pragma unroll
-        for (int c4 = 0; c4 < kDH / 32; ++c4) {
-          uint32_t r[32];
-          tmem_ld32(t_dp + hf * kDH + c4 * 32, r);
-#pragma unroll
-          for (int k4 = 0; k4 < 8; ++k4) {
-            float4 v4 = make_float4(__uint_as_float(r[4 * k4]) * p.scale,
-                                    __uint_as_float(r[4 * k4 + 1]) * p.scale,
-                                    __uint_as_float(r[4 * k4 + 2]) * p.scale,
-                                    __uint_as_float(r[4 * k4 + 3]) * p.scale);
-            *reinterpret_cast<float4*>(stage + t * 128 + ((k4 ^ (t & 7)) * 16)) = v4;
-          }
-          fence_proxy_async_smem();
-          named_barrier(1 + hf, 128);
-          if (t == 0) {
-            tma_reduce_add_3d(tm_dq, stage_s, hf * kDH + c4 * 32, q0, static_cast<int>(
-                static_cast<size_t>(b) * p.Hq + h));
-            bulk_commit_group();
-            bulk_wait_group_read0();  // the box has been read: the buffer is free again
-          }
-          named_barrier(1 + hf, 128);
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if ((threadIdx.x & 31) == 0) mbar_arrive(bars + 8 * L::kBSFree);
     }
   }
-  if (t == 0) bulk_wait_group0();  // this thread's reductions have landed
   if (!ok) return;
 
   // dK = scale * (dS^T Q summed), dV = P^T dO summed: thread t = key row,
@@ -512,10 +461,10 @@ __device__ __forceinline__ void bwd_elementwise(const BwdParams& p, const CUtens
 
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
-fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-              const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
-  using L = BwdLayout<D>;
+fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                   const BwdParams p) {
+  using L = BwdKvLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
@@ -534,8 +483,6 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     mbar_init(bars + 8 * L::kBDpFull, 1);
     mbar_init(bars + 8 * L::kBPFull, 8);   // one arrival per element-wise warp
     mbar_init(bars + 8 * L::kBDsFull, 8);
-    mbar_init(bars + 8 * L::kBDqFull, 1);
-    mbar_init(bars + 8 * L::kBSFree, 8);
     mbar_init(bars + 8 * L::kBDone, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -550,11 +497,345 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlotOff);
 
   if (warp < 8) {
-    bwd_elementwise<D>(p, &tm_dq, sbase, smem, tmem, abort_flag);
+    bwd_kv_elementwise<D>(p, sbase, smem, tmem, abort_flag);
   } else if (warp == 8) {
-    if (lane == 0) bwd_producer<D>(&tm_q, &tm_k, &tm_v, &tm_do, p, sbase, abort_flag);
+    if (lane == 0) bwd_kv_producer<D>(&tm_q, &tm_k, &tm_v, &tm_do, p, sbase, abort_flag);
   } else {
-    if (lane == 0) bwd_mma<D>(p, sbase, tmem, abort_flag);
+    if (lane == 0) bwd_kv_mma<D>(p, sbase, tmem, abort_flag);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ===========================================================================
+// dQ: query-stationary kernel
+// ===========================================================================
+template <int D>
+struct BwdQLayout {
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kBoxBytes = 128 * 128;
+  static constexpr int kStages = 2;
+  static constexpr int kQOff = 0;
+  static constexpr int kDoOff = kTileBytes;
+  static constexpr int kRingOff = 2 * kTileBytes;  // stage s: K at kRingOff + 2*s*tile, V after it
+  static constexpr int kBarOff = kRingOff + kStages * 2 * kTileBytes;
+  static constexpr int kBQ = 0;        // Q_i and dO_i loaded
+  static constexpr int kBKvFull = 1;   // [kStages]
+  static constexpr int kBKvEmpty = 3;  // [kStages]
+  static constexpr int kBSFull = 5;    // [2] one per S buffer
+  static constexpr int kBDpFull = 7;
+  static constexpr int kBDsFull = 8;   // 8 arrivals (one per element-wise warp)
+  static constexpr int kBDone = 9;
+  static constexpr int kNumBars = 10;
+  static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
+  static constexpr int kAbortOff = kTmemSlotOff + 4;
+  static constexpr int kBytes = kAbortOff + 4 + 1024;
+};
+static_assert(BwdQLayout<128>::kBytes <= 232448, "dQ shared memory over the limit");
+
+// The dQ CTAs go out heaviest first: under a causal mask (or a rectangular
+// one with more keys than queries) the last query tiles see the most keys.
+__device__ __forceinline__ void bwd_q_cta(const BwdParams& p, int& b, int& h, int& i) {
+  const int heads = p.B * p.Hq;
+  i = p.n_q_tiles - 1 - static_cast<int>(blockIdx.x) / heads;
+  const int bh = static_cast<int>(blockIdx.x) % heads;
+  b = bh / p.Hq;
+  h = bh % p.Hq;
+}
+
+// Key tiles that query tile i sees: [0, n).
+__device__ __forceinline__ int bwd_q_kv_tiles(const BwdParams& p, int i) {
+  if (!p.causal) return p.n_kv_tiles;
+  const long long q_last = min(static_cast<long long>(i) * kBwdBN + kBwdBN - 1,
+                               static_cast<long long>(p.Sq) - 1);
+  const long long k_last = q_last + (p.Skv - p.Sq);  // last key the last row sees
+  if (k_last < 0) return 0;
+  return static_cast<int>(min(static_cast<long long>(p.n_kv_tiles), k_last / kBwdBM + 1));
+}
+
+template <int D>
+__device__ __forceinline__ void bwd_q_producer(const CUtensorMap* tq, const CUtensorMap* tk,
+                                               const CUtensorMap* tv, const CUtensorMap* tdo,
+                                               const BwdParams& p, uint32_t sbase,
+                                               volatile int* abort_flag) {
+  using L = BwdQLayout<D>;
+  const uint32_t bars = sbase + L::kBarOff;
+  int b, h, i;
+  bwd_q_cta(p, b, h, i);
+  const int nk = bwd_q_kv_tiles(p, i);
+  if (nk == 0) return;
+  tma_prefetch_desc(tq);
+  tma_prefetch_desc(tk);
+  tma_prefetch_desc(tv);
+  tma_prefetch_desc(tdo);
+  const int g = h / p.group;
+  const uint32_t bq = bars + 8 * L::kBQ;
+  mbar_arrive_expect_tx(bq, 2 * L::kTileBytes);
+#pragma unroll
+  for (int kb = 0; kb < D / 64; ++kb) {
+    tma_load_3d(sbase + L::kQOff + kb * L::kBoxBytes, tq, bq, kb * 64, i * kBwdBN, b * p.Hq + h);
+    tma_load_3d(sbase + L::kDoOff + kb * L::kBoxBytes, tdo, bq, kb * 64, i * kBwdBN, b * p.Hq + h);
+  }
+  int jn = 0;  // key tiles loaded
+  for (; jn < nk; ++jn) {
+    const int s = jn % L::kStages;
+    const uint32_t use = static_cast<uint32_t>(jn / L::kStages);
+    if (!mbar_wait(bars + 8 * (L::kBKvEmpty + s), (use & 1u) ^ 1u, abort_flag, p.wait_limit_ns))
+      break;
+    const uint32_t full = bars + 8 * (L::kBKvFull + s);
+    const uint32_t ka = sbase + L::kRingOff + 2 * s * L::kTileBytes;
+    mbar_arrive_expect_tx(full, 2 * L::kTileBytes);
+#pragma unroll
+    for (int kb = 0; kb < D / 64; ++kb) {
+      tma_load_3d(ka + kb * L::kBoxBytes, tk, full, kb * 64, jn * kBwdBM, b * p.Hkv + g);
+      tma_load_3d(ka + L::kTileBytes + kb * L::kBoxBytes, tv, full, kb * 64, jn * kBwdBM,
+                  b * p.Hkv + g);
+    }
+  }
+  // drain: the CTA does not exit with copies in flight
+  mbar_wait(bq, 0u, nullptr, p.wait_limit_ns);
+  for (int k = (jn > L::kStages ? jn - L::kStages : 0); k < jn; ++k)
+    mbar_wait(bars + 8 * (L::kBKvFull + k % L::kStages),
+              static_cast<uint32_t>(k / L::kStages) & 1u, nullptr, p.wait_limit_ns);
+}
+
+// Per key tile j: dQ_j once dS_j is announced (it reads dS_j from S buffer
+// j%2 and K_j), which frees the ring stage; then dP_{j+1} (the element-wise
+// warps have read dP_j before announcing dS_j) and S_{j+2} into buffer j%2
+// (after dQ_j, which reads it, in issue order).
+template <int D>
+__device__ __forceinline__ void bwd_q_mma(const BwdParams& p, uint32_t sbase, uint32_t tmem,
+                                          volatile int* abort_flag) {
+  using L = BwdQLayout<D>;
+  const uint32_t bars = sbase + L::kBarOff;
+  constexpr uint32_t kIdDq = idesc_bf16_f32(kBwdBN, D, true);  // A TMEM, B MN-major
+  const uint32_t t_s0 = tmem, t_dp = tmem + 256, t_dq = tmem + 384;
+  int b, h, i;
+  bwd_q_cta(p, b, h, i);
+  const int nk = bwd_q_kv_tiles(p, i);
+  auto wait = [&](int bar, uint32_t parity) -> bool {
+    if (!mbar_wait(bars + 8 * bar, parity, abort_flag, p.wait_limit_ns)) return false;
+    tc_fence_after();
+    return true;
+  };
+  auto kv_wait = [&](int jj) -> bool {
+    return wait(L::kBKvFull + jj % L::kStages, static_cast<uint32_t>(jj / L::kStages) & 1u);
+  };
+  const uint64_t q_km = sw128_desc(sbase + L::kQOff, 16, 1024);
+  const uint64_t do_km = sw128_desc(sbase + L::kDoOff, 16, 1024);
+  const uint64_t k_km0 = sw128_desc(sbase + L::kRingOff, 16, 1024);
+  const uint64_t k_mn0 = sw128_desc(sbase + L::kRingOff, L::kBoxBytes, 1024);
+  constexpr uint64_t kStageStep = (2 * L::kTileBytes) >> 4;
+  constexpr uint64_t kVStep = L::kTileBytes >> 4;  // V after K
+  if (nk > 0) {
+    if (!wait(L::kBQ, 0u) || !kv_wait(0)) goto done;
+    bwd_gemm_kmajor<D>(t_s0, q_km, k_km0);               // S_0 = Q K_0^T
+    mma_commit(bars + 8 * (L::kBSFull + 0));
+    bwd_gemm_kmajor<D>(t_dp, do_km, k_km0 + kVStep);     // dP_0 = dO V_0^T
+    mma_commit(bars + 8 * L::kBDpFull);
+    if (nk > 1) {
+      if (!kv_wait(1)) goto done;
+      bwd_gemm_kmajor<D>(t_s0 + 128, q_km, k_km0 + kStageStep);
+      mma_commit(bars + 8 * (L::kBSFull + 1));
+    }
+  }
+  for (int jj = 0; jj < nk; ++jj) {
+    const int buf = jj & 1;
+    const int s = jj % L::kStages;
+    if (!wait(L::kBDsFull, static_cast<uint32_t>(jj) & 1u)) goto done;
+    const uint64_t k_mn = k_mn0 + s * kStageStep;
+    const uint32_t t_ds = t_s0 + 128 * buf;
+    static_for<kBwdBM / 16>([&](auto kk_c) {             // dQ += dS K (K-dim = keys)
+      constexpr int kk = decltype(kk_c)::value;
+      mma_ts_off<bwd_mn_off(kk)>(t_dq, t_ds + bwd_packed_col(kk), k_mn, kIdDq,
+                                 (jj > 0 || kk > 0) ? 1u : 0u);
+    });
+    mma_commit(bars + 8 * (L::kBKvEmpty + s));           // K_j, V_j consumed
+    if (jj + 1 < nk) {                                    // dP_{j+1}: V_{j+1} waited for with S_{j+1}
+      const int s1 = (jj + 1) % L::kStages;
+      bwd_gemm_kmajor<D>(t_dp, do_km, k_km0 + s1 * kStageStep + kVStep);
+      mma_commit(bars + 8 * L::kBDpFull);
+    }
+    if (jj + 2 < nk) {                                    // S_{j+2} into buffer j%2
+      if (!kv_wait(jj + 2)) goto done;
+      const int s2 = (jj + 2) % L::kStages;
+      bwd_gemm_kmajor<D>(t_ds, q_km, k_km0 + s2 * kStageStep);
+      mma_commit(bars + 8 * (L::kBSFull + buf));
+    }
+  }
+done:
+  mma_commit(bars + 8 * L::kBDone);
+  mbar_wait(bars + 8 * L::kBDone, 0u, nullptr, p.wait_limit_ns);
+}
+
+// Element-wise warpgroups: thread = query row (its TMEM lane); warpgroup hf
+// takes keys [64*hf, 64*hf + 64) of each key tile, and d-columns
+// [hf*D/2, (hf+1)*D/2) of dQ at the end.
+template <int D>
+__device__ __forceinline__ void bwd_q_elementwise(const BwdParams& p, uint32_t sbase,
+                                                  uint32_t tmem, volatile int* abort_flag) {
+  using L = BwdQLayout<D>;
+  const uint32_t bars = sbase + L::kBarOff;
+  const int hf = threadIdx.x >> 7;
+  const int warp = (threadIdx.x >> 5) & 3;
+  const int row = warp * 32 + (threadIdx.x & 31);
+  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t t_s0 = tmem + lane_off, t_dp = tmem + lane_off + 256, t_dq = tmem + lane_off + 384;
+  constexpr int kKH = kBwdBM / 2;  // keys per warpgroup
+  constexpr int kDH = D / 2;
+  int b, h, i;
+  bwd_q_cta(p, b, h, i);
+  const int nk = bwd_q_kv_tiles(p, i);
+  const int q = i * kBwdBN + row;
+  const bool real = q < p.Sq;
+  const size_t qrow = (static_cast<size_t>(b) * p.Hq + h) * p.Sq + (real ? q : 0);
+  // -LSE in log2 units (rows past Sq: -inf, weights exactly 0) and D
+  const float nlse = real ? p.lse[qrow] * -1.4426950408889634f : -INFINITY;
+  const float dval = real ? p.dsum[qrow] : 0.f;
+  const int off = p.Skv - p.Sq;
+  const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+  const float2 nl2 = make_float2(nlse, nlse);
+  bool ok = true;
+  for (int jj = 0; jj < nk; ++jj) {
+    const int buf = jj & 1;
+    const uint32_t t_s = t_s0 + 128 * buf;
+    ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (L::kBSFull + buf),
+                                           static_cast<uint32_t>(jj >> 1) & 1u, abort_flag,
+                                           p.wait_limit_ns));
+    if (!ok) break;
+    tc_fence_after();
+    // P = 2^(s*scale*log2e - LSE*log2e) for this row and the warpgroup's keys
+    const int k0 = jj * kBwdBM + hf * kKH;  // first key of this half
+    float pr[kKH];
+    {
+      uint32_t ra[64];
+      tmem_ld64_nowait(t_s + hf * kKH, ra);
+      tmem_ld_wait_hold(ra);
+      const bool all_vis = (k0 + kKH <= p.Skv) && (!p.causal || k0 + kKH - 1 <= q + off);
+      if (__all_sync(0xffffffffu, all_vis)) {
+#pragma unroll
+        for (int c2 = 0; c2 < kKH / 2; ++c2) {
+          const float2 x = ffma2(make_float2(__uint_as_float(ra[2 * c2]),
+                                             __uint_as_float(ra[2 * c2 + 1])), sl2, nl2);
+          pr[2 * c2] = ex2(x.x);
+          pr[2 * c2 + 1] = ex2(x.y);
+        }
+      } else {
+        // keys [k0, k0 + lim) of the half are visible to this row
+        const int lim = (p.causal ? min(p.Skv, q + off + 1) : p.Skv) - k0;
+#pragma unroll
+        for (int c = 0; c < kKH; ++c) {
+          const float x = fmaf(__uint_as_float(ra[c]), p.scale_log2, nlse);
+          pr[c] = (c < lim) ? ex2(x) : 0.f;
+        }
+      }
+    }
+    // dS = P * (dP - D), packed bf16 pairs into this warpgroup's own
+    // (already read) score columns: the A operand of dQ += dS K
+    ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * L::kBDpFull, static_cast<uint32_t>(jj) & 1u,
+                                           abort_flag, p.wait_limit_ns));
+    if (!ok) break;
+    tc_fence_after();
+#pragma unroll
+    for (int hk = 0; hk < 2; ++hk) {  // 32 keys per pass
+      uint32_t dp[32];
+      tmem_ld32(t_dp + hf * kKH + hk * 32, dp);
+      uint32_t dsk[16];
+#pragma unroll
+      for (int e2 = 0; e2 < 16; ++e2) {
+        const int c = hk * 32 + 2 * e2;
+        dsk[e2] = pack_bf16x2(pr[c] * (__uint_as_float(dp[2 * e2]) - dval),
+                              pr[c + 1] * (__uint_as_float(dp[2 * e2 + 1]) - dval));
+      }
+      tmem_st16(t_s + hf * kKH + hk * 16, dsk);
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bars + 8 * L::kBDsFull);
+  }
+  if (!ok) return;
+  // dQ = scale * (dS K summed): this row, the warpgroup's d-columns (zero for
+  // a tile that sees no key)
+  if (nk > 0) {
+    if (!__all_sync(0xffffffffu, mbar_wait(bars + 8 * L::kBDone, 0u, abort_flag, p.wait_limit_ns)))
+      return;
+    tc_fence_after();
+  }
+  __nv_bfloat16* out = p.dq + qrow * D + hf * kDH;
+#pragma unroll
+  for (int c4 = 0; c4 < kDH / 32; ++c4) {
+    uint32_t r[32];
+    if (nk > 0) {
+      tmem_ld32(t_dq + hf * kDH + c4 * 32, r);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) r[e] = 0u;
+    }
+    if (real) {
+#pragma unroll
+      for (int v4 = 0; v4 < 4; ++v4) {
+        uint4 w;
+        const float* f = reinterpret_cast<const float*>(r) + v4 * 8;
+        w.x = pack_bf16x2(f[0] * p.scale, f[1] * p.scale);
+        w.y = pack_bf16x2(f[2] * p.scale, f[3] * p.scale);
+        w.z = pack_bf16x2(f[4] * p.scale, f[5] * p.scale);
+        w.w = pack_bf16x2(f[6] * p.scale, f[7] * p.scale);
+        reinterpret_cast<uint4*>(out + c4 * 32)[v4] = w;
+      }
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                 const BwdParams p) {
+  using L = BwdQLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sbase = raw + pad;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbortOff);
+  const uint32_t bars = sbase + L::kBarOff;
+  if (threadIdx.x == 0) {
+    mbar_init(bars + 8 * L::kBQ, 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(bars + 8 * (L::kBKvFull + s), 1);
+      mbar_init(bars + 8 * (L::kBKvEmpty + s), 1);
+    }
+    mbar_init(bars + 8 * (L::kBSFull + 0), 1);
+    mbar_init(bars + 8 * (L::kBSFull + 1), 1);
+    mbar_init(bars + 8 * L::kBDpFull, 1);
+    mbar_init(bars + 8 * L::kBDsFull, 8);  // one arrival per element-wise warp
+    mbar_init(bars + 8 * L::kBDone, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(sbase + L::kTmemSlotOff, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlotOff);
+
+  if (warp < 8) {
+    bwd_q_elementwise<D>(p, sbase, tmem, abort_flag);
+  } else if (warp == 8) {
+    if (lane == 0) bwd_q_producer<D>(&tm_q, &tm_k, &tm_v, &tm_do, p, sbase, abort_flag);
+  } else {
+    if (lane == 0) bwd_q_mma<D>(p, sbase, tmem, abort_flag);
   }
 
   tc_fence_before();

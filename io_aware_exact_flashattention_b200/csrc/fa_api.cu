@@ -90,21 +90,6 @@ bool encode_rows256(CUtensorMap* map, const void* base, int cols, int rows) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// [planes, rows, d] fp32 rows (the backward's dq accumulator) as a 3-D map with
-// 32 x 128 x 1 boxes, 128B swizzle: the target of bulk tensor reductions.
-bool encode_f32_rows(CUtensorMap* map, void* base, int d, int rows, long long planes) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
-  if (enc == nullptr) return false;
-  const cuuint64_t r = static_cast<cuuint64_t>(rows > 0 ? rows : 1);
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), r, static_cast<cuuint64_t>(planes)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4, r * static_cast<cuuint64_t>(d) * 4};
-  cuuint32_t box[3] = {32, 128, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // One-time per-device opt-in to the prefill kernels' dynamic shared memory,
 // and the device's SM count (the persistent grid size).
 std::once_flag g_attr_once[kMaxDevices];
@@ -426,68 +411,79 @@ cudaError_t prepare_backward(int dev) {
   std::call_once(g_bwd_once[dev], [dev] {
     cudaError_t e = cudaDeviceGetAttribute(&g_bwd_sms[dev], cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(fa::fa_bwd_kernel<64>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         fa::BwdLayout<64>::kBytes);
+      e = cudaFuncSetAttribute(fa::fa_bwd_dkdv_kernel<64>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::BwdKvLayout<64>::kBytes);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(fa::fa_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::BwdLayout<128>::kBytes);
+      e = cudaFuncSetAttribute(fa::fa_bwd_dkdv_kernel<128>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::BwdKvLayout<128>::kBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::BwdQLayout<64>::kBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<128>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::BwdQLayout<128>::kBytes);
     g_bwd_err[dev] = e;
   });
   return g_bwd_err[dev];
 }
 
+// D = rowsum(dO * O) into the workspace, then the dK/dV kernel (one CTA per
+// key tile) and the dQ kernel (one CTA per query tile); neither writes what
+// the other reads, and each gradient is written once.
 template <int D>
 fa_status launch_backward(const void* q, const void* k, const void* v, const void* o,
                           const float* lse, const void* d_o, void* dq, void* dk, void* dv,
                           float* workspace, int B, int Hq, int Hkv, int Sq, int Skv, int causal,
                           float scale, cudaStream_t stream) {
   const long long q_rows = static_cast<long long>(B) * Hq * Sq;
-  float* dq_acc = workspace;
-  float* dsum = workspace + q_rows * D;
+  float* dsum = workspace;
+  if (Skv == 0) k = v = q;  // no key tile is ever loaded; any valid address will do
   fa::fa_bwd_dsum_kernel<D><<<static_cast<unsigned>((q_rows + 7) / 8), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o), dsum, dq_acc,
-      q_rows);
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o), dsum, q_rows);
   const int n_kv_tiles = (Skv + fa::kBwdBM - 1) / fa::kBwdBM;
+  const int n_q_tiles = (Sq + fa::kBwdBN - 1) / fa::kBwdBN;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!encode_bhsd(&tq, q, D, Sq, static_cast<long long>(B) * Hq) ||
+      !encode_bhsd(&tdo, d_o, D, Sq, static_cast<long long>(B) * Hq) ||
+      !encode_bhsd(&tk, k, D, Skv, static_cast<long long>(B) * Hkv) ||
+      !encode_bhsd(&tv, v, D, Skv, static_cast<long long>(B) * Hkv))
+    return FA_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (prepare_backward(dev) != cudaSuccess) return FA_ERR_CUDA;
+  fa::BwdParams p;
+  p.lse = lse;
+  p.dsum = dsum;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Sq = Sq;
+  p.Skv = Skv;
+  p.group = Hq / Hkv;
+  p.causal = causal ? 1 : 0;
+  p.n_kv_tiles = n_kv_tiles;
+  p.n_q_tiles = n_q_tiles;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_limit_ns = kWaitLimitNs;
   if (n_kv_tiles > 0) {
-    CUtensorMap tq, tk, tv, tdo, tdq;
-    if (!encode_bhsd(&tq, q, D, Sq, static_cast<long long>(B) * Hq) ||
-        !encode_bhsd(&tdo, d_o, D, Sq, static_cast<long long>(B) * Hq) ||
-        !encode_f32_rows(&tdq, dq_acc, D, Sq, static_cast<long long>(B) * Hq) ||
-        !encode_bhsd(&tk, k, D, Skv, static_cast<long long>(B) * Hkv) ||
-        !encode_bhsd(&tv, v, D, Skv, static_cast<long long>(B) * Hkv))
-      return FA_ERR_CUDA;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
-    if (prepare_backward(dev) != cudaSuccess) return FA_ERR_CUDA;
-    fa::BwdParams p;
-    p.dq_acc = dq_acc;
-    p.lse = lse;
-    p.dsum = dsum;
-    p.dk = static_cast<__nv_bfloat16*>(dk);
-    p.dv = static_cast<__nv_bfloat16*>(dv);
-    p.B = B;
-    p.Hq = Hq;
-    p.Hkv = Hkv;
-    p.Sq = Sq;
-    p.Skv = Skv;
-    p.group = Hq / Hkv;
-    p.causal = causal ? 1 : 0;
-    p.n_kv_tiles = n_kv_tiles;
-    p.n_q_tiles = (Sq + fa::kBwdBN - 1) / fa::kBwdBN;
     // about kBwdGroupWaves waves of CTAs per group (one CTA per SM)
     p.heads_per_group =
         std::max(1, std::min(B * Hkv, kBwdGroupWaves * g_bwd_sms[dev] / n_kv_tiles));
-    p.scale = scale;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    p.wait_limit_ns = kWaitLimitNs;
     const unsigned grid = static_cast<unsigned>(static_cast<long long>(B) * Hkv * n_kv_tiles);
-    fa::fa_bwd_kernel<D><<<grid, fa::kBwdThreads, fa::BwdLayout<D>::kBytes, stream>>>(tq, tk, tv,
-                                                                                      tdo, tdq, p);
+    fa::fa_bwd_dkdv_kernel<D><<<grid, fa::kBwdThreads, fa::BwdKvLayout<D>::kBytes, stream>>>(
+        tq, tk, tv, tdo, p);
   }
-  const long long n = q_rows * D;
-  fa::fa_bwd_dq_kernel<<<static_cast<unsigned>((n / 4 + 255) / 256), 256, 0, stream>>>(
-      dq_acc, static_cast<__nv_bfloat16*>(dq), n);
+  p.heads_per_group = 1;
+  const unsigned qgrid = static_cast<unsigned>(static_cast<long long>(B) * Hq * n_q_tiles);
+  fa::fa_bwd_dq_kernel<D><<<qgrid, fa::kBwdThreads, fa::BwdQLayout<D>::kBytes, stream>>>(
+      tq, tk, tv, tdo, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -523,7 +519,7 @@ extern "C" {
 
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Sq, int d) {
   if (B <= 0 || Hq <= 0 || Sq <= 0 || d <= 0) return 0;
-  return static_cast<size_t>(B) * Hq * Sq * (static_cast<size_t>(d) + 1) * sizeof(float);
+  return static_cast<size_t>(B) * Hq * Sq * sizeof(float);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -534,17 +530,21 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (B == 0 || (Sq == 0 && Skv == 0)) return FA_OK;
-  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr ||
-      d_o == nullptr || dq == nullptr || dk == nullptr || dv == nullptr || workspace == nullptr)
+  // the query-side buffers may be null with no query rows, the key-side ones
+  // with no keys (nothing is read from or written to them)
+  if ((Sq > 0 && (q == nullptr || o == nullptr || lse == nullptr || d_o == nullptr ||
+                  dq == nullptr || workspace == nullptr)) ||
+      (Skv > 0 && (k == nullptr || v == nullptr || dk == nullptr || dv == nullptr)))
     return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
       !aligned16(d_o) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
       !aligned16(workspace))
     return FA_ERR_ALIGNMENT;
   const long long n_kv_tiles = (static_cast<long long>(Skv) + fa::kBwdBM - 1) / fa::kBwdBM;
-  const long long q_elems = static_cast<long long>(B) * Hq * Sq * d;
+  const long long n_q_tiles = (static_cast<long long>(Sq) + fa::kBwdBN - 1) / fa::kBwdBN;
+  const long long q_rows = static_cast<long long>(B) * Hq * Sq;
   if (static_cast<long long>(B) * Hkv * n_kv_tiles > 0x7fffffffLL ||
-      static_cast<long long>(B) * Hq > 0x7fffffffLL || q_elems / 4 / 256 > 0x7fffffffLL ||
+      static_cast<long long>(B) * Hq * n_q_tiles > 0x7fffffffLL || q_rows / 8 > 0x7fffffffLL ||
       static_cast<long long>(B) * Hkv > 0x7fffffffLL)
     return FA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -179,15 +179,6 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
   return r;
 }
 
-// Calls f(std::integral_constant<int, i>{}) for i = 0 .. N-1.
-template <int N, int I = 0, typename F>
-__device__ __forceinline__ void static_for(F&& f) {
-  if constexpr (I < N) {
-    f(std::integral_constant<int, I>{});
-    static_for<N, I + 1>(f);
-  }
-}
-
 struct PrefillParams {
   __nv_bfloat16* o;
   float* lse;

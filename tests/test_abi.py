@@ -241,7 +241,7 @@ def test_bpt_workspace_bytes(lib):
 
 
 def test_bwd_workspace_bytes(lib):
-    assert fa.bwd_workspace_bytes(2, 4, 100, 128) == 2 * 4 * 100 * 129 * 4
+    assert fa.bwd_workspace_bytes(2, 4, 100, 128) == 2 * 4 * 100 * 4
     assert fa.bwd_workspace_bytes(0, 4, 100, 128) == 0
 
 

@@ -109,3 +109,39 @@ def test_headline_shape_eight_heads():
                 errs[name] = (float(np.abs(g - want).max()) / max(float(np.abs(want).max()), 1e-30),
                               float(np.linalg.norm(g - want)) / max(float(np.linalg.norm(want)), 1e-30))
             check(errs)
+
+
+def test_rectangular_full():
+    # no mask, more key tiles than query tiles and ragged on both sides
+    check(run_bwd(1, 4, 2, 200, 650, 128, False, seed=80))
+
+
+def test_no_keys_gives_zero_dq():
+    """Skv = 0: the dQ kernel sees no key tile and writes zeros."""
+    B, Hq, Hkv, Sq, d = 1, 2, 1, 200, 128
+    q = torch.randn(B, Hq, Sq, d, device="cuda").to(torch.bfloat16)
+    k = torch.empty(B, Hkv, 0, d, device="cuda", dtype=torch.bfloat16)
+    v = torch.empty_like(k)
+    o = torch.zeros_like(q)
+    lse = torch.full((B, Hq, Sq), -math.inf, device="cuda")
+    d_o = torch.randn_like(q)
+    dq, dk, dv = fa.attention_backward(q, k, v, o, lse, d_o, True, 0.088)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(dq).item() == 0
+    assert dk.numel() == 0 and dv.numel() == 0
+
+
+def test_repeat_calls_bit_identical():
+    """Each gradient is accumulated in one CTA's tensor memory and written
+    once, so two calls give the same bits."""
+    q, k, v = prefill_inputs(2, 4, 2, 520, 520, 128, 90, 1.0)
+    d_o = grad_output((2, 4, 520, 128), 90)
+    qc, kc, vc, doc = (t.cuda() for t in (q, k, v, d_o))
+    o = torch.empty_like(qc)
+    lse = torch.empty((2, 4, 520), device="cuda", dtype=torch.float32)
+    fa.fa_fwd(qc, kc, vc, o, lse, True, 0.088)
+    first = fa.attention_backward(qc, kc, vc, o, lse, doc, True, 0.088)
+    second = fa.attention_backward(qc, kc, vc, o, lse, doc, True, 0.088)
+    torch.cuda.synchronize()
+    for a, b in zip(first, second):
+        assert torch.equal(a, b)
