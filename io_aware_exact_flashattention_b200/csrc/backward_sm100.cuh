@@ -24,7 +24,8 @@
 //
 // fa_bwd_dq_kernel -- one CTA per (batch, query head, 128-query tile i).
 //   Q_i and dO_i stay in shared memory, dQ_i accumulates in TMEM while the
-//   key tiles the queries see stream past (two-stage ring):
+//   key tiles the queries see stream past (K in a three-stage ring, V in a
+//   two-stage one: K_j is read last by dQ_j, V_j already by dP_j):
 //     S   = Q_i K_j^T       (M=128 queries, N=128 keys; SS), two buffers
 //     dP  = dO_i V_j^T      (M=128 queries, N=128 keys; SS)
 //     dQ += dS K_j          (A = dS packed in the S buffer; B = K_j MN-major; TS)
@@ -312,18 +313,24 @@ __device__ __forceinline__ void bwd_kv_elementwise(const BwdParams& p, uint32_t 
   const int off = p.Skv - p.Sq;
   const int i0 = bwd_first_q_tile(p, j);
   uint32_t n = 0;
-  // -LSE (in log2 units) and D of this thread's query for a tile: loaded one
-  // tile ahead, so the load latency hides behind the previous tile's work.
-  // Query rows past Sq take -LSE = -inf, so their weights are exactly 0.
-  auto load_ld = [&](int hh_, int i_, float& lse_v, float& d_v) {
+  // LSE and D of this thread's query for a tile: loaded one tile ahead into
+  // registers that nothing reads until the next tile, so the load latency
+  // hides behind this tile's work (a use right after the load would stall
+  // the warp).  Rows past Sq are marked invalid and take -LSE = -inf below,
+  // so their weights are exactly 0.
+  auto load_ld = [&](int hh_, int i_, float& lse_v, float& d_v, bool& valid) {
     const int c = hf * kQH + t;
     const int q = i_ * kBwdBN + c;
     const size_t rb = (static_cast<size_t>(b) * p.Hq + g * p.group + hh_) * p.Sq;
-    lse_v = (t < kQH && q < p.Sq) ? p.lse[rb + q] * -1.4426950408889634f : -INFINITY;
-    d_v = (t < kQH && q < p.Sq) ? p.dsum[rb + q] : 0.f;
+    valid = (t < kQH && q < p.Sq);
+    if (valid) {
+      lse_v = p.lse[rb + q];
+      d_v = p.dsum[rb + q];
+    }
   };
-  float lse_next = -INFINITY, d_next = 0.f;
-  if (i0 < p.n_q_tiles) load_ld(0, i0, lse_next, d_next);
+  float lse_next = 0.f, d_next = 0.f;
+  bool valid_next = false;
+  if (i0 < p.n_q_tiles) load_ld(0, i0, lse_next, d_next, valid_next);
   // After a failed wait a warp skips the remaining work but still takes every
   // named barrier, so the other warps of its warpgroup can never block there.
   bool ok = true;
@@ -331,17 +338,17 @@ __device__ __forceinline__ void bwd_kv_elementwise(const BwdParams& p, uint32_t 
     for (int i = i0; i < p.n_q_tiles; ++i, ++n) {
       const uint32_t ph = n & 1u;
       const int q0 = i * kBwdBN;
-      // this warpgroup's 64 queries: -LSE and D into shared memory
+      // this warpgroup's 64 queries: -LSE (log2 units) and D into shared memory
       named_barrier(1 + hf, 128);
       if (t < kQH) {
-        lse_s[hf * kQH + t] = lse_next;
-        d_s[hf * kQH + t] = d_next;
+        lse_s[hf * kQH + t] = valid_next ? lse_next * -1.4426950408889634f : -INFINITY;
+        d_s[hf * kQH + t] = valid_next ? d_next : 0.f;
       }
       named_barrier(1 + hf, 128);
       {  // next tile's values (same head, or the next head's first tile)
         const bool more_i = (i + 1 < p.n_q_tiles);
-        if (more_i) load_ld(hh, i + 1, lse_next, d_next);
-        else if (hh + 1 < p.group) load_ld(hh + 1, i0, lse_next, d_next);
+        if (more_i) load_ld(hh, i + 1, lse_next, d_next, valid_next);
+        else if (hh + 1 < p.group) load_ld(hh + 1, i0, lse_next, d_next, valid_next);
       }
 
       if (!ok) continue;
@@ -352,32 +359,35 @@ __device__ __forceinline__ void bwd_kv_elementwise(const BwdParams& p, uint32_t 
       tc_fence_after();
       uint32_t pk[kQH / 2];
       {
-        uint32_t ra[64];
-        tmem_ld64_nowait(t_s + hf * kQH, ra);
-        tmem_ld_wait_hold(ra);
         const int lim = key - off;  // first query that sees this key
         const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
         const bool all_vis = (key < p.Skv) && (!p.causal || q0 + hf * kQH >= lim);
-        if (__all_sync(0xffffffffu, all_vis)) {
+        const bool fast = __all_sync(0xffffffffu, all_vis);
 #pragma unroll
-          for (int c2 = 0; c2 < kQH / 2; ++c2) {
-            const float2 nl = *reinterpret_cast<const float2*>(lse_s + hf * kQH + 2 * c2);
-            const float2 x = ffma2(make_float2(__uint_as_float(ra[2 * c2]),
-                                               __uint_as_float(ra[2 * c2 + 1])), sl2, nl);
-            pk[c2] = pack_bf16x2(ex2(x.x), ex2(x.y));
-          }
-        } else {
+        for (int hq = 0; hq < 2; ++hq) {  // 32 queries per pass
+          uint32_t ra[32];
+          tmem_ld32(t_s + hf * kQH + hq * 32, ra);
+          if (fast) {
 #pragma unroll
-          for (int c2 = 0; c2 < kQH / 2; ++c2) {
-            float pr[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int c = hf * kQH + 2 * c2 + e;
-              const bool vis = (key < p.Skv) && (!p.causal || q0 + c >= lim);
-              const float x = fmaf(__uint_as_float(ra[2 * c2 + e]), p.scale_log2, lse_s[c]);
-              pr[e] = vis ? ex2(x) : 0.f;
+            for (int c2 = 0; c2 < 16; ++c2) {
+              const float2 nl = *reinterpret_cast<const float2*>(lse_s + hf * kQH + hq * 32 + 2 * c2);
+              const float2 x = ffma2(make_float2(__uint_as_float(ra[2 * c2]),
+                                                 __uint_as_float(ra[2 * c2 + 1])), sl2, nl);
+              pk[hq * 16 + c2] = pack_bf16x2(ex2(x.x), ex2(x.y));
             }
-            pk[c2] = pack_bf16x2(pr[0], pr[1]);
+          } else {
+#pragma unroll
+            for (int c2 = 0; c2 < 16; ++c2) {
+              float pr[2];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int c = hf * kQH + hq * 32 + 2 * c2 + e;
+                const bool vis = (key < p.Skv) && (!p.causal || q0 + c >= lim);
+                const float x = fmaf(__uint_as_float(ra[2 * c2 + e]), p.scale_log2, lse_s[c]);
+                pr[e] = vis ? ex2(x) : 0.f;
+              }
+              pk[hq * 16 + c2] = pack_bf16x2(pr[0], pr[1]);
+            }
           }
         }
       }
@@ -520,19 +530,23 @@ template <int D>
 struct BwdQLayout {
   static constexpr int kTileBytes = 128 * D * 2;
   static constexpr int kBoxBytes = 128 * 128;
-  static constexpr int kStages = 2;
+  static constexpr int kKStages = 3;
+  static constexpr int kVStages = 2;
   static constexpr int kQOff = 0;
   static constexpr int kDoOff = kTileBytes;
-  static constexpr int kRingOff = 2 * kTileBytes;  // stage s: K at kRingOff + 2*s*tile, V after it
-  static constexpr int kBarOff = kRingOff + kStages * 2 * kTileBytes;
-  static constexpr int kBQ = 0;        // Q_i and dO_i loaded
-  static constexpr int kBKvFull = 1;   // [kStages]
-  static constexpr int kBKvEmpty = 3;  // [kStages]
-  static constexpr int kBSFull = 5;    // [2] one per S buffer
-  static constexpr int kBDpFull = 7;
-  static constexpr int kBDsFull = 8;   // 8 arrivals (one per element-wise warp)
-  static constexpr int kBDone = 9;
-  static constexpr int kNumBars = 10;
+  static constexpr int kKOff = 2 * kTileBytes;                    // K stage s at kKOff + s*tile
+  static constexpr int kVOff = kKOff + kKStages * kTileBytes;     // V stage s at kVOff + s*tile
+  static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
+  static constexpr int kBQ = 0;                          // Q_i and dO_i loaded
+  static constexpr int kBKFull = 1;                      // [kKStages]
+  static constexpr int kBKEmpty = kBKFull + kKStages;    // [kKStages]
+  static constexpr int kBVFull = kBKEmpty + kKStages;    // [kVStages]
+  static constexpr int kBVEmpty = kBVFull + kVStages;    // [kVStages]
+  static constexpr int kBSFull = kBVEmpty + kVStages;    // [2] one per S buffer
+  static constexpr int kBDpFull = kBSFull + 2;
+  static constexpr int kBDsFull = kBDpFull + 1;          // 8 arrivals (one per element-wise warp)
+  static constexpr int kBDone = kBDsFull + 1;
+  static constexpr int kNumBars = kBDone + 1;
   static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kAbortOff = kTmemSlotOff + 4;
   static constexpr int kBytes = kAbortOff + 4 + 1024;
@@ -582,33 +596,45 @@ __device__ __forceinline__ void bwd_q_producer(const CUtensorMap* tq, const CUte
     tma_load_3d(sbase + L::kQOff + kb * L::kBoxBytes, tq, bq, kb * 64, i * kBwdBN, b * p.Hq + h);
     tma_load_3d(sbase + L::kDoOff + kb * L::kBoxBytes, tdo, bq, kb * 64, i * kBwdBN, b * p.Hq + h);
   }
-  int jn = 0;  // key tiles loaded
+  int jn = 0;  // key tiles whose K and V were both issued
   for (; jn < nk; ++jn) {
-    const int s = jn % L::kStages;
-    const uint32_t use = static_cast<uint32_t>(jn / L::kStages);
-    if (!mbar_wait(bars + 8 * (L::kBKvEmpty + s), (use & 1u) ^ 1u, abort_flag, p.wait_limit_ns))
+    const int ks = jn % L::kKStages, vs = jn % L::kVStages;
+    if (!mbar_wait(bars + 8 * (L::kBKEmpty + ks),
+                   (static_cast<uint32_t>(jn / L::kKStages) & 1u) ^ 1u, abort_flag, p.wait_limit_ns))
       break;
-    const uint32_t full = bars + 8 * (L::kBKvFull + s);
-    const uint32_t ka = sbase + L::kRingOff + 2 * s * L::kTileBytes;
-    mbar_arrive_expect_tx(full, 2 * L::kTileBytes);
+    const uint32_t kfull = bars + 8 * (L::kBKFull + ks);
+    mbar_arrive_expect_tx(kfull, L::kTileBytes);
 #pragma unroll
-    for (int kb = 0; kb < D / 64; ++kb) {
-      tma_load_3d(ka + kb * L::kBoxBytes, tk, full, kb * 64, jn * kBwdBM, b * p.Hkv + g);
-      tma_load_3d(ka + L::kTileBytes + kb * L::kBoxBytes, tv, full, kb * 64, jn * kBwdBM,
-                  b * p.Hkv + g);
+    for (int kb = 0; kb < D / 64; ++kb)
+      tma_load_3d(sbase + L::kKOff + ks * L::kTileBytes + kb * L::kBoxBytes, tk, kfull, kb * 64,
+                  jn * kBwdBM, b * p.Hkv + g);
+    if (!mbar_wait(bars + 8 * (L::kBVEmpty + vs),
+                   (static_cast<uint32_t>(jn / L::kVStages) & 1u) ^ 1u, abort_flag, p.wait_limit_ns)) {
+      mbar_wait(kfull, static_cast<uint32_t>(jn / L::kKStages) & 1u, nullptr, p.wait_limit_ns);
+      break;
     }
+    const uint32_t vfull = bars + 8 * (L::kBVFull + vs);
+    mbar_arrive_expect_tx(vfull, L::kTileBytes);
+#pragma unroll
+    for (int kb = 0; kb < D / 64; ++kb)
+      tma_load_3d(sbase + L::kVOff + vs * L::kTileBytes + kb * L::kBoxBytes, tv, vfull, kb * 64,
+                  jn * kBwdBM, b * p.Hkv + g);
   }
   // drain: the CTA does not exit with copies in flight
   mbar_wait(bq, 0u, nullptr, p.wait_limit_ns);
-  for (int k = (jn > L::kStages ? jn - L::kStages : 0); k < jn; ++k)
-    mbar_wait(bars + 8 * (L::kBKvFull + k % L::kStages),
-              static_cast<uint32_t>(k / L::kStages) & 1u, nullptr, p.wait_limit_ns);
+  for (int k = (jn > L::kKStages ? jn - L::kKStages : 0); k < jn; ++k)
+    mbar_wait(bars + 8 * (L::kBKFull + k % L::kKStages),
+              static_cast<uint32_t>(k / L::kKStages) & 1u, nullptr, p.wait_limit_ns);
+  for (int k = (jn > L::kVStages ? jn - L::kVStages : 0); k < jn; ++k)
+    mbar_wait(bars + 8 * (L::kBVFull + k % L::kVStages),
+              static_cast<uint32_t>(k / L::kVStages) & 1u, nullptr, p.wait_limit_ns);
 }
 
 // Per key tile j: dQ_j once dS_j is announced (it reads dS_j from S buffer
-// j%2 and K_j), which frees the ring stage; then dP_{j+1} (the element-wise
-// warps have read dP_j before announcing dS_j) and S_{j+2} into buffer j%2
-// (after dQ_j, which reads it, in issue order).
+// j%2 and K_j), which frees K_j's stage; then dP_{j+1} (the element-wise
+// warps have read dP_j before announcing dS_j), which frees V_{j+1}'s stage
+// once done, and S_{j+2} into buffer j%2 (after dQ_j, which reads it, in
+// issue order).
 template <int D>
 __device__ __forceinline__ void bwd_q_mma(const BwdParams& p, uint32_t sbase, uint32_t tmem,
                                           volatile int* abort_flag) {
@@ -624,48 +650,57 @@ __device__ __forceinline__ void bwd_q_mma(const BwdParams& p, uint32_t sbase, ui
     tc_fence_after();
     return true;
   };
-  auto kv_wait = [&](int jj) -> bool {
-    return wait(L::kBKvFull + jj % L::kStages, static_cast<uint32_t>(jj / L::kStages) & 1u);
+  auto k_wait = [&](int jj) -> bool {
+    return wait(L::kBKFull + jj % L::kKStages, static_cast<uint32_t>(jj / L::kKStages) & 1u);
+  };
+  auto v_wait = [&](int jj) -> bool {
+    return wait(L::kBVFull + jj % L::kVStages, static_cast<uint32_t>(jj / L::kVStages) & 1u);
   };
   const uint64_t q_km = sw128_desc(sbase + L::kQOff, 16, 1024);
   const uint64_t do_km = sw128_desc(sbase + L::kDoOff, 16, 1024);
-  const uint64_t k_km0 = sw128_desc(sbase + L::kRingOff, 16, 1024);
-  const uint64_t k_mn0 = sw128_desc(sbase + L::kRingOff, L::kBoxBytes, 1024);
-  constexpr uint64_t kStageStep = (2 * L::kTileBytes) >> 4;
-  constexpr uint64_t kVStep = L::kTileBytes >> 4;  // V after K
+  const uint64_t k_km0 = sw128_desc(sbase + L::kKOff, 16, 1024);
+  const uint64_t k_mn0 = sw128_desc(sbase + L::kKOff, L::kBoxBytes, 1024);
+  const uint64_t v_km0 = sw128_desc(sbase + L::kVOff, 16, 1024);
+  constexpr uint64_t kTileStep = L::kTileBytes >> 4;  // one stage, descriptor units
+  // dP_j = dO V_j^T, then V_j's stage is free once it completes
+  auto issue_dp = [&](int jj) {
+    const int vs = jj % L::kVStages;
+    bwd_gemm_kmajor<D>(t_dp, do_km, v_km0 + vs * kTileStep);
+    mma_commit(bars + 8 * L::kBDpFull);
+    mma_commit(bars + 8 * (L::kBVEmpty + vs));
+  };
   if (nk > 0) {
-    if (!wait(L::kBQ, 0u) || !kv_wait(0)) goto done;
+    if (!wait(L::kBQ, 0u) || !k_wait(0)) goto done;
     bwd_gemm_kmajor<D>(t_s0, q_km, k_km0);               // S_0 = Q K_0^T
     mma_commit(bars + 8 * (L::kBSFull + 0));
-    bwd_gemm_kmajor<D>(t_dp, do_km, k_km0 + kVStep);     // dP_0 = dO V_0^T
-    mma_commit(bars + 8 * L::kBDpFull);
+    if (!v_wait(0)) goto done;
+    issue_dp(0);
     if (nk > 1) {
-      if (!kv_wait(1)) goto done;
-      bwd_gemm_kmajor<D>(t_s0 + 128, q_km, k_km0 + kStageStep);
+      if (!k_wait(1)) goto done;
+      bwd_gemm_kmajor<D>(t_s0 + 128, q_km, k_km0 + kTileStep);
       mma_commit(bars + 8 * (L::kBSFull + 1));
     }
   }
   for (int jj = 0; jj < nk; ++jj) {
     const int buf = jj & 1;
-    const int s = jj % L::kStages;
+    const int ks = jj % L::kKStages;
     if (!wait(L::kBDsFull, static_cast<uint32_t>(jj) & 1u)) goto done;
-    const uint64_t k_mn = k_mn0 + s * kStageStep;
+    const uint64_t k_mn = k_mn0 + ks * kTileStep;
     const uint32_t t_ds = t_s0 + 128 * buf;
     static_for<kBwdBM / 16>([&](auto kk_c) {             // dQ += dS K (K-dim = keys)
       constexpr int kk = decltype(kk_c)::value;
       mma_ts_off<bwd_mn_off(kk)>(t_dq, t_ds + bwd_packed_col(kk), k_mn, kIdDq,
                                  (jj > 0 || kk > 0) ? 1u : 0u);
     });
-    mma_commit(bars + 8 * (L::kBKvEmpty + s));           // K_j, V_j consumed
-    if (jj + 1 < nk) {                                    // dP_{j+1}: V_{j+1} waited for with S_{j+1}
-      const int s1 = (jj + 1) % L::kStages;
-      bwd_gemm_kmajor<D>(t_dp, do_km, k_km0 + s1 * kStageStep + kVStep);
-      mma_commit(bars + 8 * L::kBDpFull);
+    mma_commit(bars + 8 * (L::kBKEmpty + ks));           // K_j consumed
+    if (jj + 1 < nk) {
+      if (!v_wait(jj + 1)) goto done;
+      issue_dp(jj + 1);
     }
     if (jj + 2 < nk) {                                    // S_{j+2} into buffer j%2
-      if (!kv_wait(jj + 2)) goto done;
-      const int s2 = (jj + 2) % L::kStages;
-      bwd_gemm_kmajor<D>(t_ds, q_km, k_km0 + s2 * kStageStep);
+      if (!k_wait(jj + 2)) goto done;
+      const int ks2 = (jj + 2) % L::kKStages;
+      bwd_gemm_kmajor<D>(t_ds, q_km, k_km0 + ks2 * kTileStep);
       mma_commit(bars + 8 * (L::kBSFull + buf));
     }
   }
@@ -809,9 +844,13 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const uint32_t bars = sbase + L::kBarOff;
   if (threadIdx.x == 0) {
     mbar_init(bars + 8 * L::kBQ, 1);
-    for (int s = 0; s < L::kStages; ++s) {
-      mbar_init(bars + 8 * (L::kBKvFull + s), 1);
-      mbar_init(bars + 8 * (L::kBKvEmpty + s), 1);
+    for (int s = 0; s < L::kKStages; ++s) {
+      mbar_init(bars + 8 * (L::kBKFull + s), 1);
+      mbar_init(bars + 8 * (L::kBKEmpty + s), 1);
+    }
+    for (int s = 0; s < L::kVStages; ++s) {
+      mbar_init(bars + 8 * (L::kBVFull + s), 1);
+      mbar_init(bars + 8 * (L::kBVEmpty + s), 1);
     }
     mbar_init(bars + 8 * (L::kBSFull + 0), 1);
     mbar_init(bars + 8 * (L::kBSFull + 1), 1);
