@@ -134,8 +134,9 @@ fa_status fa_fwd_fp8(const void *q, const void *k, const void *v, const float *d
  *   q, o, d_o, dq [B, Hq, Sq, d] bf16     k, v, dk, dv [B, Hkv, Skv, d] bf16
  *   lse           [B, Hq, Sq] fp32 (natural log, as fa_fwd writes it)
  *   workspace     fa_bwd_workspace_bytes(B, Hq, Sq, d) bytes, 16-byte aligned,
- *                 caller-owned scratch (D per query row, fp32); its contents
- *                 on entry do not matter
+ *                 caller-owned scratch (per 128-row query tile, -LSE*log2(e)
+ *                 and D = dO . O of each row, fp32); its contents on entry
+ *                 do not matter
  *   causal, scale: as passed to fa_fwd.
  *
  * dq, dk, dv are written once each (dk = dv = 0 for keys no query sees, dq = 0
@@ -152,7 +153,8 @@ fa_status fa_bwd(const void *q, const void *k, const void *v, const void *o,
                  float *workspace, int B, int Hq, int Hkv, int Sq, int Skv, int d,
                  int causal, float scale, fa_stream_t stream);
 
-/* Bytes of scratch fa_bwd needs: B * Hq * Sq floats (0 for empty); d is unused. */
+/* Bytes of scratch fa_bwd needs: B * Hq * ceil(Sq / 128) * 256 floats (0 for
+ * empty); d is unused. */
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Sq, int d);
 
 /*

@@ -52,8 +52,9 @@ constexpr int kBwdBM = 128;  // keys per key tile
 constexpr int kBwdBN = 128;  // queries per query tile
 
 struct BwdParams {
-  const float* lse;    // [B, Hq, Sq] natural log
-  const float* dsum;   // [B, Hq, Sq]: D = dO . O
+  // per (batch, query head, 128-row query tile): 128 values of -LSE*log2(e)
+  // then 128 values of D = dO . O (rows past Sq: -inf and 0), 1 KB per tile
+  const float* ld;
   __nv_bfloat16* dq;   // [B, Hq, Sq, d]
   __nv_bfloat16* dk;   // [B, Hkv, Skv, d]
   __nv_bfloat16* dv;
@@ -65,27 +66,46 @@ struct BwdParams {
 };
 
 // ---------------------------------------------------------------------------
-// D = rowsum(dO * O) for every query row (one warp per row).
+// Per query row (one warp per row, rows padded to whole 128-row tiles):
+// D = rowsum(dO * O) and -LSE*log2(e), packed per tile as the backward
+// kernels read them (a tile's 1 KB is one bulk copy).  Rows past Sq get
+// -LSE*log2(e) = -inf and D = 0, so their weights and dS are exactly 0.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_dsum_kernel(const __nv_bfloat16* __restrict__ o,
                                                           const __nv_bfloat16* __restrict__ d_o,
-                                                          float* __restrict__ dsum,
-                                                          long long rows) {
+                                                          const float* __restrict__ lse,
+                                                          float* __restrict__ ld, int Sq,
+                                                          int n_q_tiles, long long rows_padded) {
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
+  if (row >= rows_padded) return;
+  const long long per_head = static_cast<long long>(n_q_tiles) * 128;
+  const long long bh = row / per_head;
+  const int qq = static_cast<int>(row - bh * per_head);
+  float* dst = ld + (bh * n_q_tiles + qq / 128) * 256 + (qq & 127);
+  if (qq >= Sq) {
+    if (lane == 0) {
+      dst[0] = -INFINITY;
+      dst[128] = 0.f;
+    }
+    return;
+  }
+  const long long src = bh * Sq + qq;
   float acc = 0.f;
 #pragma unroll
   for (int c = lane * 2; c < D; c += 64) {
-    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(o + row * D + c);
-    const __nv_bfloat162 y = *reinterpret_cast<const __nv_bfloat162*>(d_o + row * D + c);
+    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(o + src * D + c);
+    const __nv_bfloat162 y = *reinterpret_cast<const __nv_bfloat162*>(d_o + src * D + c);
     acc = fmaf(__bfloat162float(x.x), __bfloat162float(y.x), acc);
     acc = fmaf(__bfloat162float(x.y), __bfloat162float(y.y), acc);
   }
 #pragma unroll
   for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-  if (lane == 0) dsum[row] = acc;
+  if (lane == 0) {
+    dst[0] = lse[src] * -1.4426950408889634f;
+    dst[128] = acc;
+  }
 }
 
 // Offsets (16-byte descriptor units) of K step kk in a 128B-swizzled tile.
@@ -125,8 +145,10 @@ struct BwdKvLayout {
   static constexpr int kVOff = kTileBytes;
   static constexpr int kQOff = 2 * kTileBytes;  // stage s: Q at kQOff + 2*s*tile, dO after it
   static constexpr int kDsOff = 6 * kTileBytes;  // dS^T: 128 keys x 128 queries bf16 (2 boxes)
-  static constexpr int kLseOff = kDsOff + 128 * 128 * 2;  // [128] -LSE*log2(e), [128] D
-  static constexpr int kBarOff = kLseOff + 2 * 128 * 4;
+  // stage s: the query tile's 128 values of -LSE*log2(e), then 128 of D
+  static constexpr int kLdOff = kDsOff + 128 * 128 * 2;
+  static constexpr int kLdBytes = 2 * 128 * 4;
+  static constexpr int kBarOff = kLdOff + 2 * kLdBytes;
   static constexpr int kBKv = 0;
   static constexpr int kBQFull = 1;    // [2]
   static constexpr int kBQEmpty = 3;   // [2]
@@ -135,12 +157,16 @@ struct BwdKvLayout {
   static constexpr int kBPFull = 7;    // 8 arrivals (one per element-wise warp)
   static constexpr int kBDsFull = 8;   // 8 arrivals
   static constexpr int kBDone = 9;
-  static constexpr int kNumBars = 10;
+  static constexpr int kBStaged = 10;  // 8 arrivals: dK, dV staged for the stores
+  static constexpr int kNumBars = 11;
   static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kAbortOff = kTmemSlotOff + 4;
-  static constexpr int kBytes = kAbortOff + 4 + 1024;  // + slack for 1024-byte alignment
+  static constexpr int kContent = kAbortOff + 4;
+  // slack for aligning the base to 1024 bytes, as far as the 227 KB allow
+  // (the kernel checks that the pad it needs fits)
+  static constexpr int kBytes = kContent + 1024 <= 232448 ? kContent + 1024 : 232448;
 };
-static_assert(BwdKvLayout<128>::kBytes <= 232448, "dK/dV shared memory over the limit");
+static_assert(BwdKvLayout<128>::kContent <= 232448, "dK/dV shared memory over the limit");
 
 // First query tile that sees any key of key tile j (causal: key k is visible
 // to query q iff k <= q + Skv - Sq).
@@ -200,12 +226,14 @@ __device__ __forceinline__ void bwd_kv_producer(const CUtensorMap* tq, const CUt
         goto drain;
       const uint32_t full = bars + 8 * (L::kBQFull + s);
       const uint32_t qa = sbase + L::kQOff + 2 * s * L::kTileBytes;
-      mbar_arrive_expect_tx(full, 2 * L::kTileBytes);
+      mbar_arrive_expect_tx(full, 2 * L::kTileBytes + L::kLdBytes);
 #pragma unroll
       for (int kb = 0; kb < D / 64; ++kb) {
         tma_load_3d(qa + kb * L::kBoxBytes, tq, full, kb * 64, i * kBwdBN, plane);
         tma_load_3d(qa + L::kTileBytes + kb * L::kBoxBytes, tdo, full, kb * 64, i * kBwdBN, plane);
       }
+      bulk_load(sbase + L::kLdOff + s * L::kLdBytes,
+                p.ld + (static_cast<size_t>(plane) * p.n_q_tiles + i) * 256, L::kLdBytes, full);
     }
   }
 drain:
@@ -293,6 +321,8 @@ done:
 template <int D>
 __device__ __forceinline__ void bwd_kv_elementwise(const BwdParams& p, uint32_t sbase,
                                                    uint8_t* smem, uint32_t tmem,
+                                                   const CUtensorMap* tm_dk,
+                                                   const CUtensorMap* tm_dv,
                                                    volatile int* abort_flag) {
   using L = BwdKvLayout<D>;
   const uint32_t bars = sbase + L::kBarOff;
@@ -304,8 +334,6 @@ __device__ __forceinline__ void bwd_kv_elementwise(const BwdParams& p, uint32_t 
   const uint32_t t_s = tmem + lane_off + 256, t_dp = tmem + lane_off + 384;
   constexpr int kQH = kBwdBN / 2;   // queries per warpgroup
   constexpr int kDH = D / 2;        // d-columns per warpgroup
-  float* lse_s = reinterpret_cast<float*>(smem + L::kLseOff);
-  float* d_s = lse_s + 128;
   uint8_t* ds_smem = smem + L::kDsOff;
   int b, g, j;
   bwd_kv_cta(p, b, g, j);
@@ -313,49 +341,22 @@ __device__ __forceinline__ void bwd_kv_elementwise(const BwdParams& p, uint32_t 
   const int off = p.Skv - p.Sq;
   const int i0 = bwd_first_q_tile(p, j);
   uint32_t n = 0;
-  // LSE and D of this thread's query for a tile: loaded one tile ahead into
-  // registers that nothing reads until the next tile, so the load latency
-  // hides behind this tile's work (a use right after the load would stall
-  // the warp).  Rows past Sq are marked invalid and take -LSE = -inf below,
-  // so their weights are exactly 0.
-  auto load_ld = [&](int hh_, int i_, float& lse_v, float& d_v, bool& valid) {
-    const int c = hf * kQH + t;
-    const int q = i_ * kBwdBN + c;
-    const size_t rb = (static_cast<size_t>(b) * p.Hq + g * p.group + hh_) * p.Sq;
-    valid = (t < kQH && q < p.Sq);
-    if (valid) {
-      lse_v = p.lse[rb + q];
-      d_v = p.dsum[rb + q];
-    }
-  };
-  float lse_next = 0.f, d_next = 0.f;
-  bool valid_next = false;
-  if (i0 < p.n_q_tiles) load_ld(0, i0, lse_next, d_next, valid_next);
-  // After a failed wait a warp skips the remaining work but still takes every
-  // named barrier, so the other warps of its warpgroup can never block there.
   bool ok = true;
-  for (int hh = 0; hh < p.group; ++hh) {
+  for (int hh = 0; hh < p.group && ok; ++hh) {
     for (int i = i0; i < p.n_q_tiles; ++i, ++n) {
       const uint32_t ph = n & 1u;
       const int q0 = i * kBwdBN;
-      // this warpgroup's 64 queries: -LSE (log2 units) and D into shared memory
-      named_barrier(1 + hf, 128);
-      if (t < kQH) {
-        lse_s[hf * kQH + t] = valid_next ? lse_next * -1.4426950408889634f : -INFINITY;
-        d_s[hf * kQH + t] = valid_next ? d_next : 0.f;
-      }
-      named_barrier(1 + hf, 128);
-      {  // next tile's values (same head, or the next head's first tile)
-        const bool more_i = (i + 1 < p.n_q_tiles);
-        if (more_i) load_ld(hh, i + 1, lse_next, d_next, valid_next);
-        else if (hh + 1 < p.group) load_ld(hh + 1, i0, lse_next, d_next, valid_next);
-      }
-
-      if (!ok) continue;
+      // the tile's -LSE (log2 units) and D arrived with its Q and dO (the
+      // stage is reloaded only after dK_n, which follows this tile's dS)
+      const float* lse_s = reinterpret_cast<const float*>(smem + L::kLdOff + (n & 1u) * L::kLdBytes);
+      const float* d_s = lse_s + 128;
+      ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (L::kBQFull + (n & 1u)), (n >> 1) & 1u,
+                                             abort_flag, p.wait_limit_ns));
+      if (!ok) break;
       // P^T for this key and the warpgroup's queries: p = 2^(s*scale*log2e - LSE*log2e)
       // (a key that every query of the half sees takes the branch without masks)
       ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * L::kBSFull, ph, abort_flag, p.wait_limit_ns));
-      if (!ok) continue;
+      if (!ok) break;
       tc_fence_after();
       uint32_t pk[kQH / 2];
       {
@@ -402,7 +403,7 @@ __device__ __forceinline__ void bwd_kv_elementwise(const BwdParams& p, uint32_t 
       // dS = P * (dP - D) to shared memory: rows = keys, 64-query boxes, 128B
       // swizzle (the K-major A operand of dK += dS^T Q)
       ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * L::kBDpFull, ph, abort_flag, p.wait_limit_ns));
-      if (!ok) continue;
+      if (!ok) break;
       tc_fence_after();
 #pragma unroll
       for (int hq = 0; hq < 2; ++hq) {  // 32 queries per pass
@@ -436,36 +437,51 @@ __device__ __forceinline__ void bwd_kv_elementwise(const BwdParams& p, uint32_t 
   if (!ok) return;
 
   // dK = scale * (dS^T Q summed), dV = P^T dO summed: thread t = key row,
-  // this warpgroup's d-columns
+  // this warpgroup's d-columns, staged as 128B-swizzled boxes in the (now
+  // idle) Q/dO ring and written by tiled bulk stores, which skip rows past Skv.
   if (!__all_sync(0xffffffffu, mbar_wait(bars + 8 * L::kBDone, 0u, abort_flag, p.wait_limit_ns)))
     return;
   tc_fence_after();
   const bool any = (i0 < p.n_q_tiles);
-  // tcgen05.ld is warp-collective: every thread loads, only rows of real keys
-  // are stored.
-  const bool real = key < p.Skv;
-  const size_t krow = (static_cast<size_t>(b) * p.Hkv + g) * p.Skv + (real ? key : 0);
+  constexpr int kBoxes = D / 64;  // 64-column boxes per gradient tile
 #pragma unroll
   for (int which = 0; which < 2; ++which) {
-    __nv_bfloat16* out = (which == 0 ? p.dv : p.dk) + krow * D + hf * kDH;
     const float mul = (which == 0) ? 1.f : p.scale;
+    uint8_t* stage = smem + L::kQOff + which * kBoxes * L::kBoxBytes;
 #pragma unroll
     for (int c4 = 0; c4 < kDH / 32; ++c4) {
       uint32_t r[32];
       tmem_ld32((which == 0 ? t_dv : t_dk) + hf * kDH + c4 * 32, r);
-      if (real) {
+      const int col0 = hf * kDH + c4 * 32;  // first d-column of these 32
 #pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4) {
-          uint4 w;
-          const float* f = reinterpret_cast<const float*>(r) + v4 * 8;
-          w.x = pack_bf16x2(any ? f[0] * mul : 0.f, any ? f[1] * mul : 0.f);
-          w.y = pack_bf16x2(any ? f[2] * mul : 0.f, any ? f[3] * mul : 0.f);
-          w.z = pack_bf16x2(any ? f[4] * mul : 0.f, any ? f[5] * mul : 0.f);
-          w.w = pack_bf16x2(any ? f[6] * mul : 0.f, any ? f[7] * mul : 0.f);
-          reinterpret_cast<uint4*>(out + c4 * 32)[v4] = w;
-        }
+      for (int v4 = 0; v4 < 4; ++v4) {
+        const float* f = reinterpret_cast<const float*>(r) + v4 * 8;
+        const int col = col0 + v4 * 8;
+        const int chunk = (col & 63) >> 3;
+        uint4* dst = reinterpret_cast<uint4*>(stage + (col >> 6) * L::kBoxBytes + t * 128 +
+                                              ((chunk ^ (t & 7)) * 16));
+        *dst = make_uint4(pack_bf16x2(any ? f[0] * mul : 0.f, any ? f[1] * mul : 0.f),
+                          pack_bf16x2(any ? f[2] * mul : 0.f, any ? f[3] * mul : 0.f),
+                          pack_bf16x2(any ? f[4] * mul : 0.f, any ? f[5] * mul : 0.f),
+                          pack_bf16x2(any ? f[6] * mul : 0.f, any ? f[7] * mul : 0.f));
       }
     }
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bars + 8 * L::kBStaged);
+  // one thread stores once every warp has staged its rows (a bounded wait:
+  // a warp that gave up earlier never arrives, and then nothing is stored)
+  if (threadIdx.x == 0 && mbar_wait(bars + 8 * L::kBStaged, 0u, abort_flag, p.wait_limit_ns)) {
+#pragma unroll
+    for (int which = 0; which < 2; ++which)
+#pragma unroll
+      for (int kb = 0; kb < kBoxes; ++kb)
+        tma_store_3d(which == 0 ? tm_dv : tm_dk,
+                     sbase + L::kQOff + (which * kBoxes + kb) * L::kBoxBytes, kb * 64,
+                     j * kBwdBM, b * p.Hkv + g);
+    bulk_commit_group();
+    bulk_wait_group0();
   }
 }
 
@@ -473,11 +489,16 @@ template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                   const BwdParams p) {
+                   const __grid_constant__ CUtensorMap tm_dk,
+                   const __grid_constant__ CUtensorMap tm_dv, const BwdParams p) {
   using L = BwdKvLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+  if (pad + L::kContent > static_cast<uint32_t>(L::kBytes)) {  // uniform: every thread leaves
+    if (threadIdx.x == 0) atomicExch(&g_device_status, kStatusTimeout);
+    return;
+  }
   uint8_t* smem = smem_raw + pad;
   const uint32_t sbase = raw + pad;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -494,6 +515,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     mbar_init(bars + 8 * L::kBPFull, 8);   // one arrival per element-wise warp
     mbar_init(bars + 8 * L::kBDsFull, 8);
     mbar_init(bars + 8 * L::kBDone, 1);
+    mbar_init(bars + 8 * L::kBStaged, 8);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -507,7 +529,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlotOff);
 
   if (warp < 8) {
-    bwd_kv_elementwise<D>(p, sbase, smem, tmem, abort_flag);
+    bwd_kv_elementwise<D>(p, sbase, smem, tmem, &tm_dk, &tm_dv, abort_flag);
   } else if (warp == 8) {
     if (lane == 0) bwd_kv_producer<D>(&tm_q, &tm_k, &tm_v, &tm_do, p, sbase, abort_flag);
   } else {
@@ -546,10 +568,12 @@ struct BwdQLayout {
   static constexpr int kBDpFull = kBSFull + 2;
   static constexpr int kBDsFull = kBDpFull + 1;          // 8 arrivals (one per element-wise warp)
   static constexpr int kBDone = kBDsFull + 1;
-  static constexpr int kNumBars = kBDone + 1;
+  static constexpr int kBStaged = kBDone + 1;            // 8 arrivals: dQ staged for the stores
+  static constexpr int kNumBars = kBStaged + 1;
   static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kAbortOff = kTmemSlotOff + 4;
-  static constexpr int kBytes = kAbortOff + 4 + 1024;
+  static constexpr int kContent = kAbortOff + 4;
+  static constexpr int kBytes = kContent + 1024 <= 232448 ? kContent + 1024 : 232448;
 };
 static_assert(BwdQLayout<128>::kBytes <= 232448, "dQ shared memory over the limit");
 
@@ -714,7 +738,9 @@ done:
 // [hf*D/2, (hf+1)*D/2) of dQ at the end.
 template <int D>
 __device__ __forceinline__ void bwd_q_elementwise(const BwdParams& p, uint32_t sbase,
-                                                  uint32_t tmem, volatile int* abort_flag) {
+                                                  uint8_t* smem, uint32_t tmem,
+                                                  const CUtensorMap* tm_dq,
+                                                  volatile int* abort_flag) {
   using L = BwdQLayout<D>;
   const uint32_t bars = sbase + L::kBarOff;
   const int hf = threadIdx.x >> 7;
@@ -728,11 +754,10 @@ __device__ __forceinline__ void bwd_q_elementwise(const BwdParams& p, uint32_t s
   bwd_q_cta(p, b, h, i);
   const int nk = bwd_q_kv_tiles(p, i);
   const int q = i * kBwdBN + row;
-  const bool real = q < p.Sq;
-  const size_t qrow = (static_cast<size_t>(b) * p.Hq + h) * p.Sq + (real ? q : 0);
   // -LSE in log2 units (rows past Sq: -inf, weights exactly 0) and D
-  const float nlse = real ? p.lse[qrow] * -1.4426950408889634f : -INFINITY;
-  const float dval = real ? p.dsum[qrow] : 0.f;
+  const float* ldt = p.ld + (static_cast<size_t>(b * p.Hq + h) * p.n_q_tiles + i) * 256;
+  const float nlse = ldt[row];
+  const float dval = ldt[128 + row];
   const int off = p.Skv - p.Sq;
   const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
   const float2 nl2 = make_float2(nlse, nlse);
@@ -803,7 +828,9 @@ __device__ __forceinline__ void bwd_q_elementwise(const BwdParams& p, uint32_t s
       return;
     tc_fence_after();
   }
-  __nv_bfloat16* out = p.dq + qrow * D + hf * kDH;
+  // staged as 128B-swizzled boxes in the (now idle) Q/dO buffers and written
+  // by tiled bulk stores, which skip rows past Sq
+  uint8_t* stage = smem + L::kQOff;
 #pragma unroll
   for (int c4 = 0; c4 < kDH / 32; ++c4) {
     uint32_t r[32];
@@ -813,18 +840,30 @@ __device__ __forceinline__ void bwd_q_elementwise(const BwdParams& p, uint32_t s
 #pragma unroll
       for (int e = 0; e < 32; ++e) r[e] = 0u;
     }
-    if (real) {
+    const int col0 = hf * kDH + c4 * 32;
 #pragma unroll
-      for (int v4 = 0; v4 < 4; ++v4) {
-        uint4 w;
-        const float* f = reinterpret_cast<const float*>(r) + v4 * 8;
-        w.x = pack_bf16x2(f[0] * p.scale, f[1] * p.scale);
-        w.y = pack_bf16x2(f[2] * p.scale, f[3] * p.scale);
-        w.z = pack_bf16x2(f[4] * p.scale, f[5] * p.scale);
-        w.w = pack_bf16x2(f[6] * p.scale, f[7] * p.scale);
-        reinterpret_cast<uint4*>(out + c4 * 32)[v4] = w;
-      }
+    for (int v4 = 0; v4 < 4; ++v4) {
+      const float* f = reinterpret_cast<const float*>(r) + v4 * 8;
+      const int col = col0 + v4 * 8;
+      const int chunk = (col & 63) >> 3;
+      uint4* dst = reinterpret_cast<uint4*>(stage + (col >> 6) * L::kBoxBytes + row * 128 +
+                                            ((chunk ^ (row & 7)) * 16));
+      *dst = make_uint4(pack_bf16x2(f[0] * p.scale, f[1] * p.scale),
+                        pack_bf16x2(f[2] * p.scale, f[3] * p.scale),
+                        pack_bf16x2(f[4] * p.scale, f[5] * p.scale),
+                        pack_bf16x2(f[6] * p.scale, f[7] * p.scale));
     }
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bars + 8 * L::kBStaged);
+  if (threadIdx.x == 0 && mbar_wait(bars + 8 * L::kBStaged, 0u, abort_flag, p.wait_limit_ns)) {
+#pragma unroll
+    for (int kb = 0; kb < D / 64; ++kb)
+      tma_store_3d(tm_dq, sbase + L::kQOff + kb * L::kBoxBytes, kb * 64, i * kBwdBN,
+                   b * p.Hq + h);
+    bulk_commit_group();
+    bulk_wait_group0();
   }
 }
 
@@ -832,11 +871,15 @@ template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                 const BwdParams p) {
+                 const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using L = BwdQLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+  if (pad + L::kContent > static_cast<uint32_t>(L::kBytes)) {  // uniform: every thread leaves
+    if (threadIdx.x == 0) atomicExch(&g_device_status, kStatusTimeout);
+    return;
+  }
   uint8_t* smem = smem_raw + pad;
   const uint32_t sbase = raw + pad;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -857,6 +900,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     mbar_init(bars + 8 * L::kBDpFull, 1);
     mbar_init(bars + 8 * L::kBDsFull, 8);  // one arrival per element-wise warp
     mbar_init(bars + 8 * L::kBDone, 1);
+    mbar_init(bars + 8 * L::kBStaged, 8);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -870,7 +914,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlotOff);
 
   if (warp < 8) {
-    bwd_q_elementwise<D>(p, sbase, tmem, abort_flag);
+    bwd_q_elementwise<D>(p, sbase, smem, tmem, &tm_dq, abort_flag);
   } else if (warp == 8) {
     if (lane == 0) bwd_q_producer<D>(&tm_q, &tm_k, &tm_v, &tm_do, p, sbase, abort_flag);
   } else {

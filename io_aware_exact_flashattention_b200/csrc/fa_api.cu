@@ -438,25 +438,32 @@ fa_status launch_backward(const void* q, const void* k, const void* v, const voi
                           const float* lse, const void* d_o, void* dq, void* dk, void* dv,
                           float* workspace, int B, int Hq, int Hkv, int Sq, int Skv, int causal,
                           float scale, cudaStream_t stream) {
-  const long long q_rows = static_cast<long long>(B) * Hq * Sq;
-  float* dsum = workspace;
-  if (Skv == 0) k = v = q;  // no key tile is ever loaded; any valid address will do
-  fa::fa_bwd_dsum_kernel<D><<<static_cast<unsigned>((q_rows + 7) / 8), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o), dsum, q_rows);
-  const int n_kv_tiles = (Skv + fa::kBwdBM - 1) / fa::kBwdBM;
   const int n_q_tiles = (Sq + fa::kBwdBN - 1) / fa::kBwdBN;
-  CUtensorMap tq, tk, tv, tdo;
+  const long long rows_padded = static_cast<long long>(B) * Hq * n_q_tiles * fa::kBwdBN;
+  float* ld = workspace;
+  // no key tile is loaded or stored without keys; any valid address will do
+  if (Skv == 0) {
+    k = v = q;
+    dk = dv = dq;
+  }
+  fa::fa_bwd_dsum_kernel<D><<<static_cast<unsigned>(rows_padded / 8), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o), lse, ld, Sq,
+      n_q_tiles, rows_padded);
+  const int n_kv_tiles = (Skv + fa::kBwdBM - 1) / fa::kBwdBM;
+  CUtensorMap tq, tk, tv, tdo, tdq, tdk, tdv;
   if (!encode_bhsd(&tq, q, D, Sq, static_cast<long long>(B) * Hq) ||
       !encode_bhsd(&tdo, d_o, D, Sq, static_cast<long long>(B) * Hq) ||
+      !encode_bhsd(&tdq, dq, D, Sq, static_cast<long long>(B) * Hq) ||
       !encode_bhsd(&tk, k, D, Skv, static_cast<long long>(B) * Hkv) ||
-      !encode_bhsd(&tv, v, D, Skv, static_cast<long long>(B) * Hkv))
+      !encode_bhsd(&tv, v, D, Skv, static_cast<long long>(B) * Hkv) ||
+      !encode_bhsd(&tdk, dk, D, Skv, static_cast<long long>(B) * Hkv) ||
+      !encode_bhsd(&tdv, dv, D, Skv, static_cast<long long>(B) * Hkv))
     return FA_ERR_CUDA;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
   if (prepare_backward(dev) != cudaSuccess) return FA_ERR_CUDA;
   fa::BwdParams p;
-  p.lse = lse;
-  p.dsum = dsum;
+  p.ld = ld;
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
@@ -478,12 +485,12 @@ fa_status launch_backward(const void* q, const void* k, const void* v, const voi
         std::max(1, std::min(B * Hkv, kBwdGroupWaves * g_bwd_sms[dev] / n_kv_tiles));
     const unsigned grid = static_cast<unsigned>(static_cast<long long>(B) * Hkv * n_kv_tiles);
     fa::fa_bwd_dkdv_kernel<D><<<grid, fa::kBwdThreads, fa::BwdKvLayout<D>::kBytes, stream>>>(
-        tq, tk, tv, tdo, p);
+        tq, tk, tv, tdo, tdk, tdv, p);
   }
   p.heads_per_group = 1;
   const unsigned qgrid = static_cast<unsigned>(static_cast<long long>(B) * Hq * n_q_tiles);
   fa::fa_bwd_dq_kernel<D><<<qgrid, fa::kBwdThreads, fa::BwdQLayout<D>::kBytes, stream>>>(
-      tq, tk, tv, tdo, p);
+      tq, tk, tv, tdo, tdq, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -519,7 +526,9 @@ extern "C" {
 
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Sq, int d) {
   if (B <= 0 || Hq <= 0 || Sq <= 0 || d <= 0) return 0;
-  return static_cast<size_t>(B) * Hq * Sq * sizeof(float);
+  // per 128-row query tile: 128 values of -LSE*log2(e) and 128 of D, fp32
+  const size_t tiles = (static_cast<size_t>(Sq) + 127) / 128;
+  return static_cast<size_t>(B) * Hq * tiles * 256 * sizeof(float);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -542,9 +551,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     return FA_ERR_ALIGNMENT;
   const long long n_kv_tiles = (static_cast<long long>(Skv) + fa::kBwdBM - 1) / fa::kBwdBM;
   const long long n_q_tiles = (static_cast<long long>(Sq) + fa::kBwdBN - 1) / fa::kBwdBN;
-  const long long q_rows = static_cast<long long>(B) * Hq * Sq;
   if (static_cast<long long>(B) * Hkv * n_kv_tiles > 0x7fffffffLL ||
-      static_cast<long long>(B) * Hq * n_q_tiles > 0x7fffffffLL || q_rows / 8 > 0x7fffffffLL ||
+      static_cast<long long>(B) * Hq * n_q_tiles * 16 > 0x7fffffffLL ||
       static_cast<long long>(B) * Hkv > 0x7fffffffLL)
     return FA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -241,7 +241,8 @@ def test_bpt_workspace_bytes(lib):
 
 
 def test_bwd_workspace_bytes(lib):
-    assert fa.bwd_workspace_bytes(2, 4, 100, 128) == 2 * 4 * 100 * 4
+    assert fa.bwd_workspace_bytes(2, 4, 100, 128) == 2 * 4 * 1 * 256 * 4
+    assert fa.bwd_workspace_bytes(2, 4, 300, 64) == 2 * 4 * 3 * 256 * 4
     assert fa.bwd_workspace_bytes(0, 4, 100, 128) == 0
 
 
