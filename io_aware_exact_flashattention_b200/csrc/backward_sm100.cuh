@@ -61,6 +61,7 @@ struct BwdParams {
   int B, Hq, Hkv, Sq, Skv, group, causal;
   int n_kv_tiles, n_q_tiles;
   int heads_per_group;  // dK/dV CTA order: groups of this many (b, kv-head) pairs
+  int n_kv_ctas;        // grid: the first n_kv_ctas CTAs are dK/dV CTAs, the rest dQ CTAs
   float scale, scale_log2;
   unsigned long long wait_limit_ns;
 };
@@ -185,8 +186,9 @@ __device__ __forceinline__ void bwd_kv_cta(const BwdParams& p, int& b, int& g, i
   // cover about two groups, whose Q and dO rows stay in L2 while all their
   // key tiles stream them.
   const int per_group = p.heads_per_group * p.n_kv_tiles;
-  const int grp = static_cast<int>(blockIdx.x) / per_group;
-  const int r = static_cast<int>(blockIdx.x) % per_group;
+  const int cta = static_cast<int>(blockIdx.x);  // dK/dV CTAs come first in the grid
+  const int grp = cta / per_group;
+  const int r = cta % per_group;
   const int units = p.B * p.Hkv;
   const int in_group = min(p.heads_per_group, units - grp * p.heads_per_group);
   j = r / in_group;
@@ -486,16 +488,25 @@ __device__ __forceinline__ void bwd_kv_elementwise(const BwdParams& p, uint32_t 
 }
 
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1)
-fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                   const __grid_constant__ CUtensorMap tm_dk,
-                   const __grid_constant__ CUtensorMap tm_dv, const BwdParams p) {
+struct BwdQLayout;
+
+// Shared memory of a backward CTA: the larger of the two roles' layouts.
+template <int D>
+__host__ __device__ constexpr int bwd_smem_bytes() {
+  return BwdKvLayout<D>::kBytes > BwdQLayout<D>::kBytes ? BwdKvLayout<D>::kBytes
+                                                         : BwdQLayout<D>::kBytes;
+}
+
+// One dK/dV CTA (the whole block).
+template <int D>
+__device__ __forceinline__ void bwd_dkdv_block(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                                               const CUtensorMap* tm_v, const CUtensorMap* tm_do,
+                                               const CUtensorMap* tm_dk, const CUtensorMap* tm_dv,
+                                               const BwdParams& p, uint8_t* smem_raw) {
   using L = BwdKvLayout<D>;
-  extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
-  if (pad + L::kContent > static_cast<uint32_t>(L::kBytes)) {  // uniform: every thread leaves
+  if (pad + L::kContent > static_cast<uint32_t>(bwd_smem_bytes<D>())) {  // uniform: every thread leaves
     if (threadIdx.x == 0) atomicExch(&g_device_status, kStatusTimeout);
     return;
   }
@@ -529,9 +540,9 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlotOff);
 
   if (warp < 8) {
-    bwd_kv_elementwise<D>(p, sbase, smem, tmem, &tm_dk, &tm_dv, abort_flag);
+    bwd_kv_elementwise<D>(p, sbase, smem, tmem, tm_dk, tm_dv, abort_flag);
   } else if (warp == 8) {
-    if (lane == 0) bwd_kv_producer<D>(&tm_q, &tm_k, &tm_v, &tm_do, p, sbase, abort_flag);
+    if (lane == 0) bwd_kv_producer<D>(tm_q, tm_k, tm_v, tm_do, p, sbase, abort_flag);
   } else {
     if (lane == 0) bwd_kv_mma<D>(p, sbase, tmem, abort_flag);
   }
@@ -581,8 +592,9 @@ static_assert(BwdQLayout<128>::kBytes <= 232448, "dQ shared memory over the limi
 // one with more keys than queries) the last query tiles see the most keys.
 __device__ __forceinline__ void bwd_q_cta(const BwdParams& p, int& b, int& h, int& i) {
   const int heads = p.B * p.Hq;
-  i = p.n_q_tiles - 1 - static_cast<int>(blockIdx.x) / heads;
-  const int bh = static_cast<int>(blockIdx.x) % heads;
+  const int cta = static_cast<int>(blockIdx.x) - p.n_kv_ctas;  // dQ CTAs follow the dK/dV ones
+  i = p.n_q_tiles - 1 - cta / heads;
+  const int bh = cta % heads;
   b = bh / p.Hq;
   h = bh % p.Hq;
 }
@@ -867,16 +879,16 @@ __device__ __forceinline__ void bwd_q_elementwise(const BwdParams& p, uint32_t s
   }
 }
 
+// One dQ CTA (the whole block).
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1)
-fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                 const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+__device__ __forceinline__ void bwd_dq_block(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                                             const CUtensorMap* tm_v, const CUtensorMap* tm_do,
+                                             const CUtensorMap* tm_dq, const BwdParams& p,
+                                             uint8_t* smem_raw) {
   using L = BwdQLayout<D>;
-  extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
-  if (pad + L::kContent > static_cast<uint32_t>(L::kBytes)) {  // uniform: every thread leaves
+  if (pad + L::kContent > static_cast<uint32_t>(bwd_smem_bytes<D>())) {  // uniform: every thread leaves
     if (threadIdx.x == 0) atomicExch(&g_device_status, kStatusTimeout);
     return;
   }
@@ -914,9 +926,9 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlotOff);
 
   if (warp < 8) {
-    bwd_q_elementwise<D>(p, sbase, smem, tmem, &tm_dq, abort_flag);
+    bwd_q_elementwise<D>(p, sbase, smem, tmem, tm_dq, abort_flag);
   } else if (warp == 8) {
-    if (lane == 0) bwd_q_producer<D>(&tm_q, &tm_k, &tm_v, &tm_do, p, sbase, abort_flag);
+    if (lane == 0) bwd_q_producer<D>(tm_q, tm_k, tm_v, tm_do, p, sbase, abort_flag);
   } else {
     if (lane == 0) bwd_q_mma<D>(p, sbase, tmem, abort_flag);
   }
@@ -928,6 +940,22 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+// The backward in one launch: CTAs [0, n_kv_ctas) take dK/dV key tiles
+// (heavy first), the rest dQ query tiles (heavy first).  Blocks start in
+// index order, so the dQ CTAs fill the SMs as the dK/dV tail drains.
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+              const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dk,
+              const __grid_constant__ CUtensorMap tm_dv, const BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  if (static_cast<int>(blockIdx.x) < p.n_kv_ctas)
+    bwd_dkdv_block<D>(&tm_q, &tm_k, &tm_v, &tm_do, &tm_dk, &tm_dv, p, smem_raw);
+  else
+    bwd_dq_block<D>(&tm_q, &tm_k, &tm_v, &tm_do, &tm_dq, p, smem_raw);
 }
 
 }  // namespace fa

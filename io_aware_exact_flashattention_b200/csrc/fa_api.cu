@@ -411,20 +411,11 @@ cudaError_t prepare_backward(int dev) {
   std::call_once(g_bwd_once[dev], [dev] {
     cudaError_t e = cudaDeviceGetAttribute(&g_bwd_sms[dev], cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(fa::fa_bwd_dkdv_kernel<64>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::BwdKvLayout<64>::kBytes);
+      e = cudaFuncSetAttribute(fa::fa_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::bwd_smem_bytes<64>());
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(fa::fa_bwd_dkdv_kernel<128>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::BwdKvLayout<128>::kBytes);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::BwdQLayout<64>::kBytes);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<128>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::BwdQLayout<128>::kBytes);
+      e = cudaFuncSetAttribute(fa::fa_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::bwd_smem_bytes<128>());
     g_bwd_err[dev] = e;
   });
   return g_bwd_err[dev];
@@ -479,18 +470,16 @@ fa_status launch_backward(const void* q, const void* k, const void* v, const voi
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_limit_ns = kWaitLimitNs;
-  if (n_kv_tiles > 0) {
-    // about kBwdGroupWaves waves of CTAs per group (one CTA per SM)
-    p.heads_per_group =
-        std::max(1, std::min(B * Hkv, kBwdGroupWaves * g_bwd_sms[dev] / n_kv_tiles));
-    const unsigned grid = static_cast<unsigned>(static_cast<long long>(B) * Hkv * n_kv_tiles);
-    fa::fa_bwd_dkdv_kernel<D><<<grid, fa::kBwdThreads, fa::BwdKvLayout<D>::kBytes, stream>>>(
-        tq, tk, tv, tdo, tdk, tdv, p);
-  }
-  p.heads_per_group = 1;
-  const unsigned qgrid = static_cast<unsigned>(static_cast<long long>(B) * Hq * n_q_tiles);
-  fa::fa_bwd_dq_kernel<D><<<qgrid, fa::kBwdThreads, fa::BwdQLayout<D>::kBytes, stream>>>(
-      tq, tk, tv, tdo, tdq, p);
+  // about kBwdGroupWaves waves of dK/dV CTAs per group (one CTA per SM)
+  p.heads_per_group =
+      n_kv_tiles > 0
+          ? std::max(1, std::min(B * Hkv, kBwdGroupWaves * g_bwd_sms[dev] / n_kv_tiles))
+          : 1;
+  p.n_kv_ctas = static_cast<int>(static_cast<long long>(B) * Hkv * n_kv_tiles);
+  const long long q_ctas = static_cast<long long>(B) * Hq * n_q_tiles;
+  const unsigned grid = static_cast<unsigned>(p.n_kv_ctas + q_ctas);
+  fa::fa_bwd_kernel<D><<<grid, fa::kBwdThreads, fa::bwd_smem_bytes<D>(), stream>>>(
+      tq, tk, tv, tdo, tdq, tdk, tdv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -551,7 +540,9 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     return FA_ERR_ALIGNMENT;
   const long long n_kv_tiles = (static_cast<long long>(Skv) + fa::kBwdBM - 1) / fa::kBwdBM;
   const long long n_q_tiles = (static_cast<long long>(Sq) + fa::kBwdBN - 1) / fa::kBwdBN;
-  if (static_cast<long long>(B) * Hkv * n_kv_tiles > 0x7fffffffLL ||
+  // one grid of dK/dV and dQ CTAs; the D kernel's grid has 16 blocks per query tile
+  if (static_cast<long long>(B) * Hkv * n_kv_tiles + static_cast<long long>(B) * Hq * n_q_tiles >
+          0x7fffffffLL ||
       static_cast<long long>(B) * Hq * n_q_tiles * 16 > 0x7fffffffLL ||
       static_cast<long long>(B) * Hkv > 0x7fffffffLL)
     return FA_ERR_UNSUPPORTED;
