@@ -50,6 +50,11 @@ namespace fa {
 constexpr int kBwdThreads = 320;
 constexpr int kBwdBM = 128;  // keys per key tile
 constexpr int kBwdBN = 128;  // queries per query tile
+// Of every 8 pairs of weights formed without masks in the dK/dV kernel, this
+// many use the FMA-pipe polynomial instead of the MUFU: on B200, 2 of 8 took
+// 2-3 % less time than none (in the dQ kernel, where the MUFU is not what
+// sets the tile period, it gained nothing and stays off).
+constexpr int kBwdPolyPairsPer8 = 2;
 
 struct BwdParams {
   // per (batch, query head, 128-row query tile): 128 values of -LSE*log2(e)
@@ -376,7 +381,12 @@ __device__ __forceinline__ void bwd_kv_elementwise(const BwdParams& p, uint32_t 
               const float2 nl = *reinterpret_cast<const float2*>(lse_s + hf * kQH + hq * 32 + 2 * c2);
               const float2 x = ffma2(make_float2(__uint_as_float(ra[2 * c2]),
                                                  __uint_as_float(ra[2 * c2 + 1])), sl2, nl);
-              pk[hq * 16 + c2] = pack_bf16x2(ex2(x.x), ex2(x.y));
+              if ((c2 & 7) >= 8 - kBwdPolyPairsPer8) {  // the FMA-pipe polynomial
+                const float2 e = exp2_poly2(x);
+                pk[hq * 16 + c2] = pack_bf16x2(e.x, e.y);
+              } else {
+                pk[hq * 16 + c2] = pack_bf16x2(ex2(x.x), ex2(x.y));
+              }
             }
           } else {
 #pragma unroll

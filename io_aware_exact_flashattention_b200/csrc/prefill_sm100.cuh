@@ -74,16 +74,6 @@ constexpr float kRescaleThreshold = 24.0f;  // log2 units
 constexpr float kRescaleThresholdF8 = 2.0f;  // log2 units, 8-bit P
 constexpr float kPOffsetF8 = 6.0f;           // 8-bit P is stored as p * 2^6
 
-// 2^x for part of the softmax on the FMA pipe instead of the MUFU: with
-// n = round(x) and f = x - n in [-1/2, 1/2], 2^x = 2^n * p(f) where p is the
-// degree-3 minimax fit of 2^f below (max relative error 7.5e-5; derived by
-// exp2_poly_fit.py next to this file).  2^n is applied by adding n to the
-// exponent field.  Arguments are clamped to >= -126; larger ones stay <= 24
-// because the reference max is never more than 2^24 below the row max.
-constexpr float kExp2C0 = 9.999280572e-01f;
-constexpr float kExp2C1 = 6.932609677e-01f;
-constexpr float kExp2C2 = 2.426111251e-01f;
-constexpr float kExp2C3 = 5.517166853e-02f;
 // Of every 8 pairs of scores, this many use the polynomial.  Off: on B200,
 // with the other choices in this kernel, every share tried (1 to 4 of 8)
 // took more cycles than the MUFU alone (2-7 %); the polynomial stays as a
@@ -94,21 +84,6 @@ constexpr int kPolyPairsPer8 = 0;
 // period: on B200, 2 of 8 pairs on the polynomial took 2.6 % (S = 2048) and
 // 4.4 % (S = 8192) less time than none, 3 of 8 about the same, 4 of 8 more.
 constexpr int kPolyPairsPer8F8 = 2;
-
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
-  const float2 t = fadd2(x, make_float2(kRound, kRound));
-  const float2 n = fadd2(t, make_float2(-kRound, -kRound));
-  const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
-  float2 q = ffma2(f, make_float2(kExp2C3, kExp2C3), make_float2(kExp2C2, kExp2C2));
-  q = ffma2(q, f, make_float2(kExp2C1, kExp2C1));
-  q = ffma2(q, f, make_float2(kExp2C0, kExp2C0));
-  // the low bits of t hold n, so (bits(t) << 23) == (n << 23) modulo 2^32
-  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
-}
 
 // D[tmem] (+)= A[smem] * B[smem], kind::f8f6f4 (A and B both E4M3 here).
 __device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,

@@ -363,6 +363,38 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
       : "memory");
 }
 
+// Packed two-wide fp32 arithmetic (sm_100): one instruction per pair.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+
+// 2^x for part of a softmax on the FMA pipe instead of the MUFU: with
+// n = round(x) and f = x - n in [-1/2, 1/2], 2^x = 2^n * p(f) where p is the
+// degree-3 minimax fit of 2^f below (max relative error 7.5e-5; derived by
+// exp2_poly_fit.py next to this file).  2^n is applied by adding n to the
+// exponent field.  Arguments are clamped to >= -126; callers keep them small
+// (at most 24 in the forward, whose reference max is never more than 2^24
+// below the row max; at most about 0 in the backward, where x is the score
+// minus the row's LSE).
+constexpr float kExp2C0 = 9.999280572e-01f;
+constexpr float kExp2C1 = 6.932609677e-01f;
+constexpr float kExp2C2 = 2.426111251e-01f;
+constexpr float kExp2C3 = 5.517166853e-02f;
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = fadd2(x, make_float2(kRound, kRound));
+  const float2 n = fadd2(t, make_float2(-kRound, -kRound));
+  const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
+  float2 q = ffma2(f, make_float2(kExp2C3, kExp2C3), make_float2(kExp2C2, kExp2C2));
+  q = ffma2(q, f, make_float2(kExp2C1, kExp2C1));
+  q = ffma2(q, f, make_float2(kExp2C0, kExp2C0));
+  // the low bits of t hold n, so (bits(t) << 23) == (n << 23) modulo 2^32
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (tensor-core operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -428,11 +460,6 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-
-// Packed two-wide fp32 arithmetic (sm_100): one instruction per pair.
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
-__device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
 // max of three (sm_100 three-input max)
 __device__ __forceinline__ float fmax3(float a, float b, float c) {

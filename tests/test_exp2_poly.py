@@ -1,4 +1,5 @@
-"""The polynomial 2^x used for part of the prefill softmax.
+"""The polynomial 2^x used for part of the softmax weights (the FP8 prefill
+and the backward's dK/dV kernel).
 
 CPU: the fit is re-derived from its definition (exp2_poly_fit.py, a Remez
 exchange for minimal relative error of a cubic on [-1/2, 1/2]); the kernel's
@@ -25,7 +26,7 @@ BOUND = 8e-5  # the fit's max relative error is 7.48e-5; fp32 evaluation adds < 
 
 
 def kernel_constants():
-    text = open(os.path.join(fabuild.CSRC, "prefill_sm100.cuh")).read()
+    text = open(os.path.join(fabuild.CSRC, "sm100.cuh")).read()
     return [float(re.search(r"kExp2C%d = ([0-9.eE+-]+)f;" % i, text).group(1)) for i in range(4)]
 
 
