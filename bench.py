@@ -577,11 +577,12 @@ def measure_extras(args, world, rank, dev, stream, flush, peaks, do_pre, do_dec,
                 {"value": aggregate_rate(world, bw_flops, K, bw_ms) / 1e12, "unit": "TFLOP/s",
                  "workload": ce.name, "ms_per_call": bw_ms / K},
                 **tensor_fracs(bw_tf, peaks),
-                algorithmic="%.4g FLOP per call (2.5 x the forward's: five products)" % bw_flops,
-                kernels="fa_bwd_dsum_kernel (also zeroes the dq workspace) + fa_bwd_kernel<128> "
-                        "+ fa_bwd_dq_kernel",
+                algorithmic="%.4g FLOP per call (2.5 x the forward's: five products; the "
+                            "kernel executes 3.5 x, its dQ CTAs recompute S and dP)" % bw_flops,
+                kernels="fa_bwd_dsum_kernel (D and -LSE*log2e per query tile) + "
+                        "fa_bwd_kernel<128> (dK/dV CTAs, then dQ CTAs)",
                 traffic_main_kernel=profiled_traffic("backward:" + ce.name),
-                gpu_launches=3 * K,
+                gpu_launches=2 * K,
                 note="dq, dk, dv from the forward's O and LSE; measured outside the step")
             del dq, dk, dv, ws, d_o
 
