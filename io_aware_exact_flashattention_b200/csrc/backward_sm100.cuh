@@ -65,8 +65,11 @@ struct BwdParams {
   __nv_bfloat16* dv;
   int B, Hq, Hkv, Sq, Skv, group, causal;
   int n_kv_tiles, n_q_tiles;
-  int heads_per_group;  // dK/dV CTA order: groups of this many (b, kv-head) pairs
-  int n_kv_ctas;        // grid: the first n_kv_ctas CTAs are dK/dV CTAs, the rest dQ CTAs
+  // CTA order (see bwd_tile)
+  int interleave;         // 1: per group of pairs, its dK/dV CTAs then its dQ CTAs
+  int heads_per_group;    // (batch, kv-head) pairs per group (dK/dV CTAs, or both roles)
+  int q_heads_per_group;  // (batch, query head) pairs per dQ group when not interleaved
+  int n_kv_ctas;          // dK/dV CTAs in the grid
   float scale, scale_log2;
   unsigned long long wait_limit_ns;
 };
@@ -183,23 +186,81 @@ __device__ __forceinline__ int bwd_first_q_tile(const BwdParams& p, int j) {
   return static_cast<int>(need / kBwdBN);
 }
 
+// The CTA's role and tile.  CTAs go out in groups of heads, heavy tiles first
+// within a group and role (under a causal mask key tile 0 sees every query
+// tile, and the last query tiles see the most keys), so that the data a group
+// streams stays in L2 while the launch order stays longest-first.  Two orders:
+//  - interleaved: per group of p.heads_per_group (batch, kv-head) pairs, its
+//    dK/dV CTAs, key tile by key tile, then the dQ CTAs of its query heads,
+//    query tile by query tile: a group's Q, dO, K and V are read from DRAM once
+//    for both roles.  Chosen when a group that hides its own longest CTA also
+//    leaves room in L2 for the next one.
+//  - by role: all dK/dV CTAs (groups of p.heads_per_group pairs), then all dQ
+//    CTAs (groups of p.q_heads_per_group query heads).  Chosen when the dK/dV
+//    CTAs are long (several query heads per kv head and long sequences): they
+//    then all start first, and only short dQ CTAs form the tail; the dQ CTAs
+//    read their inputs from DRAM a second time.
+struct BwdTile {
+  bool kv;    // dK/dV CTA (else dQ CTA)
+  int b, hg;  // batch; kv head (dK/dV) or query head (dQ)
+  int t;      // key tile (dK/dV) or query tile (dQ)
+};
+__device__ __forceinline__ BwdTile bwd_tile(const BwdParams& p) {
+  const int blk = static_cast<int>(blockIdx.x);
+  BwdTile tile;
+  if (p.interleave) {
+    const int units = p.B * p.Hkv;
+    const int full = p.heads_per_group * (p.n_kv_tiles + p.group * p.n_q_tiles);
+    const int grp = blk / full;
+    const int r = blk - grp * full;
+    const int in_group = min(p.heads_per_group, units - grp * p.heads_per_group);
+    const int kv_ctas = in_group * p.n_kv_tiles;
+    if (r < kv_ctas) {
+      tile.kv = true;
+      tile.t = r / in_group;
+      const int bg = grp * p.heads_per_group + r % in_group;
+      tile.b = bg / p.Hkv;
+      tile.hg = bg % p.Hkv;
+    } else {
+      // the group's query heads are consecutive: (b, g)'s are b*Hq + g*group + [0, group)
+      const int q_heads = in_group * p.group;
+      const int r2 = r - kv_ctas;
+      tile.kv = false;
+      tile.t = p.n_q_tiles - 1 - r2 / q_heads;
+      const int bh = grp * p.heads_per_group * p.group + r2 % q_heads;
+      tile.b = bh / p.Hq;
+      tile.hg = bh % p.Hq;
+    }
+  } else if (blk < p.n_kv_ctas) {
+    const int per_group = p.heads_per_group * p.n_kv_tiles;
+    const int grp = blk / per_group;
+    const int r = blk % per_group;
+    const int in_group = min(p.heads_per_group, p.B * p.Hkv - grp * p.heads_per_group);
+    tile.kv = true;
+    tile.t = r / in_group;
+    const int bg = grp * p.heads_per_group + r % in_group;
+    tile.b = bg / p.Hkv;
+    tile.hg = bg % p.Hkv;
+  } else {
+    const int cta = blk - p.n_kv_ctas;
+    const int per_group = p.q_heads_per_group * p.n_q_tiles;
+    const int grp = cta / per_group;
+    const int r = cta % per_group;
+    const int in_group = min(p.q_heads_per_group, p.B * p.Hq - grp * p.q_heads_per_group);
+    tile.kv = false;
+    tile.t = p.n_q_tiles - 1 - r / in_group;
+    const int bh = grp * p.q_heads_per_group + r % in_group;
+    tile.b = bh / p.Hq;
+    tile.hg = bh % p.Hq;
+  }
+  return tile;
+}
+
 __device__ __forceinline__ void bwd_kv_cta(const BwdParams& p, int& b, int& g, int& j) {
-  // CTAs go out in groups of p.heads_per_group (batch, key/value head)
-  // pairs; within a group key tile by key tile, heavy tiles first (under a
-  // causal mask key tile 0 sees every query tile), so the launch order stays
-  // longest-first and the tail is short.  The CTAs resident at a time then
-  // cover about two groups, whose Q and dO rows stay in L2 while all their
-  // key tiles stream them.
-  const int per_group = p.heads_per_group * p.n_kv_tiles;
-  const int cta = static_cast<int>(blockIdx.x);  // dK/dV CTAs come first in the grid
-  const int grp = cta / per_group;
-  const int r = cta % per_group;
-  const int units = p.B * p.Hkv;
-  const int in_group = min(p.heads_per_group, units - grp * p.heads_per_group);
-  j = r / in_group;
-  const int bg = grp * p.heads_per_group + r % in_group;
-  b = bg / p.Hkv;
-  g = bg % p.Hkv;
+  const BwdTile tile = bwd_tile(p);
+  b = tile.b;
+  g = tile.hg;
+  j = tile.t;
 }
 
 template <int D>
@@ -598,15 +659,11 @@ struct BwdQLayout {
 };
 static_assert(BwdQLayout<128>::kBytes <= 232448, "dQ shared memory over the limit");
 
-// The dQ CTAs go out heaviest first: under a causal mask (or a rectangular
-// one with more keys than queries) the last query tiles see the most keys.
 __device__ __forceinline__ void bwd_q_cta(const BwdParams& p, int& b, int& h, int& i) {
-  const int heads = p.B * p.Hq;
-  const int cta = static_cast<int>(blockIdx.x) - p.n_kv_ctas;  // dQ CTAs follow the dK/dV ones
-  i = p.n_q_tiles - 1 - cta / heads;
-  const int bh = cta % heads;
-  b = bh / p.Hq;
-  h = bh % p.Hq;
+  const BwdTile tile = bwd_tile(p);
+  b = tile.b;
+  h = tile.hg;
+  i = tile.t;
 }
 
 // Key tiles that query tile i sees: [0, n).
@@ -952,9 +1009,8 @@ __device__ __forceinline__ void bwd_dq_block(const CUtensorMap* tm_q, const CUte
   }
 }
 
-// The backward in one launch: CTAs [0, n_kv_ctas) take dK/dV key tiles
-// (heavy first), the rest dQ query tiles (heavy first).  Blocks start in
-// index order, so the dQ CTAs fill the SMs as the dK/dV tail drains.
+// The backward in one launch: each CTA takes a dK/dV key tile or a dQ query
+// tile, in the order bwd_tile gives.
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -962,7 +1018,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
               const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dk,
               const __grid_constant__ CUtensorMap tm_dv, const BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
-  if (static_cast<int>(blockIdx.x) < p.n_kv_ctas)
+  if (bwd_tile(p).kv)
     bwd_dkdv_block<D>(&tm_q, &tm_k, &tm_v, &tm_do, &tm_dk, &tm_dv, p, smem_raw);
   else
     bwd_dq_block<D>(&tm_q, &tm_k, &tm_v, &tm_do, &tm_dq, p, smem_raw);

@@ -22,8 +22,11 @@ namespace {
 
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s per mbarrier wait
 // Backward CTA order: groups of (batch, kv-head) pairs worth this many waves
-// of CTAs (see bwd_cta).
+// of CTAs (see fa::bwd_tile).
 constexpr int kBwdGroupWaves = 4;
+// The interleaved backward order is used while a group's K, V, Q and dO stay
+// within this many bytes (two groups in flight fit the 126 MB L2 with room).
+constexpr double kBwdInterleaveBytes = 48.0 * 1024 * 1024;
 constexpr int kMaxDevices = 64;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -421,6 +424,61 @@ cudaError_t prepare_backward(int dev) {
   return g_bwd_err[dev];
 }
 
+// CTA order of the backward launch (fa::bwd_tile).  Work of a CTA in tile
+// steps: a dK/dV CTA on key tile j visits group * (query tiles from the first
+// that sees j); a dQ CTA on query tile i visits the key tiles i sees.
+struct BwdOrder {
+  bool interleave;
+  int heads_per_group, q_heads_per_group;
+};
+BwdOrder backward_order(int B, int Hq, int Hkv, int Sq, int Skv, int d, bool causal,
+                        int n_kv_tiles, int n_q_tiles, int sms) {
+  const int group = Hq / Hkv;
+  const long long off = static_cast<long long>(Skv) - Sq;
+  long long pair_steps = 0, longest = 1;  // per (batch, kv-head) pair
+  for (int j = 0; j < n_kv_tiles; ++j) {
+    long long first = 0;
+    if (causal) {
+      const long long need = static_cast<long long>(j) * fa::kBwdBM - off;
+      first = need <= 0 ? 0 : need / fa::kBwdBN;
+    }
+    const long long steps = group * std::max(0LL, n_q_tiles - first);
+    pair_steps += steps;
+    longest = std::max(longest, steps);
+  }
+  for (int i = 0; i < n_q_tiles; ++i) {
+    long long keys = n_kv_tiles;
+    if (causal) {
+      const long long q_last = std::min(static_cast<long long>(i) * fa::kBwdBN + fa::kBwdBN - 1,
+                                        static_cast<long long>(Sq) - 1);
+      const long long k_last = q_last + off;
+      keys = k_last < 0 ? 0 : std::min<long long>(n_kv_tiles, k_last / fa::kBwdBM + 1);
+    }
+    pair_steps += group * keys;
+    longest = std::max(longest, keys);
+  }
+  const int pairs = B * Hkv;
+  const int ctas_per_pair = n_kv_tiles + group * n_q_tiles;
+  BwdOrder o;
+  // interleaved: about kBwdGroupWaves waves per group, and enough pairs that a
+  // group's span on the SMs is at least twice its longest CTA
+  long long g = std::max<long long>(1, kBwdGroupWaves * static_cast<long long>(sms) / ctas_per_pair);
+  if (pair_steps > 0)
+    g = std::max(g, (2 * longest * sms + pair_steps - 1) / pair_steps);
+  g = std::min<long long>(g, pairs);
+  // bytes a group streams: K, V of its pairs and Q, dO of their query heads
+  const double pair_bytes = 2.0 * 2.0 * d * (static_cast<double>(Skv) + group * static_cast<double>(Sq));
+  o.interleave = g * pair_bytes <= kBwdInterleaveBytes;
+  if (o.interleave) {
+    o.heads_per_group = static_cast<int>(g);
+    o.q_heads_per_group = 1;  // unused
+  } else {
+    o.heads_per_group = std::max(1, std::min(pairs, kBwdGroupWaves * sms / std::max(1, n_kv_tiles)));
+    o.q_heads_per_group = std::max(1, std::min(B * Hq, kBwdGroupWaves * sms / std::max(1, n_q_tiles)));
+  }
+  return o;
+}
+
 // D = rowsum(dO * O) into the workspace, then the dK/dV kernel (one CTA per
 // key tile) and the dQ kernel (one CTA per query tile); neither writes what
 // the other reads, and each gradient is written once.
@@ -470,14 +528,15 @@ fa_status launch_backward(const void* q, const void* k, const void* v, const voi
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_limit_ns = kWaitLimitNs;
-  // about kBwdGroupWaves waves of dK/dV CTAs per group (one CTA per SM)
-  p.heads_per_group =
-      n_kv_tiles > 0
-          ? std::max(1, std::min(B * Hkv, kBwdGroupWaves * g_bwd_sms[dev] / n_kv_tiles))
-          : 1;
-  p.n_kv_ctas = static_cast<int>(static_cast<long long>(B) * Hkv * n_kv_tiles);
+  const BwdOrder order = backward_order(B, Hq, Hkv, Sq, Skv, D, causal != 0, n_kv_tiles,
+                                        n_q_tiles, g_bwd_sms[dev]);
+  p.interleave = order.interleave ? 1 : 0;
+  p.heads_per_group = order.heads_per_group;
+  p.q_heads_per_group = order.q_heads_per_group;
+  const long long kv_ctas = static_cast<long long>(B) * Hkv * n_kv_tiles;
+  p.n_kv_ctas = static_cast<int>(kv_ctas);
   const long long q_ctas = static_cast<long long>(B) * Hq * n_q_tiles;
-  const unsigned grid = static_cast<unsigned>(p.n_kv_ctas + q_ctas);
+  const unsigned grid = static_cast<unsigned>(kv_ctas + q_ctas);
   fa::fa_bwd_kernel<D><<<grid, fa::kBwdThreads, fa::bwd_smem_bytes<D>(), stream>>>(
       tq, tk, tv, tdo, tdq, tdk, tdv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;

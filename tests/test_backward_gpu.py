@@ -145,3 +145,30 @@ def test_repeat_calls_bit_identical():
     torch.cuda.synchronize()
     for a, b in zip(first, second):
         assert torch.equal(a, b)
+
+
+def test_gqa_long_dkdv_ctas_order_by_role():
+    """GQA with four query heads per kv head at S = 4096: each dK/dV CTA is long,
+    so the launch takes the by-role CTA order (all dK/dV CTAs, then the dQ
+    ones).  The whole problem is launched; kv head 7 and its four query heads
+    are checked against the oracle."""
+    B, Hq, Hkv, S, d = 1, 32, 8, 4096, 128
+    q, k, v = prefill_inputs(B, Hq, Hkv, S, S, d, 95, 1.0)
+    d_o = grad_output((B, Hq, S, d), 95)
+    scale = 1.0 / math.sqrt(d)
+    qc, kc, vc, doc = (t.cuda() for t in (q, k, v, d_o))
+    o = torch.empty_like(qc)
+    lse = torch.empty((B, Hq, S), device="cuda", dtype=torch.float32)
+    fa.fa_fwd(qc, kc, vc, o, lse, True, scale)
+    dq, dk, dv = fa.attention_backward(qc, kc, vc, o, lse, doc, True, scale)
+    torch.cuda.synchronize()
+    hq, hk = slice(28, 32), slice(7, 8)
+    ref = oracle.attn_bwd(q[:, hq], k[:, hk], v[:, hk], d_o[:, hq], True, scale)
+    errs = {}
+    for name, got, want in (("dq", dq[:, hq], ref[0]), ("dk", dk[:, hk], ref[1]),
+                            ("dv", dv[:, hk], ref[2])):
+        g = got.float().cpu().numpy().astype(np.float64)
+        assert np.isfinite(g).all(), name + ": non-finite"
+        errs[name] = (float(np.abs(g - want).max()) / max(float(np.abs(want).max()), 1e-30),
+                      float(np.linalg.norm(g - want)) / max(float(np.linalg.norm(want)), 1e-30))
+    check(errs)
