@@ -50,7 +50,8 @@ CSRC = "io_aware_exact_flashattention_b200/csrc/"
 SOURCES = {
     "prefill": [CSRC + "prefill_sm100.cuh", CSRC + "sm100.cuh"],
     "decode": [CSRC + "decode_sm100.cuh", CSRC + "sm100.cuh"],
-    "backward": [CSRC + "backward_sm100.cuh", CSRC + "sm100.cuh"],
+    # the host file chooses the backward's CTA order, which sets its traffic
+    "backward": [CSRC + "backward_sm100.cuh", CSRC + "sm100.cuh", CSRC + "fa_api.cu"],
     "ffn": [CSRC + "ffn_sm100.cuh", CSRC + "sm100.cuh"],
 }
 
