@@ -483,14 +483,18 @@ __device__ __forceinline__ void bwd_kv_elementwise(const BwdParams& p, uint32_t 
         uint32_t dp[32];
         tmem_ld32(t_dp + hf * kQH + hq * 32, dp);
         uint32_t dsk[16];
+        const float2 m1 = make_float2(-1.f, -1.f);
 #pragma unroll
         for (int e2 = 0; e2 < 16; ++e2) {
           const int cl = hq * 32 + 2 * e2;  // local query index in the half
-          const __nv_bfloat162 pb = *reinterpret_cast<const __nv_bfloat162*>(&pk[cl >> 1]);
-          const int c = hf * kQH + cl;
-          const float d0 = __bfloat162float(pb.x) * (__uint_as_float(dp[2 * e2]) - d_s[c]);
-          const float d1 = __bfloat162float(pb.y) * (__uint_as_float(dp[2 * e2 + 1]) - d_s[c + 1]);
-          dsk[e2] = pack_bf16x2(d0, d1);
+          // the pair of bf16 weights as fp32, and dP - D rounded once, as pairs
+          const uint32_t pw = pk[cl >> 1];
+          const float2 pf = make_float2(__uint_as_float(pw << 16), __uint_as_float(pw & 0xffff0000u));
+          const float2 dd = *reinterpret_cast<const float2*>(d_s + hf * kQH + cl);
+          const float2 t2 = ffma2(dd, m1, make_float2(__uint_as_float(dp[2 * e2]),
+                                                      __uint_as_float(dp[2 * e2 + 1])));
+          const float2 ds2 = fmul2(pf, t2);
+          dsk[e2] = pack_bf16x2(ds2.x, ds2.y);
         }
         // queries hf*64 + hq*32 .. +31: box hf, 16-byte chunks hq*4 .. +3 of row t
 #pragma unroll
@@ -886,11 +890,14 @@ __device__ __forceinline__ void bwd_q_elementwise(const BwdParams& p, uint32_t s
       uint32_t dp[32];
       tmem_ld32(t_dp + hf * kKH + hk * 32, dp);
       uint32_t dsk[16];
+      const float2 nd2 = make_float2(-dval, -dval);
 #pragma unroll
       for (int e2 = 0; e2 < 16; ++e2) {
         const int c = hk * 32 + 2 * e2;
-        dsk[e2] = pack_bf16x2(pr[c] * (__uint_as_float(dp[2 * e2]) - dval),
-                              pr[c + 1] * (__uint_as_float(dp[2 * e2 + 1]) - dval));
+        const float2 ds2 = fmul2(make_float2(pr[c], pr[c + 1]),
+                                 fadd2(make_float2(__uint_as_float(dp[2 * e2]),
+                                                   __uint_as_float(dp[2 * e2 + 1])), nd2));
+        dsk[e2] = pack_bf16x2(ds2.x, ds2.y);
       }
       tmem_st16(t_s + hf * kKH + hk * 16, dsk);
     }
