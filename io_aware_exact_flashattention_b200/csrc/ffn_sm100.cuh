@@ -20,9 +20,10 @@
 // K chunk k*64 of a token is column (k*64) % d of head (k*64) / d, one TMA box
 // of the [B*Hq, S, d] view, so the concatenation over heads is never formed.
 //
-// Roles (192 threads): warps 0-3 epilogue (thread = row = TMEM lane), warp 4
-// TMA producer (4-stage ring of A and B boxes), warp 5 MMA issuer and TMEM
-// owner.  The kernel is persistent (one CTA per SM over the launch's output
+// Roles (320 threads): warps 0-7 epilogue (thread = row = TMEM lane; warps w
+// and w + 4 share a lane quarter and take one half of the tile's columns
+// each), warp 8 TMA producer (4-stage ring of A and B boxes), warp 9 MMA
+// issuer and TMEM owner.  The kernel is persistent (one CTA per SM over the launch's output
 // tiles) with two accumulators in tensor memory, so a tile's epilogue
 // overlaps the next tile's products.  Every mbarrier wait is bounded (see
 // mbar_wait).
@@ -37,7 +38,10 @@ constexpr int kFfnBM = 128;       // tokens per tile (TMEM lanes)
 constexpr int kFfnBN = 256;       // output columns per tile (fp32 TMEM columns)
 constexpr int kFfnBK = 64;        // K per ring stage: one 128-byte swizzle box of bf16
 constexpr int kFfnStages = 4;
-constexpr int kFfnThreads = 192;
+constexpr int kFfnEpiWarps = 8;   // two per TMEM lane quarter, one per column half
+constexpr int kFfnThreads = 32 * kFfnEpiWarps + 64;
+constexpr int kFfnProducerWarp = kFfnEpiWarps;
+constexpr int kFfnMmaWarp = kFfnEpiWarps + 1;
 
 struct FfnLayout {
   static constexpr int kABytes = kFfnBM * kFfnBK * 2;     // 16 KB
@@ -120,13 +124,13 @@ fa_ffn_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bars + 8 * (L::kBarAccFull + a), 1);
-      mbar_init(bars + 8 * (L::kBarAccEmpty + a), 4);  // one arrival per epilogue warp
+      mbar_init(bars + 8 * (L::kBarAccEmpty + a), kFfnEpiWarps);  // one arrival per epilogue warp
     }
     mbar_init(bars + 8 * L::kBarDone, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kFfnMmaWarp) {
     tmem_alloc(sbase + L::kTmemSlotOff, 2 * kFfnBN);
     tmem_relinquish();
   }
@@ -135,7 +139,7 @@ fa_ffn_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlotOff);
 
-  if (warp == 4) {
+  if (warp == kFfnProducerWarp) {
     if (lane == 0) {
       // producer: A and B boxes of every K step of every tile into the ring
       tma_prefetch_desc(&tm_a);
@@ -167,7 +171,7 @@ fa_ffn_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
       for (uint32_t k = (issued > S ? issued - S : 0u); k < issued; ++k)
         mbar_wait(bars + 8 * (L::kBarFull + k % S), (k / S) & 1u, nullptr, p.wait_limit_ns);
     }
-  } else if (warp == 5) {
+  } else if (warp == kFfnMmaWarp) {
     if (lane == 0) {
       // MMA issuer: acc[i & 1] [128 x 256] (+)= A_k B_k^T, four K = 16 steps per stage
       constexpr uint32_t kId = idesc_bf16_f32(kFfnBM, kFfnBN, false);
@@ -206,9 +210,12 @@ fa_ffn_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
       mbar_wait(bars + 8 * L::kBarDone, 0u, nullptr, p.wait_limit_ns);
     }
   } else {
-    // epilogue: row r of the tile, 32 columns per TMEM load
-    const int r = threadIdx.x;  // warps 0-3: TMEM lanes 0-127
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    // epilogue: row r of the tile (the warp's TMEM lane quarter), the warp's
+    // half of the columns, 32 columns per TMEM load
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    constexpr int kHalfCols = kFfnBN / 2;
     int i = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
       const FfnTile f = ffn_tile(p, t);
@@ -221,11 +228,12 @@ fa_ffn_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
       const long long row = p.c_tokens
                                 ? static_cast<long long>(f.b) * p.S_out + p.tok0 + f.t0 + r
                                 : static_cast<long long>(f.local_row0) + r;
-      uint4* dst = reinterpret_cast<uint4*>(p.c + row * p.N + f.n0);
+      uint4* dst = reinterpret_cast<uint4*>(p.c + row * p.N + f.n0 + half * kHalfCols);
 #pragma unroll 1
-      for (int c = 0; c < kFfnBN / 32; ++c) {
+      for (int c = 0; c < kHalfCols / 32; ++c) {
         uint32_t v[32];
-        tmem_ld32(tmem + lane_off + acc * kFfnBN + static_cast<uint32_t>(c * 32), v);
+        tmem_ld32(tmem + lane_off + acc * kFfnBN + static_cast<uint32_t>(half * kHalfCols + c * 32),
+                  v);
         uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -251,7 +259,7 @@ fa_ffn_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kFfnMmaWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 2 * kFfnBN);
