@@ -383,6 +383,20 @@ fa_status fa_get_device_status(void);
 fa_status fa_debug_timeout_probe(unsigned int limit_us, fa_stream_t stream);
 
 /*
+ * Test hook for the backward's CTA order (host only; no CUDA call).  For the
+ * backward problem the sizes describe and a device of `sms` SMs, writes the
+ * number of CTAs fa_bwd launches to *n_ctas, whether it runs them
+ * interleaved by head group (1) or by role (0) to *interleave, and, when
+ * tiles is not null, the unit of every CTA in launch order: tiles[4*c ..
+ * 4*c+3] = {1 for a dK/dV CTA or 0 for a dQ CTA, batch, kv head (dK/dV) or
+ * query head (dQ), key tile (dK/dV) or query tile (dQ)}.  capacity is the
+ * number of 4-int entries tiles holds (FA_ERR_INVALID_ARG if fewer than
+ * *n_ctas).  Sizes as for fa_bwd with Sq >= 1; d in {64, 128}.
+ */
+fa_status fa_debug_bwd_tiles(int B, int Hq, int Hkv, int Sq, int Skv, int d, int causal, int sms,
+                             int *tiles, long long capacity, long long *n_ctas, int *interleave);
+
+/*
  * Test hook for the polynomial 2^x that the prefill kernel evaluates on the
  * FMA pipe for part of its softmax (the rest uses the hardware exp2):
  * y[i] = 2^n * p(x[i] - n), n = round(x[i]), p the degree-3 minimax fit of

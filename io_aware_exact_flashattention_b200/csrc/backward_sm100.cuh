@@ -205,15 +205,17 @@ struct BwdTile {
   int b, hg;  // batch; kv head (dK/dV) or query head (dQ)
   int t;      // key tile (dK/dV) or query tile (dQ)
 };
-__device__ __forceinline__ BwdTile bwd_tile(const BwdParams& p) {
-  const int blk = static_cast<int>(blockIdx.x);
+__host__ __device__ inline int bwd_imin(int a, int b) { return a < b ? a : b; }
+
+// The tile of CTA blk (host and device: the host checks the mapping).
+__host__ __device__ inline BwdTile bwd_tile_of(const BwdParams& p, int blk) {
   BwdTile tile;
   if (p.interleave) {
     const int units = p.B * p.Hkv;
     const int full = p.heads_per_group * (p.n_kv_tiles + p.group * p.n_q_tiles);
     const int grp = blk / full;
     const int r = blk - grp * full;
-    const int in_group = min(p.heads_per_group, units - grp * p.heads_per_group);
+    const int in_group = bwd_imin(p.heads_per_group, units - grp * p.heads_per_group);
     const int kv_ctas = in_group * p.n_kv_tiles;
     if (r < kv_ctas) {
       tile.kv = true;
@@ -235,7 +237,7 @@ __device__ __forceinline__ BwdTile bwd_tile(const BwdParams& p) {
     const int per_group = p.heads_per_group * p.n_kv_tiles;
     const int grp = blk / per_group;
     const int r = blk % per_group;
-    const int in_group = min(p.heads_per_group, p.B * p.Hkv - grp * p.heads_per_group);
+    const int in_group = bwd_imin(p.heads_per_group, p.B * p.Hkv - grp * p.heads_per_group);
     tile.kv = true;
     tile.t = r / in_group;
     const int bg = grp * p.heads_per_group + r % in_group;
@@ -246,7 +248,7 @@ __device__ __forceinline__ BwdTile bwd_tile(const BwdParams& p) {
     const int per_group = p.q_heads_per_group * p.n_q_tiles;
     const int grp = cta / per_group;
     const int r = cta % per_group;
-    const int in_group = min(p.q_heads_per_group, p.B * p.Hq - grp * p.q_heads_per_group);
+    const int in_group = bwd_imin(p.q_heads_per_group, p.B * p.Hq - grp * p.q_heads_per_group);
     tile.kv = false;
     tile.t = p.n_q_tiles - 1 - r / in_group;
     const int bh = grp * p.q_heads_per_group + r % in_group;
@@ -254,6 +256,9 @@ __device__ __forceinline__ BwdTile bwd_tile(const BwdParams& p) {
     tile.hg = bh % p.Hq;
   }
   return tile;
+}
+__device__ __forceinline__ BwdTile bwd_tile(const BwdParams& p) {
+  return bwd_tile_of(p, static_cast<int>(blockIdx.x));
 }
 
 __device__ __forceinline__ void bwd_kv_cta(const BwdParams& p, int& b, int& g, int& j) {

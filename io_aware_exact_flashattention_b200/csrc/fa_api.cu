@@ -479,6 +479,20 @@ BwdOrder backward_order(int B, int Hq, int Hkv, int Sq, int Skv, int d, bool cau
   return o;
 }
 
+// Sets the order fields of p (whose sizes are set) and returns the grid: the
+// dK/dV CTAs (one per batch, kv head and key tile) plus the dQ CTAs (one per
+// batch, query head and query tile).
+long long fill_backward_order(fa::BwdParams& p, int d, int sms) {
+  const BwdOrder order = backward_order(p.B, p.Hq, p.Hkv, p.Sq, p.Skv, d, p.causal != 0,
+                                        p.n_kv_tiles, p.n_q_tiles, sms);
+  p.interleave = order.interleave ? 1 : 0;
+  p.heads_per_group = order.heads_per_group;
+  p.q_heads_per_group = order.q_heads_per_group;
+  const long long kv_ctas = static_cast<long long>(p.B) * p.Hkv * p.n_kv_tiles;
+  p.n_kv_ctas = static_cast<int>(kv_ctas);
+  return kv_ctas + static_cast<long long>(p.B) * p.Hq * p.n_q_tiles;
+}
+
 // D = rowsum(dO * O) into the workspace, then the dK/dV kernel (one CTA per
 // key tile) and the dQ kernel (one CTA per query tile); neither writes what
 // the other reads, and each gradient is written once.
@@ -528,15 +542,7 @@ fa_status launch_backward(const void* q, const void* k, const void* v, const voi
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_limit_ns = kWaitLimitNs;
-  const BwdOrder order = backward_order(B, Hq, Hkv, Sq, Skv, D, causal != 0, n_kv_tiles,
-                                        n_q_tiles, g_bwd_sms[dev]);
-  p.interleave = order.interleave ? 1 : 0;
-  p.heads_per_group = order.heads_per_group;
-  p.q_heads_per_group = order.q_heads_per_group;
-  const long long kv_ctas = static_cast<long long>(B) * Hkv * n_kv_tiles;
-  p.n_kv_ctas = static_cast<int>(kv_ctas);
-  const long long q_ctas = static_cast<long long>(B) * Hq * n_q_tiles;
-  const unsigned grid = static_cast<unsigned>(kv_ctas + q_ctas);
+  const unsigned grid = static_cast<unsigned>(fill_backward_order(p, D, g_bwd_sms[dev]));
   fa::fa_bwd_kernel<D><<<grid, fa::kBwdThreads, fa::bwd_smem_bytes<D>(), stream>>>(
       tq, tk, tv, tdo, tdq, tdk, tdv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -1014,6 +1020,37 @@ fa_status fa_debug_exp2_poly(const float* x, float* y, int n, fa_stream_t stream
   const int pairs = (n + 1) / 2;
   exp2_poly_kernel<<<(pairs + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_debug_bwd_tiles(int B, int Hq, int Hkv, int Sq, int Skv, int d, int causal, int sms,
+                             int* tiles, long long capacity, long long* n_ctas, int* interleave) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || Skv < 0 || sms < 1 || Hq % Hkv != 0 ||
+      n_ctas == nullptr || interleave == nullptr || capacity < 0)
+    return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  fa::BwdParams p{};
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Sq = Sq;
+  p.Skv = Skv;
+  p.group = Hq / Hkv;
+  p.causal = causal ? 1 : 0;
+  p.n_kv_tiles = (Skv + fa::kBwdBM - 1) / fa::kBwdBM;
+  p.n_q_tiles = (Sq + fa::kBwdBN - 1) / fa::kBwdBN;
+  const long long grid = fill_backward_order(p, d, sms);
+  *n_ctas = grid;
+  *interleave = p.interleave;
+  if (tiles == nullptr) return FA_OK;
+  if (capacity < grid) return FA_ERR_INVALID_ARG;
+  for (long long blk = 0; blk < grid; ++blk) {
+    const fa::BwdTile t = fa::bwd_tile_of(p, static_cast<int>(blk));
+    tiles[4 * blk + 0] = t.kv ? 1 : 0;
+    tiles[4 * blk + 1] = t.b;
+    tiles[4 * blk + 2] = t.hg;
+    tiles[4 * blk + 3] = t.t;
+  }
+  return FA_OK;
 }
 
 fa_status fa_debug_timeout_probe(unsigned int limit_us, fa_stream_t stream) {

@@ -48,6 +48,7 @@ SIGNATURES = {
     "fa_debug_timeout_probe": (_I, [ctypes.c_uint, _VP]),
     "fa_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP]),
     "fa_debug_exp2_poly": (_I, [_VP, _VP, _I, _VP]),
+    "fa_debug_bwd_tiles": (_I, [_I] * 8 + [_VP, ctypes.c_longlong, _VP, _VP]),
     "fa_shard_units": (_I, [_I, _I, _I, _I, ctypes.POINTER(ctypes.c_int),
                             ctypes.POINTER(ctypes.c_int)]),
     "fa_shard_sequences": (_I, [_VP, _I, _I, _VP]),
