@@ -75,45 +75,72 @@ struct BwdParams {
 };
 
 // ---------------------------------------------------------------------------
-// Per query row (one warp per row, rows padded to whole 128-row tiles):
-// D = rowsum(dO * O) and -LSE*log2(e), packed per tile as the backward
-// kernels read them (a tile's 1 KB is one bulk copy).  Rows past Sq get
-// -LSE*log2(e) = -inf and D = 0, so their weights and dS are exactly 0.
-// ---------------------------------------------------------------------------
+// Per query row (rows padded to whole 128-row tiles): D = rowsum(dO * O) and
+// -LSE*log2(e), packed per tile as the backward kernels read them (a tile's
+// 1 KB is one bulk copy).  Rows past Sq get -LSE*log2(e) = -inf and D = 0, so
+// their weights and dS are exactly 0.  The kernel only streams O and dO, so
+// it is shaped for bandwidth: a lane loads 16 bytes of each, a row is D/8
+// lanes, a warp covers kDsumRowsPerWarp rows with all its loads issued before
+// the first use.
+constexpr int kDsumRowsPerWarp = 8;
+constexpr int kDsumRowsPerBlock = 8 * kDsumRowsPerWarp;  // 256 threads
+
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_dsum_kernel(const __nv_bfloat16* __restrict__ o,
                                                           const __nv_bfloat16* __restrict__ d_o,
                                                           const float* __restrict__ lse,
                                                           float* __restrict__ ld, int Sq,
                                                           int n_q_tiles, long long rows_padded) {
-  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= rows_padded) return;
+  constexpr int kLanesPerRow = D / 8;                     // 16-byte chunks per row
+  constexpr int kRowsPerLoad = 32 / kLanesPerRow;         // rows one warp load covers
+  constexpr int kLoads = kDsumRowsPerWarp / kRowsPerLoad;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane / kLanesPerRow, chunk = lane % kLanesPerRow;
+  const long long row0 = static_cast<long long>(blockIdx.x) * kDsumRowsPerBlock +
+                         warp * kDsumRowsPerWarp;
+  if (row0 >= rows_padded) return;  // (uniform per warp)
+  // a warp's rows lie in one head's padded rows (128 is a multiple of them)
   const long long per_head = static_cast<long long>(n_q_tiles) * 128;
-  const long long bh = row / per_head;
-  const int qq = static_cast<int>(row - bh * per_head);
-  float* dst = ld + (bh * n_q_tiles + qq / 128) * 256 + (qq & 127);
-  if (qq >= Sq) {
-    if (lane == 0) {
-      dst[0] = -INFINITY;
-      dst[128] = 0.f;
+  const long long bh = row0 / per_head;
+  const int q0 = static_cast<int>(row0 - bh * per_head);
+  const __nv_bfloat16* o_h = o + bh * Sq * static_cast<long long>(D);
+  const __nv_bfloat16* do_h = d_o + bh * Sq * static_cast<long long>(D);
+  uint4 xo[kLoads], xd[kLoads];
+#pragma unroll
+  for (int l = 0; l < kLoads; ++l) {
+    const int qq = q0 + l * kRowsPerLoad + sub;
+    xo[l] = make_uint4(0u, 0u, 0u, 0u);
+    xd[l] = make_uint4(0u, 0u, 0u, 0u);
+    if (qq < Sq) {
+      const long long src = static_cast<long long>(qq) * D + chunk * 8;
+      xo[l] = __ldg(reinterpret_cast<const uint4*>(o_h + src));
+      xd[l] = __ldg(reinterpret_cast<const uint4*>(do_h + src));
     }
-    return;
   }
-  const long long src = bh * Sq + qq;
-  float acc = 0.f;
+  float* dst_h = ld + bh * n_q_tiles * 256;
 #pragma unroll
-  for (int c = lane * 2; c < D; c += 64) {
-    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(o + src * D + c);
-    const __nv_bfloat162 y = *reinterpret_cast<const __nv_bfloat162*>(d_o + src * D + c);
-    acc = fmaf(__bfloat162float(x.x), __bfloat162float(y.x), acc);
-    acc = fmaf(__bfloat162float(x.y), __bfloat162float(y.y), acc);
-  }
+  for (int l = 0; l < kLoads; ++l) {
+    const uint32_t* a = reinterpret_cast<const uint32_t*>(&xo[l]);
+    const uint32_t* c = reinterpret_cast<const uint32_t*>(&xd[l]);
+    float acc = 0.f;
 #pragma unroll
-  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-  if (lane == 0) {
-    dst[0] = lse[src] * -1.4426950408889634f;
-    dst[128] = acc;
+    for (int e = 0; e < 4; ++e) {
+      acc = fmaf(__uint_as_float(a[e] << 16), __uint_as_float(c[e] << 16), acc);
+      acc = fmaf(__uint_as_float(a[e] & 0xffff0000u), __uint_as_float(c[e] & 0xffff0000u), acc);
+    }
+#pragma unroll
+    for (int s = kLanesPerRow / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+    const int qq = q0 + l * kRowsPerLoad + sub;
+    if (chunk == 0) {
+      float* dst = dst_h + (qq / 128) * 256 + (qq & 127);
+      if (qq >= Sq) {
+        dst[0] = -INFINITY;
+        dst[128] = 0.f;
+      } else {
+        dst[0] = lse[bh * Sq + qq] * -1.4426950408889634f;
+        dst[128] = acc;
+      }
+    }
   }
 }
 

@@ -509,7 +509,8 @@ fa_status launch_backward(const void* q, const void* k, const void* v, const voi
     k = v = q;
     dk = dv = dq;
   }
-  fa::fa_bwd_dsum_kernel<D><<<static_cast<unsigned>(rows_padded / 8), 256, 0, stream>>>(
+  fa::fa_bwd_dsum_kernel<D><<<static_cast<unsigned>(rows_padded / fa::kDsumRowsPerBlock), 256, 0,
+                               stream>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o), lse, ld, Sq,
       n_q_tiles, rows_padded);
   const int n_kv_tiles = (Skv + fa::kBwdBM - 1) / fa::kBwdBM;
