@@ -140,11 +140,16 @@ fa_status fa_fwd_fp8(const void *q, const void *k, const void *v, const float *d
  *   causal, scale: as passed to fa_fwd.
  *
  * dq, dk, dv are written once each (dk = dv = 0 for keys no query sees, dq = 0
- * for queries that see no key): dk, dv by a kernel with one CTA per key tile,
- * dq by one with one CTA per query tile, each accumulating in tensor memory,
- * so the result does not depend on scheduling.  P and dS enter the
- * tensor-core products as bf16; accumulation is fp32.
+ * for queries that see no key) by one kernel with two kinds of CTA: one per
+ * key tile for dk, dv and one per query tile for dq, each accumulating in
+ * tensor memory, so the result does not depend on scheduling.  A first,
+ * bandwidth-bound kernel writes the workspace; the second is launched with
+ * programmatic stream serialisation, so its setup and its loads of q, k, v,
+ * d_o overlap the first's end, and it reads the workspace only after the
+ * first has completed.  P and dS enter the tensor-core products as bf16;
+ * accumulation is fp32.
  * Supported: d in {64, 128}; Hq % Hkv == 0.  All pointers 16-byte aligned;
+ * dq, dk, dv and workspace must not overlap the inputs or one another.
  * k, v, dk, dv may be null when Skv = 0, and q, o, lse, d_o, dq, workspace
  * when Sq = 0.  Errors as for fa_fwd.
  */

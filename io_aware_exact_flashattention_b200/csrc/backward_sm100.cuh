@@ -94,6 +94,9 @@ __global__ void __launch_bounds__(256) fa_bwd_dsum_kernel(const __nv_bfloat16* _
   constexpr int kLanesPerRow = D / 8;                     // 16-byte chunks per row
   constexpr int kRowsPerLoad = 32 / kLanesPerRow;         // rows one warp load covers
   constexpr int kLoads = kDsumRowsPerWarp / kRowsPerLoad;
+  // the backward kernel, launched next, may start its setup and loads now;
+  // it waits for this grid before reading its output
+  grid_dep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sub = lane / kLanesPerRow, chunk = lane % kLanesPerRow;
   const long long row0 = static_cast<long long>(blockIdx.x) * kDsumRowsPerBlock +
@@ -332,6 +335,7 @@ __device__ __forceinline__ void bwd_kv_producer(const CUtensorMap* tq, const CUt
         tma_load_3d(qa + kb * L::kBoxBytes, tq, full, kb * 64, i * kBwdBN, plane);
         tma_load_3d(qa + L::kTileBytes + kb * L::kBoxBytes, tdo, full, kb * 64, i * kBwdBN, plane);
       }
+      grid_dep_wait();  // the D kernel's per-tile values are complete (free after the first)
       bulk_load(sbase + L::kLdOff + s * L::kLdBytes,
                 p.ld + (static_cast<size_t>(plane) * p.n_q_tiles + i) * 256, L::kLdBytes, full);
     }
@@ -870,6 +874,7 @@ __device__ __forceinline__ void bwd_q_elementwise(const BwdParams& p, uint32_t s
   const int nk = bwd_q_kv_tiles(p, i);
   const int q = i * kBwdBN + row;
   // -LSE in log2 units (rows past Sq: -inf, weights exactly 0) and D
+  grid_dep_wait();  // the D kernel's per-tile values are complete
   const float* ldt = p.ld + (static_cast<size_t>(b * p.Hq + h) * p.n_q_tiles + i) * 256;
   const float nlse = ldt[row];
   const float dval = ldt[128 + row];

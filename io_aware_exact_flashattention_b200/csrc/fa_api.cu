@@ -544,8 +544,21 @@ fa_status launch_backward(const void* q, const void* k, const void* v, const voi
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_limit_ns = kWaitLimitNs;
   const unsigned grid = static_cast<unsigned>(fill_backward_order(p, D, g_bwd_sms[dev]));
-  fa::fa_bwd_kernel<D><<<grid, fa::kBwdThreads, fa::bwd_smem_bytes<D>(), stream>>>(
-      tq, tk, tv, tdo, tdq, tdk, tdv, p);
+  // programmatic dependent launch: the CTAs' setup and their K, V, Q and dO
+  // loads overlap the D kernel's tail; the reads of its output wait for it
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(fa::kBwdThreads);
+  cfg.dynamicSmemBytes = fa::bwd_smem_bytes<D>();
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, fa::fa_bwd_kernel<D>, tq, tk, tv, tdo, tdq, tdk, tdv, p) !=
+      cudaSuccess)
+    return FA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
