@@ -413,18 +413,6 @@ __device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
-// Programmatic dependent launch: the grid launched after this one with
-// programmatic stream serialisation may start once every CTA of this grid
-// has executed launch_dependents (or exited); it must wait (grid_dep_wait)
-// before reading anything this grid writes.  Both are no-ops for a grid
-// launched without that attribute.
-__device__ __forceinline__ void grid_dep_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void grid_dep_wait() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-
 // Wait until every committed bulk operation of this thread has completed.
 __device__ __forceinline__ void bulk_wait_group0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
