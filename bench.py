@@ -51,8 +51,9 @@ SOURCES = {
     "prefill": [CSRC + "prefill_sm100.cuh", CSRC + "sm100.cuh"],
     "decode": [CSRC + "decode_sm100.cuh", CSRC + "sm100.cuh"],
     # the host file chooses the backward's CTA order, which sets its traffic
-    "backward": [CSRC + "backward_sm100.cuh", CSRC + "sm100.cuh", CSRC + "fa_api.cu"],
-    "ffn": [CSRC + "ffn_sm100.cuh", CSRC + "sm100.cuh"],
+    "backward": [CSRC + "backward_sm100.cuh", CSRC + "sm100.cuh", CSRC + "launch_dep.cuh",
+                 CSRC + "fa_api.cu"],
+    "ffn": [CSRC + "ffn_sm100.cuh", CSRC + "sm100.cuh", CSRC + "launch_dep.cuh"],
 }
 
 

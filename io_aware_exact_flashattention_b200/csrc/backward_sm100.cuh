@@ -44,6 +44,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include "sm100.cuh"
+#include "launch_dep.cuh"
 
 namespace fa {
 
@@ -82,18 +83,6 @@ struct BwdParams {
 // it is shaped for bandwidth: a lane loads 16 bytes of each, a row is D/8
 // lanes, a warp covers kDsumRowsPerWarp rows with all its loads issued before
 // the first use.
-// Programmatic dependent launch: the grid launched after this one with
-// programmatic stream serialisation may start once every CTA of this grid
-// has executed launch_dependents (or exited); it must wait (grid_dep_wait)
-// before reading anything this grid writes.  Both are no-ops for a grid
-// launched without that attribute.
-__device__ __forceinline__ void grid_dep_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void grid_dep_wait() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-
 constexpr int kDsumRowsPerWarp = 8;
 constexpr int kDsumRowsPerBlock = 8 * kDsumRowsPerWarp;  // 256 threads
 

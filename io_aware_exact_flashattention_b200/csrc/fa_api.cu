@@ -586,8 +586,19 @@ void launch_ffn(const CUtensorMap& tm_a, const CUtensorMap& tm_b, fa::FfnParams 
   p.n_row_tiles = row_tiles;
   const int tiles = row_tiles * (p.N / fa::kFfnBN);
   const int grid = std::max(1, std::min(tiles, g_ffn_sms[dev]));
-  fa::fa_ffn_gemm_kernel<<<static_cast<unsigned>(grid), fa::kFfnThreads, fa::FfnLayout::kBytes,
-                           s>>>(tm_a, tm_b, p);
+  // programmatic dependent launch: the CTAs' setup overlaps the previous
+  // kernel's end; the kernel waits for it before its first load
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(fa::kFfnThreads);
+  cfg.dynamicSmemBytes = fa::FfnLayout::kBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  (void)cudaLaunchKernelEx(&cfg, fa::fa_ffn_gemm_kernel, tm_a, tm_b, p);
 }
 
 extern "C" {

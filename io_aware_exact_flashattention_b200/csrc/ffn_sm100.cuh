@@ -31,6 +31,7 @@
 
 #include <cuda.h>
 #include "sm100.cuh"
+#include "launch_dep.cuh"
 
 namespace fa {
 
@@ -139,11 +140,18 @@ fa_ffn_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlotOff);
 
+  // The next launch of the call (the other product, or the next chunk) may
+  // start its setup now; it waits for this grid before its first load.
+  grid_dep_launch_dependents();
   if (warp == kFfnProducerWarp) {
     if (lane == 0) {
       // producer: A and B boxes of every K step of every tile into the ring
       tma_prefetch_desc(&tm_a);
       tma_prefetch_desc(&tm_b);
+      // The previous kernel of the call (the attention, or the other
+      // product, which reads this launch's output buffer) has completed
+      // before any load; every store of this grid follows these loads.
+      grid_dep_wait();
       uint32_t issued = 0;
       bool stop = false;
       for (int t = blockIdx.x; t < n_tiles && !stop; t += gridDim.x) {
