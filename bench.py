@@ -49,7 +49,7 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 CSRC = "io_aware_exact_flashattention_b200/csrc/"
 SOURCES = {
     "prefill": [CSRC + "prefill_sm100.cuh", CSRC + "sm100.cuh"],
-    "decode": [CSRC + "decode_sm100.cuh", CSRC + "sm100.cuh"],
+    "decode": [CSRC + "decode_sm100.cuh", CSRC + "sm100.cuh", CSRC + "launch_dep.cuh"],
     # the host file chooses the backward's CTA order, which sets its traffic
     "backward": [CSRC + "backward_sm100.cuh", CSRC + "sm100.cuh", CSRC + "launch_dep.cuh",
                  CSRC + "fa_api.cu"],

@@ -42,6 +42,7 @@
 
 #include <cuda.h>
 #include "sm100.cuh"
+#include "launch_dep.cuh"
 
 namespace fa {
 
@@ -576,6 +577,9 @@ fa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v32,
                        const __grid_constant__ CUtensorMap tm_q, const DecodeParams p) {
   using L = DecodeLayout<D>;
+  // the combine, launched next as a dependent, may be scheduled now; it
+  // waits for this grid before reading the partials
+  grid_dep_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
@@ -646,6 +650,9 @@ fa_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ ls
                   __nv_bfloat16* __restrict__ o, float* __restrict__ lse, int rows, int n_splits) {
   constexpr float kLog2e = 1.44269504088896340736f;
   constexpr int EPL = D / 32;  // elements per lane: 4 (D=128) or 2 (D=64)
+  // launched as a programmatic dependent: the kernel before it on the stream
+  // (normally the split kernel writing the partials) has completed after this
+  grid_dep_wait();
   const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;

@@ -957,14 +957,26 @@ fa_status fa_combine(const float* o_partial, const float* lse_partial, void* o, 
   if (rows > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   const unsigned blocks = static_cast<unsigned>((rows + 3) / 4);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64)
-    fa::fa_combine_kernel<64><<<blocks, 128, 0, s>>>(o_partial, lse_partial,
-                                                     static_cast<__nv_bfloat16*>(o), lse,
-                                                     static_cast<int>(rows), num_splits);
-  else
-    fa::fa_combine_kernel<128><<<blocks, 128, 0, s>>>(o_partial, lse_partial,
-                                                      static_cast<__nv_bfloat16*>(o), lse,
-                                                      static_cast<int>(rows), num_splits);
+  // programmatic dependent launch: scheduled while the previous kernel (the
+  // split) finishes; the kernel waits for it before reading the partials
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(o);
+  const int nrows = static_cast<int>(rows);
+  const cudaError_t e =
+      d == 64 ? cudaLaunchKernelEx(&cfg, fa::fa_combine_kernel<64>, o_partial, lse_partial, ob, lse,
+                                   nrows, num_splits)
+              : cudaLaunchKernelEx(&cfg, fa::fa_combine_kernel<128>, o_partial, lse_partial, ob,
+                                   lse, nrows, num_splits);
+  if (e != cudaSuccess) return FA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
