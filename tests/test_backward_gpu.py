@@ -172,3 +172,35 @@ def test_gqa_long_dkdv_ctas_order_by_role():
         errs[name] = (float(np.abs(g - want).max()) / max(float(np.abs(want).max()), 1e-30),
                       float(np.linalg.norm(g - want)) / max(float(np.linalg.norm(want)), 1e-30))
     check(errs)
+
+
+def test_inputs_written_just_before_the_call():
+    """The main backward kernel is a programmatic dependent of the D kernel:
+    its K, V, Q and dO loads may start before the D kernel ends, and only its
+    reads of the D kernel's output wait.  Inputs written by a kernel enqueued
+    right before the call (here: dO, o and lse rewritten in place on the same
+    stream, no synchronisation) must still be seen, and a following call's D
+    kernel must not overwrite the workspace under a running main kernel: the
+    result equals a call made after a full synchronisation, bit for bit."""
+    B, Hq, Hkv, S, d = 2, 8, 2, 1000, 128
+    q, k, v = prefill_inputs(B, Hq, Hkv, S, S, d, 91, 1.0)
+    d_o = grad_output((B, Hq, S, d), 91)
+    qc, kc, vc, doc = (t.cuda() for t in (q, k, v, d_o))
+    o = torch.empty_like(qc)
+    lse = torch.empty((B, Hq, S), device="cuda", dtype=torch.float32)
+    fa.fa_fwd(qc, kc, vc, o, lse, True, 0.088)
+    torch.cuda.synchronize()
+    ref = [t.clone() for t in fa.attention_backward(qc, kc, vc, o, lse, doc, True, 0.088)]
+    torch.cuda.synchronize()
+    # scramble the inputs, then restore them with kernels on the compute
+    # stream immediately before each call
+    saved = [t.clone() for t in (o, lse, doc)]
+    for _ in range(3):
+        for t in (o, lse, doc):
+            t.fill_(7.0)
+        for t, s in zip((o, lse, doc), saved):
+            t.copy_(s)
+        got = fa.attention_backward(qc, kc, vc, o, lse, doc, True, 0.088)
+    torch.cuda.synchronize()
+    for a, b in zip(got, ref):
+        assert torch.equal(a, b)

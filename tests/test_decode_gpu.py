@@ -133,3 +133,29 @@ def test_full_size_decode_config_every_sequence():
                                        np.array([L], np.int32), c.scale)
         cmp(o[b:b + 1].float().cpu().numpy(), o_ref, O_TOL, "O b=%d" % b)
         cmp(lse[b:b + 1].cpu().numpy(), lse_ref, LSE_TOL, "LSE b=%d" % b)
+
+
+def test_combine_after_partials_written_just_before():
+    """fa_combine is a programmatic dependent of the kernel before it: it must
+    wait for it before reading the partials.  Partials rewritten in place on
+    the same stream right before the call (no synchronisation) give the
+    synchronised result bit for bit."""
+    g = torch.Generator().manual_seed(5)
+    B, Hq, n, d = 8, 16, 9, 128
+    op = torch.randn(B, Hq, n, d, generator=g).cuda()
+    lp = (torch.randn(B, Hq, n, generator=g) * 5).cuda()
+    o_ref = torch.empty(B, Hq, d, device="cuda", dtype=torch.bfloat16)
+    lse_ref = torch.empty(B, Hq, device="cuda")
+    fa.fa_combine(op, lp, o_ref, lse_ref)
+    torch.cuda.synchronize()
+    saved = (op.clone(), lp.clone())
+    o = torch.empty_like(o_ref)
+    lse = torch.empty_like(lse_ref)
+    for _ in range(3):
+        op.fill_(1.0e6)
+        lp.fill_(100.0)
+        op.copy_(saved[0])
+        lp.copy_(saved[1])
+        fa.fa_combine(op, lp, o, lse)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
